@@ -1,0 +1,304 @@
+"""CPU oracle for the block-scaled (NVFP4 / MXFP8) linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  It shares no code with the CUDA library and never calls it.
+
+The scalar, bit-exact parts (format decoders, round-to-nearest-even encoders,
+the NVFP4 and MXFP8 group quantizers and the 128x4 scale-tile map) are plain C
+in ``bsp_oracle.c``, compiled with gcc and no floating-point contraction.  The
+contraction is a float64 matrix product of the decoded operands (numpy, a
+library matmul used as one step):
+
+    y[m, n] = alpha * row_scale[m] * sum_k decA[m, k] * decB[n, k] + bias[n]
+
+which is the definition of the block-scaled GEMM the pages call
+(``mm_fp4(x_fp4, w_fp4.T, x_scale, w_scale.T, 1/(gs_x*gs_w), bf16)`` followed by
+``out + bias`` in hao-ai-lab-FastVideo nvfp4_qat_config.py,
+``NVFP4QATQuantizeMethod.apply``; the MXFP8 product of vllm-omni
+mxfp8_config.py, ``NPUMxfp8LinearMethod._quant_matmul``, with alpha = 1).
+
+Parity pins for every function live in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bsp_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``bsp_oracle.c`` into ``_build/liboracle.so`` (gcc)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        i64, f32, f64, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_int
+        vp = ctypes.c_void_p
+        L.bspo_bf16_value.restype = f64
+        L.bspo_bf16_value.argtypes = [ctypes.c_uint16]
+        L.bspo_e2m1_value.restype = f64
+        L.bspo_e2m1_value.argtypes = [i32]
+        L.bspo_e4m3_value.restype = f64
+        L.bspo_e4m3_value.argtypes = [i32]
+        L.bspo_e8m0_value.restype = f64
+        L.bspo_e8m0_value.argtypes = [i32]
+        L.bspo_e2m1_encode.restype = i32
+        L.bspo_e2m1_encode.argtypes = [f64]
+        L.bspo_e4m3_encode.restype = i32
+        L.bspo_e4m3_encode.argtypes = [f64]
+        L.bspo_bf16_round.restype = ctypes.c_uint16
+        L.bspo_bf16_round.argtypes = [f64]
+        L.bspo_sf_offset.restype = i64
+        L.bspo_sf_offset.argtypes = [i64, i64, i64]
+        L.bspo_sf_bytes.restype = i64
+        L.bspo_sf_bytes.argtypes = [i64, i64]
+        L.bspo_amax_bf16.restype = f32
+        L.bspo_amax_bf16.argtypes = [vp, i64]
+        L.bspo_nvfp4_global_scale.restype = f32
+        L.bspo_nvfp4_global_scale.argtypes = [f32]
+        L.bspo_row_global_scales.restype = None
+        L.bspo_row_global_scales.argtypes = [vp, i64, i64, i64, vp, vp]
+        L.bspo_nvfp4_quantize_group.restype = None
+        L.bspo_nvfp4_quantize_group.argtypes = [vp, f32, vp, vp]
+        L.bspo_nvfp4_quantize.restype = i32
+        L.bspo_nvfp4_quantize.argtypes = [vp, i64, i64, i64, vp, i32, vp, vp]
+        L.bspo_mxfp8_quantize_group.restype = None
+        L.bspo_mxfp8_quantize_group.argtypes = [vp, vp, vp]
+        L.bspo_mxfp8_quantize.restype = i32
+        L.bspo_mxfp8_quantize.argtypes = [vp, i64, i64, i64, vp, vp]
+        L.bspo_nvfp4_dequantize_rows.restype = None
+        L.bspo_nvfp4_dequantize_rows.argtypes = [vp, vp, i64, vp, i64, vp]
+        L.bspo_mxfp8_dequantize_rows.restype = None
+        L.bspo_mxfp8_dequantize_rows.argtypes = [vp, vp, i64, vp, i64, vp]
+        L.bspo_bf16_round_array.restype = None
+        L.bspo_bf16_round_array.argtypes = [vp, i64, vp]
+        L.bspo_e4m3_encode_array.restype = None
+        L.bspo_e4m3_encode_array.argtypes = [vp, i64, vp]
+        L.bspo_e2m1_encode_array.restype = None
+        L.bspo_e2m1_encode_array.argtypes = [vp, i64, vp]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def _threads(threads):
+    return max(1, threads if threads else (os.cpu_count() or 1))
+
+
+# --------------------------------------------------------------------------- scalars
+def bf16_value(bits: int) -> float:
+    return lib().bspo_bf16_value(int(bits))
+
+
+def e2m1_value(code: int) -> float:
+    return lib().bspo_e2m1_value(int(code))
+
+
+def e4m3_value(byte: int) -> float:
+    return lib().bspo_e4m3_value(int(byte))
+
+
+def e8m0_value(byte: int) -> float:
+    return lib().bspo_e8m0_value(int(byte))
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """e2m1 RNE-satfinite codes (0..15, sign in bit 3) of fp32 values; -1 for NaN."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float32).reshape(-1))
+    out = np.empty(a.size, dtype=np.int8)
+    lib().bspo_e2m1_encode_array(_ptr(a), a.size, _ptr(out))
+    return out.reshape(np.shape(v))
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """e4m3fn RNE-satfinite bytes of fp32 values (NaN -> 0x7F)."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float32).reshape(-1))
+    out = np.empty(a.size, dtype=np.uint8)
+    lib().bspo_e4m3_encode_array(_ptr(a), a.size, _ptr(out))
+    return out.reshape(np.shape(v))
+
+
+def bf16_round(y) -> np.ndarray:
+    """Nearest-even bf16 bit patterns (uint16) of float64 values, rounded once."""
+    a = np.ascontiguousarray(np.asarray(y, dtype=np.float64).reshape(-1))
+    out = np.empty(a.size, dtype=np.uint16)
+    lib().bspo_bf16_round_array(_ptr(a), a.size, _ptr(out))
+    return out.reshape(np.shape(y))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact values of bf16 bit patterns (a bf16 is the top half of an fp32)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def sf_offset(r: int, c: int, cols_padded: int) -> int:
+    return lib().bspo_sf_offset(int(r), int(c), int(cols_padded))
+
+
+def sf_bytes(rows: int, cols: int) -> int:
+    """Bytes of a tile-mapped scale buffer for [rows, cols] scales."""
+    return lib().bspo_sf_bytes(int(rows), int(cols))
+
+
+# --------------------------------------------------------------------------- global scales
+def amax_bf16(x: np.ndarray) -> float:
+    a = np.ascontiguousarray(x, dtype=np.uint16).reshape(-1)
+    return float(np.float32(lib().bspo_amax_bf16(_ptr(a), a.size)))
+
+
+def nvfp4_global_scale(amax: float) -> np.float32:
+    return np.float32(lib().bspo_nvfp4_global_scale(float(np.float32(amax))))
+
+
+def row_global_scales(x: np.ndarray):
+    """Per-row (per-token) encode scales gs[m] and decode factors 1/gs[m] (fp32)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    gs = np.empty(M, np.float32)
+    inv = np.empty(M, np.float32)
+    lib().bspo_row_global_scales(_ptr(x), M, K, K, _ptr(gs), _ptr(inv))
+    return gs, inv
+
+
+# --------------------------------------------------------------------------- quantizers
+def _row_chunks(M: int, threads: int):
+    """Row ranges starting at multiples of 128, so each owns whole scale bands."""
+    per = -(-M // max(1, threads))
+    per = -(-per // 128) * 128
+    return [(m0, min(M, m0 + per)) for m0 in range(0, M, per)]
+
+
+def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None = None):
+    """NVFP4 quantization of bf16 bit patterns ``x`` [M, K] along K.
+
+    Returns (codes uint8 [M, K/2], sf uint8 [sf_bytes(M, K/16)] in the 128x4 map).
+    ``gs`` is one fp32 encode scale, or one per row if ``per_row``.
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    g = np.ascontiguousarray(np.asarray(gs, dtype=np.float32).reshape(-1))
+    if per_row and g.size != M:
+        raise ValueError("per-row scales need one value per row")
+    codes = np.empty((M, K // 2), np.uint8)
+    cols = K // 16
+    cols_p = -(-cols // 4) * 4
+    sf = np.empty(sf_bytes(M, cols), np.uint8)
+    if M == 0:
+        return codes, sf
+    L = lib()
+
+    def run(rng):
+        m0, m1 = rng
+        gp = _ptr(g) + (4 * m0 if per_row else 0)
+        rc = L.bspo_nvfp4_quantize(_ptr(x) + 2 * m0 * K, m1 - m0, K, K, gp, int(per_row),
+                                   _ptr(codes) + m0 * (K // 2), _ptr(sf) + m0 * cols_p)
+        assert rc == 0
+
+    chunks = _row_chunks(M, _threads(threads))
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        list(ex.map(run, chunks))
+    return codes, sf
+
+
+def mxfp8_quantize(x: np.ndarray, threads: int | None = None):
+    """MXFP8 quantization of bf16 bit patterns ``x`` [M, K] (groups of 32 along K).
+
+    Returns (q uint8 e4m3 [M, K], sf uint8 e8m0 [sf_bytes(M, K/32)] in the 128x4 map).
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    q = np.empty((M, K), np.uint8)
+    cols = K // 32
+    cols_p = -(-cols // 4) * 4
+    sf = np.empty(sf_bytes(M, cols), np.uint8)
+    if M == 0:
+        return q, sf
+    L = lib()
+
+    def run(rng):
+        m0, m1 = rng
+        rc = L.bspo_mxfp8_quantize(_ptr(x) + 2 * m0 * K, m1 - m0, K, K,
+                                   _ptr(q) + m0 * K, _ptr(sf) + m0 * cols_p)
+        assert rc == 0
+
+    chunks = _row_chunks(M, _threads(threads))
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        list(ex.map(run, chunks))
+    return q, sf
+
+
+# --------------------------------------------------------------------------- decoders
+def _dequant(fn, codes, sf, K, rows, threads):
+    rows = np.ascontiguousarray(np.arange(codes.shape[0]) if rows is None else rows, dtype=np.int64)
+    out = np.empty((rows.size, K), np.float64)
+    if rows.size == 0:
+        return out
+    codes = np.ascontiguousarray(codes)
+    sf = np.ascontiguousarray(sf)
+    n = _threads(threads)
+    parts = np.array_split(np.arange(rows.size), min(n, rows.size))
+
+    def run(idx):
+        i0 = int(idx[0])
+        fn(_ptr(codes), _ptr(sf), K, _ptr(rows) + 8 * i0, idx.size, _ptr(out) + 8 * K * i0)
+
+    with ThreadPoolExecutor(len(parts)) as ex:
+        list(ex.map(run, parts))
+    return out
+
+
+def nvfp4_dequantize(codes: np.ndarray, sf: np.ndarray, K: int, rows=None, threads=None) -> np.ndarray:
+    """Real values e2m1(code) * e4m3(scale) of the chosen rows, float64 [len(rows), K]."""
+    return _dequant(lib().bspo_nvfp4_dequantize_rows, codes, sf, K, rows, threads)
+
+
+def mxfp8_dequantize(q: np.ndarray, sf: np.ndarray, K: int, rows=None, threads=None) -> np.ndarray:
+    """Real values e4m3(q) * e8m0(scale) of the chosen rows, float64 [len(rows), K]."""
+    return _dequant(lib().bspo_mxfp8_dequantize_rows, q, sf, K, rows, threads)
+
+
+# --------------------------------------------------------------------------- contraction
+def linear_reference(decA: np.ndarray, decB: np.ndarray, alpha: float = 1.0,
+                     row_scale=None, bias=None):
+    """y = alpha * row_scale[m] * (decA @ decB.T) + bias[n] in float64.
+
+    Returns (y, bound) where bound[m, n] = |alpha * row_scale[m]| * sum_k |decA * decB|,
+    the scale of the accumulation-error tolerance.
+    """
+    acc = decA @ decB.T
+    mag = np.abs(decA) @ np.abs(decB).T
+    f = np.float64(np.float32(alpha))
+    if row_scale is not None:
+        f = f * np.asarray(row_scale, dtype=np.float32).astype(np.float64)[:, None]
+    y = f * acc
+    if bias is not None:
+        y = y + bf16_bits_to_f64(bias)[None, :]
+    return y, np.abs(f) * mag
