@@ -1,0 +1,468 @@
+"""Benchmark of the block-scaled linear-layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Default workload (N=1): the Wan-2.1-1.3B-shaped attention projection as an NVFP4
+W4A4 linear layer, A bf16 [32760, 1536] (N(0,1) with 0.1% x50 outliers),
+W [1536, 1536] ~N(0, 1/sqrt(1536)), bias [1536] ~N(0, 0.01), static activation
+scale 1.0; the weight is quantized once before timing (load time).  One step =
+quantize A (NVFP4 kernel) + block-scaled GEMM with alpha and bias fused (tcgen05
+kernel), inputs resident in HBM.  `value` = 2*M*N*K per step / step time
+(TFLOP/s) summed over ranks; L2 is flushed (256 MiB write) before every timed
+step, outside the timed events.
+
+Other --config values (wan14_in, wan14_out, mxfp8, skinny_m<M>, tiny) time the
+corresponding workload the same way.
+
+--impl reference times the CPU oracle (oracle/, plain C + numpy float64) on a
+bounded row sample of the same workload, on the host cores.
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(replicas; the path has no exchange step), timing is the max over ranks, and
+`value` is the total over ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GEMM TFLOP/s & % dense-FP4 peak; quantize GB/s & % HBM (1×B200)"
+FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor rate (9 / 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "block_scaled_precision_05_b200", "csrc")
+    for name in sorted(os.listdir(cdir)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(cdir, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
+    summary, or None when missing or taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {  # nvmlClocksEventReason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+        self._period = period_s
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _handle(self, idx):
+        import torch
+        nv = self._nv
+        try:
+            uuid = str(torch.cuda.get_device_properties(idx).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- workloads
+def make_workload(name: str):
+    from block_scaled_precision_05_b200 import workloads as wl
+    if name == "wan13":
+        return wl.wan13(), "nvfp4"
+    if name == "tiny":
+        return wl.tiny(), "nvfp4"
+    if name in ("wan14_in", "wan14_out"):
+        return getattr(wl, name)(), "nvfp4"
+    if name == "mxfp8":
+        return wl.mxfp8(), "mxfp8"
+    if name.startswith("skinny_m"):
+        return wl.skinny(int(name[len("skinny_m"):])), "nvfp4"
+    raise SystemExit(f"unknown --config {name}")
+
+
+def describe(lin, kind):
+    d = {"workload": f"{lin.name}: {kind.upper()} linear A[{lin.M},{lin.K}] x W[{lin.N},{lin.K}]^T"
+                     + (" + bias" if lin.bias is not None else "")
+                     + (" (per-token activation scales)" if lin.per_token else ""),
+         "M": lin.M, "N": lin.N, "K": lin.K,
+         "l2": "flushed before every timed step (256 MiB write, outside the timed events)"}
+    return d
+
+
+def quant_bytes(M, K, kind):
+    """Algorithmic HBM bytes of one activation quantize launch."""
+    if kind == "nvfp4":
+        return M * K * 2 + M * K // 2 + (-(-M // 128) * 128) * (-(-(K // 16) // 4) * 4)
+    return M * K * 2 + M * K + (-(-M // 128) * 128) * (-(-(K // 32) // 4) * 4)
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from block_scaled_precision_05_b200 import api
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lin, kind = make_workload(args.config)
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    A = up(lin.A)
+    W = up(lin.W)
+    bias = None if lin.bias is None else up(lin.bias)
+    if kind == "nvfp4":
+        layer = api.NVFP4Linear(W, bias, per_token=lin.per_token)
+    else:
+        layer = api.MXFP8Linear(W, bias)
+    del W
+    M, N, K = lin.M, lin.N, lin.K
+    flops = 2.0 * M * N * K
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # preallocated outputs: the timed step launches exactly our two kernels
+    if kind == "nvfp4":
+        xq = api.NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                             torch.empty(api.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+        if lin.per_token:
+            xq.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
+            xq.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
+    else:
+        xq = api.MXFP8Tensor(torch.empty((M, K), dtype=torch.uint8, device=dev),
+                             torch.empty(api.mxfp8_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def quantize():
+        if kind == "nvfp4":
+            api.nvfp4_quantize(A, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=xq)
+        else:
+            api.mxfp8_quantize(A, out=xq)
+
+    def gemm():
+        if kind == "nvfp4":
+            api.nvfp4_gemm(xq, layer.weight, layer.alpha, xq.row_inv_gs if lin.per_token else None, layer.bias,
+                           out=D)
+        else:
+            api.mxfp8_gemm(xq, layer.weight, None, layer.bias, out=D)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        quantize()
+        gemm()
+    torch.cuda.synchronize()
+    if api.device_status() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for s in range(args.steps):
+            flush.zero_()
+            ev[s][0].record(stream)
+            quantize()
+            ev[s][1].record(stream)
+            gemm()
+            ev[s][2].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    t_q = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    t_g = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
+    total_ms = float(sum(t_q) + sum(t_g))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if api.device_status() != 0:
+        raise RuntimeError("device error word set during timing")
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API: pinned host A in, D back to pinned host
+    A_host = torch.from_numpy(np.ascontiguousarray(lin.A).view(np.int16)).view(torch.bfloat16).pin_memory()
+    D_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    A_dev = torch.empty_like(A)
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        A_dev.copy_(A_host, non_blocking=True)
+        y = layer(A_dev)
+        D_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    q_ms = statistics.mean(t_q)
+    g_ms = statistics.mean(t_g)
+    qb = quant_bytes(M, K, kind)
+    q_gbs = qb / (q_ms * 1e-3) / 1e9
+    g_tflops = flops / (g_ms * 1e-3) / 1e12
+    ratio = FP4_PER_BF16 if kind == "nvfp4" else FP8_PER_BF16
+    tensor_peak = peaks["bf16_tflops"] * ratio
+    hbm_peak = peaks["hbm_gbs"]
+    wname = args.config
+    if g_ms >= q_ms:
+        roof = {"kernel": f"{kind}_gemm", "bound": "tensor", "achieved": round(g_tflops, 1),
+                "peak": round(tensor_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / tensor_peak, 4),
+                "traffic": traffic_for(f"{kind}_gemm", wname),
+                "peak_source": f"{peak_src}: bf16_tflops (burst) x {ratio:g} nominal {kind} ratio",
+                "algorithmic": f"2*M*N*K = {flops:.4g} flop per launch"}
+    else:
+        roof = {"kernel": f"{kind}_quantize", "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4), "traffic": traffic_for(f"{kind}_quantize", wname),
+                "peak_source": f"{peak_src}: hbm_gbs", "algorithmic": f"{qb} bytes per launch"}
+
+    cfg = describe(lin, kind)
+    cfg["parallelism"] = f"replicas x{world}"
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4" if kind == "nvfp4" else "mxfp8", "data": "synthetic (seeded numpy)",
+        "config": cfg, "roofline": roof,
+        "kernels": {
+            f"{kind}_quantize": {"ms": round(q_ms, 5), "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / hbm_peak, 4)},
+            f"{kind}_gemm": {"ms": round(g_ms, 5), "TFLOP/s": round(g_tflops, 1),
+                             "frac_tensor_peak": round(g_tflops / tensor_peak, 4)},
+        },
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(A_host.numel() * 2), "d2h_bytes_per_step": int(D_host.numel() * 2),
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_baseline(lin, kind, budget_s=args.cpu_budget)
+    return out
+
+
+# --------------------------------------------------------------------------- oracle arm
+def oracle_step(lin, kind, rows, wq):
+    """The oracle's linear layer on `rows` of A: quantize, decode, float64 GEMM, epilogue."""
+    import oracle
+    K = lin.K
+    A = lin.A[rows]
+    if kind == "nvfp4":
+        gs_w, codes_b, sf_b, decB = wq
+        if lin.per_token:
+            gs, inv = oracle.row_global_scales(A)
+            ca, sa = oracle.nvfp4_quantize(A, gs, per_row=True)
+            alpha, rs = np.float32(1) / gs_w, inv
+        else:
+            ca, sa = oracle.nvfp4_quantize(A, 1.0)
+            alpha, rs = np.float32(1) / (np.float32(1) * gs_w), None
+        decA = oracle.nvfp4_dequantize(ca, sa, K)
+    else:
+        _, _, _, decB = wq
+        qa, sa = oracle.mxfp8_quantize(A)
+        decA = oracle.mxfp8_dequantize(qa, sa, K)
+        alpha, rs = 1.0, None
+    y, _ = oracle.linear_reference(decA, decB, alpha=alpha, row_scale=rs, bias=lin.bias)
+    return oracle.bf16_round(y)
+
+
+def oracle_weights(lin, kind):
+    import oracle
+    if kind == "nvfp4":
+        gs_w = oracle.nvfp4_global_scale(oracle.amax_bf16(lin.W))
+        cb, sb = oracle.nvfp4_quantize(lin.W, gs_w)
+        return gs_w, cb, sb, oracle.nvfp4_dequantize(cb, sb, lin.K)
+    qb, sb = oracle.mxfp8_quantize(lin.W)
+    return None, qb, sb, oracle.mxfp8_dequantize(qb, sb, lin.K)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_baseline(lin, kind, budget_s=10.0):
+    """Times the oracle on a bounded row sample, scaled to TFLOP/s."""
+    wq = oracle_weights(lin, kind)
+    rng = np.random.default_rng(123)
+    rows = np.sort(rng.choice(lin.M, size=min(lin.M, 128), replace=False))
+    t0 = time.perf_counter()
+    oracle_step(lin, kind, rows, wq)
+    dt = time.perf_counter() - t0
+    n = int(min(lin.M, max(128, 128 * budget_s / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(lin.M, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle_step(lin, kind, rows, wq)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * n * lin.N * lin.K
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": max(os.cpu_count() or 1, blas_threads()),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"{n} random rows of A (of {lin.M}): quantize + decode + float64 GEMM + epilogue + bf16 "
+                      f"rounding; weight quantized beforehand (load time)"}
+
+
+def run_reference(args):
+    lin, kind = make_workload(args.config)
+    wq = oracle_weights(lin, kind)
+    rng = np.random.default_rng(7)
+    n = min(lin.M, args.ref_rows)
+    for _ in range(args.warmup):
+        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * n * lin.N * lin.K * args.steps
+    value = flops / dt / 1e12
+    cores = max(os.cpu_count() or 1, blas_threads())
+    sample = (f"{n} random rows of A per step (of {lin.M}): quantize + decode + float64 GEMM + epilogue + bf16 "
+              f"rounding; weight quantized beforehand (load time)")
+    cfg = describe(lin, kind)
+    cfg["parallelism"] = "host cores"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64 (oracle)", "data": "synthetic (seeded numpy)", "config": cfg,
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="wan13")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=256, help="rows per oracle step for --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,264 @@
+"""PyTorch-facing API over the C ABI (include/bsp.h).
+
+PyTorch provides device memory and the current stream; every step of the
+quantize / GEMM path runs in libbsp's CUDA kernels.  Functions here only check
+arguments, allocate outputs and pass pointers.
+
+Sources (page title, then symbol):
+  hao-ai-lab-FastVideo nvfp4_qat_config.py -- NVFP4QATQuantizeMethod.apply
+      (flatten to [-1, K], quantize with the static activation scale 1.0,
+      mm_fp4 with alpha = 1/(gs_x*gs_w), add bias, restore leading dims);
+      convert_model_to_fp4 (weight amax -> gs_w = 448*6/amax -> quantize).
+  hao-ai-lab-FastVideo nvfp4_config.py -- _coerce_fp4_input_dtype (fp32 input
+      is cast to bf16, non-float input is a TypeError), the register_fake
+      shapes of nvfp4_quantize ([M, K/2] codes) and mm_fp4 ([*a.shape[:-1], N]).
+  sglang nvfp4_online.py -- per-token activation scales; the all-zero weight
+      guard (scale 1 when amax is 0); K % 16 == 0 and 2-D weights required.
+  vllm-omni mxfp8_config.py -- MXFPLinearMethodBase.apply (reshape, quantize
+      the activation with one e8m0 scale per 32, GEMM with bias, reshape).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _native as nat
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _require_cuda(*ts: torch.Tensor | None) -> None:
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libbsp runs on CUDA tensors only (no CPU path)")
+
+
+def coerce_input(x: torch.Tensor) -> torch.Tensor:
+    """Activation dtype rule of the pages: bf16 passes, other floats are cast to
+    bf16, anything else is an error."""
+    if not x.is_floating_point():
+        raise TypeError(f"block-scaled linear expects floating-point inputs, got {x.dtype}")
+    return x if x.dtype == torch.bfloat16 else x.to(torch.bfloat16)
+
+
+def nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return int(nat.lib().bsp_nvfp4_sf_bytes(rows, K))
+
+
+def mxfp8_sf_bytes(rows: int, K: int) -> int:
+    return int(nat.lib().bsp_mxfp8_sf_bytes(rows, K))
+
+
+# --------------------------------------------------------------------------- scales
+def amax(x: torch.Tensor) -> torch.Tensor:
+    """fp32 [1] device tensor: max |x| over a bf16 tensor (NaN as 0, inf as bf16 max)."""
+    _require_cuda(x)
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("amax expects a contiguous bf16 tensor")
+    out = torch.empty(1, dtype=torch.float32, device=x.device)
+    nat.check(nat.lib().bsp_amax_bf16(_ptr(x), x.numel(), _ptr(out), _stream()), "bsp_amax_bf16")
+    return out
+
+
+def nvfp4_global_scale(amax_t: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """(gs, 1/gs) fp32 [1] device tensors with gs = 448*6/amax (1 for amax 0)."""
+    _require_cuda(amax_t)
+    gs = torch.empty(1, dtype=torch.float32, device=amax_t.device)
+    inv = torch.empty_like(gs)
+    nat.check(nat.lib().bsp_nvfp4_global_scale(_ptr(amax_t), _ptr(gs), _ptr(inv), _stream()),
+              "bsp_nvfp4_global_scale")
+    return gs, inv
+
+
+def nvfp4_alpha(gs_x: torch.Tensor, gs_w: torch.Tensor) -> torch.Tensor:
+    """alpha = 1/(gs_x * gs_w), fp32 [1] device tensor."""
+    _require_cuda(gs_x, gs_w)
+    out = torch.empty(1, dtype=torch.float32, device=gs_x.device)
+    nat.check(nat.lib().bsp_nvfp4_alpha(_ptr(gs_x), _ptr(gs_w), _ptr(out), _stream()), "bsp_nvfp4_alpha")
+    return out
+
+
+# --------------------------------------------------------------------------- quantize
+@dataclass
+class NVFP4Tensor:
+    """Packed NVFP4 rows: codes uint8 [M, K/2], scales uint8 (128x4 layout)."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    K: int
+    row_gs: torch.Tensor | None = None      # per-row encode scales (PER_ROW)
+    row_inv_gs: torch.Tensor | None = None  # per-row decode factors 1/gs (PER_ROW)
+
+    @property
+    def rows(self) -> int:
+        return self.codes.shape[0]
+
+
+@dataclass
+class MXFP8Tensor:
+    """MXFP8 rows: e4m3 bytes [M, K], e8m0 scales (128x4 layout)."""
+    q: torch.Tensor
+    sf: torch.Tensor
+    K: int
+
+    @property
+    def rows(self) -> int:
+        return self.q.shape[0]
+
+
+def _as_2d(x: torch.Tensor) -> torch.Tensor:
+    x2 = x.reshape(-1, x.shape[-1])
+    if x2.stride(-1) != 1:
+        x2 = x2.contiguous()
+    return x2
+
+
+def nvfp4_quantize(x: torch.Tensor, global_sf: torch.Tensor | None = None, per_row: bool = False,
+                   out: NVFP4Tensor | None = None) -> NVFP4Tensor:
+    """Quantize bf16 [..., K] to NVFP4 along K (leading dims flattened)."""
+    _require_cuda(x, global_sf)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("nvfp4_quantize expects bf16 input (use coerce_input first)")
+    x2 = _as_2d(x)
+    M, K = x2.shape
+    dev = x2.device
+    if out is None:
+        out = NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+        if per_row:
+            out.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
+            out.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
+    if not per_row and global_sf is None:
+        raise ValueError("per-tensor quantization needs global_sf (fp32 device tensor)")
+    st = nat.lib().nvfp4_quantize(
+        _ptr(x2), M, K, x2.stride(0), None if per_row else _ptr(global_sf),
+        nat.BSP_SF_PER_ROW if per_row else nat.BSP_SF_PER_TENSOR,
+        _ptr(out.row_gs) if per_row else None, _ptr(out.row_inv_gs) if per_row else None,
+        _ptr(out.codes), _ptr(out.sf), _stream())
+    nat.check(st, "nvfp4_quantize")
+    return out
+
+
+def mxfp8_quantize(x: torch.Tensor, out: MXFP8Tensor | None = None) -> MXFP8Tensor:
+    """Quantize bf16 [..., K] to MXFP8 along K (leading dims flattened)."""
+    _require_cuda(x)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("mxfp8_quantize expects bf16 input (use coerce_input first)")
+    x2 = _as_2d(x)
+    M, K = x2.shape
+    dev = x2.device
+    if out is None:
+        out = MXFP8Tensor(torch.empty((M, K), dtype=torch.uint8, device=dev),
+                          torch.empty(mxfp8_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+    nat.check(nat.lib().mxfp8_quantize(_ptr(x2), M, K, x2.stride(0), _ptr(out.q), _ptr(out.sf), _stream()),
+              "mxfp8_quantize")
+    return out
+
+
+# --------------------------------------------------------------------------- GEMM
+def _out(M: int, N: int, dtype: torch.dtype, device, out: torch.Tensor | None) -> tuple[torch.Tensor, int]:
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("output dtype must be bf16 or fp32")
+    if out is None:
+        out = torch.empty((M, N), dtype=dtype, device=device)
+    if out.dtype != dtype or out.dim() != 2 or out.shape[0] != M or out.shape[1] != N or out.stride(1) != 1:
+        raise ValueError("out must be a row-major [M, N] tensor of the output dtype")
+    return out, (nat.BSP_OUT_F32 if dtype == torch.float32 else nat.BSP_OUT_BF16)
+
+
+def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, alpha: torch.Tensor | None = None,
+               row_scale: torch.Tensor | None = None, bias: torch.Tensor | None = None,
+               out_dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """D = alpha * row_scale[m] * (A (x) sfA)(B (x) sfB)^T + bias, fp32 accumulate."""
+    if a.K != b.K:
+        raise ValueError("A and B disagree on K")
+    _require_cuda(a.codes, b.codes, alpha, row_scale, bias)
+    M, N = a.rows, b.rows
+    out, d_dtype = _out(M, N, out_dtype, a.codes.device, out)
+    st = nat.lib().nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, a.K,
+                              _ptr(alpha), _ptr(row_scale), _ptr(bias), _ptr(out), d_dtype, out.stride(0),
+                              _stream())
+    nat.check(st, "nvfp4_gemm")
+    return out
+
+
+def mxfp8_gemm(a: MXFP8Tensor, b: MXFP8Tensor, alpha: torch.Tensor | None = None,
+               bias: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    """D = alpha * (A (x) 2^sA)(B (x) 2^sB)^T + bias, fp32 accumulate."""
+    if a.K != b.K:
+        raise ValueError("A and B disagree on K")
+    _require_cuda(a.q, b.q, alpha, bias)
+    M, N = a.rows, b.rows
+    out, d_dtype = _out(M, N, out_dtype, a.q.device, out)
+    st = nat.lib().mxfp8_gemm(_ptr(a.q), _ptr(a.sf), _ptr(b.q), _ptr(b.sf), M, N, a.K, _ptr(alpha), _ptr(bias),
+                              _ptr(out), d_dtype, out.stride(0), _stream())
+    nat.check(st, "mxfp8_gemm")
+    return out
+
+
+def device_status() -> int:
+    """Synchronise the current stream and read/clear the device error word."""
+    return int(nat.lib().bsp_device_status(_stream()))
+
+
+# --------------------------------------------------------------------------- linear layers
+class NVFP4Linear:
+    """W4A4 NVFP4 linear layer: the weight is quantized once at construction
+    (amax -> gs_w -> quantize; the bf16 weight is not kept), each call quantizes
+    the activation and runs the block-scaled GEMM with alpha and bias fused.
+
+    per_token=False: static activation scale gs_x = 1.0 (no reduction, no host
+    sync, capturable in a CUDA graph).  per_token=True: per-row activation
+    scales computed inside the quantize kernel and applied in the GEMM epilogue.
+    """
+
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None, per_token: bool = False):
+        if weight.dim() != 2:
+            raise ValueError(f"expects a 2-D weight, got shape {tuple(weight.shape)}")
+        if weight.shape[1] % 16 != 0:
+            raise ValueError(f"K must be a multiple of 16, got shape {tuple(weight.shape)}")
+        w = coerce_input(weight).contiguous()
+        self.out_features, self.in_features = w.shape
+        self.per_token = per_token
+        self.gs_w, self.inv_gs_w = nvfp4_global_scale(amax(w))
+        self.weight = nvfp4_quantize(w, self.gs_w)
+        self.gs_x = torch.ones(1, dtype=torch.float32, device=w.device)
+        # per-token: the GEMM applies 1/gs_w here and 1/gs_x[m] as the row scale
+        self.alpha = self.inv_gs_w if per_token else nvfp4_alpha(self.gs_x, self.gs_w)
+        self.bias = None if bias is None else coerce_input(bias).contiguous()
+
+    def quantize_input(self, x: torch.Tensor) -> NVFP4Tensor:
+        x = coerce_input(x)
+        return nvfp4_quantize(x, None if self.per_token else self.gs_x, per_row=self.per_token)
+
+    def __call__(self, x: torch.Tensor, pre_quantized: NVFP4Tensor | None = None,
+                 out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+        lead = x.shape[:-1]
+        xq = pre_quantized if pre_quantized is not None else self.quantize_input(x)
+        y = nvfp4_gemm(xq, self.weight, self.alpha, xq.row_inv_gs if self.per_token else None, self.bias,
+                       out_dtype=out_dtype)
+        return y.view(*lead, self.out_features)
+
+
+class MXFP8Linear:
+    """W8A8 MXFP8 linear layer (weight quantized once; activation per call)."""
+
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None):
+        if weight.dim() != 2 or weight.shape[1] % 32 != 0:
+            raise ValueError(f"expects a 2-D weight with K % 32 == 0, got {tuple(weight.shape)}")
+        w = coerce_input(weight).contiguous()
+        self.out_features, self.in_features = w.shape
+        self.weight = mxfp8_quantize(w)
+        self.bias = None if bias is None else coerce_input(bias).contiguous()
+
+    def __call__(self, x: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+        lead = x.shape[:-1]
+        xq = mxfp8_quantize(coerce_input(x))
+        return mxfp8_gemm(xq, self.weight, None, self.bias, out_dtype=out_dtype).view(*lead, self.out_features)

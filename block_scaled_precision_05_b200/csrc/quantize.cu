@@ -1,0 +1,486 @@
+// quantize.cu -- bf16 -> NVFP4 / MXFP8 block quantization, global scales, and
+// the diagnostic entry points.
+//
+// NVFP4 (hao-ai-lab-FastVideo nvfp4_config.py, module docstring: e2m1
+// elements, group size 16, e4m3 scale per group, fp32 global scale,
+// layout_128x4), per group of 16 along K:
+//   amax = max|x|;  s = fl32(fl32(amax/6) * gs);  sfb = e4m3_rne_sat(s)
+//   inv = sfb ? fl32(gs / value(sfb)) : 0;  code_i = e2m1_rne_sat(fl32(x_i*inv))
+// MXFP8 (vllm-omni mxfp8_config.py, DiffusionMXFP8Config: 32 elements per
+// float8_e8m0fnu scale, e4m3 elements, OCP MX), per group of 32:
+//   e = clamp(floor(log2 amax) - 8, -127, 127);  sfb = e + 127;
+//   q_i = e4m3_rne_sat(x_i * 2^-e)
+// Scale bytes go straight to the 128x4 tile layout:
+//   ((r/128)*(cols4/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4
+//
+// HBM-bound streaming kernels.  Fast paths (K % 64 == 0 for NVFP4, K % 128 ==
+// 0 for MXFP8): one warp per row, every lane one 16-byte bf16 load per step
+// (a warp step reads 512 contiguous bytes), group amax by warp shuffles in the
+// integer domain (|bf16| bit patterns order like their values), hardware cvt
+// with round-to-nearest-even and saturation, 4-byte code stores, and the four
+// scale bytes of a 128x4 tile row gathered by shuffles into one 4-byte store.
+#include "bsp_device.cuh"
+#include "bsp_internal.h"
+
+namespace bsp {
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kUnroll = 4;
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+__device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// |x| bit pattern of a bf16 for the amax reductions: NaN counts as 0 and
+// +-inf as the largest finite bf16 (x.abs().nan_to_num()).
+__device__ __forceinline__ uint32_t sane_mag(uint32_t b16) {
+  uint32_t m = b16 & 0x7FFFu;
+  if (m > 0x7F80u) return 0u;
+  if (m == 0x7F80u) return 0x7F7Fu;
+  return m;
+}
+
+__device__ __forceinline__ uint32_t max_mag8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  return m;
+}
+
+__device__ __forceinline__ uint32_t max_sane_mag8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(sane_mag(w[i] & 0xFFFFu), sane_mag(w[i] >> 16)));
+  return m;
+}
+
+__device__ __forceinline__ uint32_t warp_max(uint32_t m) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+  return m;
+}
+
+// gs = amax > 0 ? fl32(2688 / amax) : 1, from a sanitized |bf16| bit pattern.
+__device__ __forceinline__ float global_scale_from_mag(uint32_t mag) {
+  return mag == 0u ? 1.0f : __fdiv_rn(2688.0f, bf16_bits_to_f32(mag));
+}
+
+// NVFP4 scale byte and reciprocal of one group with amax bit pattern `mag`.
+__device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sfb, float& inv) {
+  const float amax = bf16_bits_to_f32(mag);
+  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+  sfb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
+  inv = (sfb == 0u) ? 0.0f : __fdiv_rn(gs, e4m3_pos_to_f32(sfb));
+}
+
+// Eight bf16 (one 16-byte chunk) times inv -> eight e2m1 codes in one word.
+__device__ __forceinline__ uint32_t nvfp4_codes8(const uint4& v, float inv) {
+  return cvt_e2m1x8(__fmul_rn(bf16_bits_to_f32(v.x & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.x >> 16), inv),
+                    __fmul_rn(bf16_bits_to_f32(v.y & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.y >> 16), inv),
+                    __fmul_rn(bf16_bits_to_f32(v.z & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.z >> 16), inv),
+                    __fmul_rn(bf16_bits_to_f32(v.w & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.w >> 16), inv));
+}
+
+// Byte offset of the first of the four scale bytes (r, 4*tile_col .. +3).
+__device__ __forceinline__ int64_t sf_row_base(int64_t r, int64_t tiles_per_band) {
+  return (r >> 7) * tiles_per_band * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+}
+
+// Per-row encode scale of row r (warp-cooperative); lane 0 stores gs and 1/gs.
+__device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row, int64_t K, int64_t r,
+                                                float* row_gs, float* row_inv) {
+  const uint32_t lane = lane_id();
+  uint32_t m = 0;
+  for (int64_t c = lane * 8; c < K; c += 256) m = max(m, max_sane_mag8(ldg16(row + c)));
+  m = warp_max(m);
+  const float gs = global_scale_from_mag(m);
+  if (lane == 0) {
+    if (row_gs) row_gs[r] = gs;
+    if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
+  }
+  return gs;
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4, K % 64 == 0.  Rows [M, Mp) are the scale padding (zeros).
+// A "quad" is 64 elements = one 128x4 tile row = 8 lanes; a warp step is 4 quads.
+// ---------------------------------------------------------------------------
+template <bool kPerRow>
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
+    float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  const uint32_t lane = lane_id();
+  const uint32_t sub = lane >> 3, j = lane & 7u;
+  const int64_t quads = K >> 6;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+
+  for (int64_t r = warp; r < Mp; r += nwarps) {
+    const bool live = r < M;
+    const uint16_t* row = x + r * ld_x;
+    float gs = gs_tensor;
+    if (kPerRow && live) gs = row_scale_pass(row, K, r, row_gs, row_inv);
+    uint8_t* crow = codes + r * (K >> 1);
+    const int64_t sfb_row = sf_row_base(r, quads);
+
+    for (int64_t q0 = 0; q0 < quads; q0 += 4 * kUnroll) {
+      uint4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t q = q0 + 4 * u + sub;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (live && q < quads) v[u] = ldg16(row + q * 64 + j * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t q = q0 + 4 * u + sub;
+        uint32_t mag = max_mag8(v[u]);
+        mag = max(mag, __shfl_xor_sync(kFull, mag, 1));  // lanes 2g, 2g+1 hold group g
+        uint32_t sfb;
+        float inv;
+        nvfp4_scale(mag, gs, sfb, inv);
+        const uint32_t word = nvfp4_codes8(v[u], inv);
+        const uint32_t s1 = __shfl_down_sync(kFull, sfb, 2);
+        const uint32_t s2 = __shfl_down_sync(kFull, sfb, 4);
+        const uint32_t s3 = __shfl_down_sync(kFull, sfb, 6);
+        if (q < quads) {
+          if (live) *reinterpret_cast<uint32_t*>(crow + q * 32 + j * 4) = word;
+          if (j == 0)
+            *reinterpret_cast<uint32_t*>(sf + sfb_row + q * 512) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4, any K % 16 == 0: one warp per row, one lane per group of 16.
+// ---------------------------------------------------------------------------
+template <bool kPerRow>
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
+    float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  const uint32_t lane = lane_id();
+  const int64_t groups = K >> 4, cols4 = (groups + 3) & ~int64_t(3);
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+
+  for (int64_t r = warp; r < Mp; r += nwarps) {
+    const bool live = r < M;
+    const uint16_t* row = x + r * ld_x;
+    float gs = gs_tensor;
+    if (kPerRow && live) gs = row_scale_pass(row, K, r, row_gs, row_inv);
+    const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
+    for (int64_t c = lane; c < cols4; c += 32) {
+      uint32_t sfb = 0;
+      if (live && c < groups) {
+        const uint4 a = ldg16(row + c * 16), b = ldg16(row + c * 16 + 8);
+        float inv;
+        nvfp4_scale(max(max_mag8(a), max_mag8(b)), gs, sfb, inv);
+        uint2 w;
+        w.x = nvfp4_codes8(a, inv);
+        w.y = nvfp4_codes8(b, inv);
+        *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
+      }
+      sf[sfb_row + (c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfb);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8.
+// ---------------------------------------------------------------------------
+// Scale exponent e (and the multiplier 2^-e) of a group with |amax| bits `mag`.
+__device__ __forceinline__ void mx_scale(uint32_t mag, uint32_t& sfb, float& mul) {
+  int E;
+  if (mag >= 0x80u)
+    E = static_cast<int>(mag >> 7) - 127;                       // normal: exponent field
+  else if (mag != 0u)
+    E = (31 - __clz(static_cast<int>(mag))) - 133;              // subnormal: m * 2^-133
+  else
+    E = -100000;                                                // amax 0: log2 = -inf
+  int e = E - 8;                                                // 8: exponent of 448, the e4m3 max
+  e = e < -127 ? -127 : (e > 127 ? 127 : e);
+  sfb = static_cast<uint32_t>(e + 127);
+  mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, exact (e <= 119 for finite bf16)
+}
+
+__device__ __forceinline__ uint2 mx_elems8(const uint4& v, float mul) {
+  uint2 o;
+  o.x = cvt_e4m3x2(__fmul_rn(bf16_bits_to_f32(v.x & 0xFFFFu), mul), __fmul_rn(bf16_bits_to_f32(v.x >> 16), mul)) |
+        (cvt_e4m3x2(__fmul_rn(bf16_bits_to_f32(v.y & 0xFFFFu), mul), __fmul_rn(bf16_bits_to_f32(v.y >> 16), mul))
+         << 16);
+  o.y = cvt_e4m3x2(__fmul_rn(bf16_bits_to_f32(v.z & 0xFFFFu), mul), __fmul_rn(bf16_bits_to_f32(v.z >> 16), mul)) |
+        (cvt_e4m3x2(__fmul_rn(bf16_bits_to_f32(v.w & 0xFFFFu), mul), __fmul_rn(bf16_bits_to_f32(v.w >> 16), mul))
+         << 16);
+  return o;
+}
+
+// K % 128 == 0: a quad is 128 elements (4 groups of 32, one 128x4 tile row) =
+// 16 lanes; a warp step is 2 quads.
+__global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_k128_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                                          int64_t Mp, int64_t K, int64_t ld_x,
+                                                                          uint8_t* __restrict__ q,
+                                                                          uint8_t* __restrict__ sf) {
+  const uint32_t lane = lane_id();
+  const uint32_t sub = lane >> 4, j = lane & 15u;
+  const int64_t quads = K >> 7;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t r = warp; r < Mp; r += nwarps) {
+    const bool live = r < M;
+    const uint16_t* row = x + r * ld_x;
+    uint8_t* qrow = q + r * K;
+    const int64_t sfb_row = sf_row_base(r, quads);
+    for (int64_t q0 = 0; q0 < quads; q0 += 2 * kUnroll) {
+      uint4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t qq = q0 + 2 * u + sub;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (live && qq < quads) v[u] = ldg16(row + qq * 128 + j * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t qq = q0 + 2 * u + sub;
+        uint32_t mag = max_mag8(v[u]);
+        mag = max(mag, __shfl_xor_sync(kFull, mag, 1));
+        mag = max(mag, __shfl_xor_sync(kFull, mag, 2));  // lanes 4g..4g+3 hold group g
+        uint32_t sfb;
+        float mul;
+        mx_scale(mag, sfb, mul);
+        const uint2 o = mx_elems8(v[u], mul);
+        const uint32_t s1 = __shfl_down_sync(kFull, sfb, 4);
+        const uint32_t s2 = __shfl_down_sync(kFull, sfb, 8);
+        const uint32_t s3 = __shfl_down_sync(kFull, sfb, 12);
+        if (qq < quads) {
+          if (live) *reinterpret_cast<uint2*>(qrow + qq * 128 + j * 8) = o;
+          if (j == 0)
+            *reinterpret_cast<uint32_t*>(sf + sfb_row + qq * 512) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+      }
+    }
+  }
+}
+
+// Any K % 32 == 0: one warp per row, one lane per group of 32.
+__global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_generic_kernel(const uint16_t* __restrict__ x,
+                                                                             int64_t M, int64_t Mp, int64_t K,
+                                                                             int64_t ld_x, uint8_t* __restrict__ q,
+                                                                             uint8_t* __restrict__ sf) {
+  const uint32_t lane = lane_id();
+  const int64_t groups = K >> 5, cols4 = (groups + 3) & ~int64_t(3);
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = warp; r < Mp; r += nwarps) {
+    const bool live = r < M;
+    const uint16_t* row = x + r * ld_x;
+    const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
+    for (int64_t c = lane; c < cols4; c += 32) {
+      uint32_t sfb = 0;
+      if (live && c < groups) {
+        uint4 v[4];
+        uint32_t mag = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[i] = ldg16(row + c * 32 + i * 8);
+          mag = max(mag, max_mag8(v[i]));
+        }
+        float mul;
+        mx_scale(mag, sfb, mul);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2*>(q + r * K + c * 32 + i * 8) = mx_elems8(v[i], mul);
+      }
+      sf[sfb_row + (c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfb);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Global scales.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQuantThreads) amax_bf16_kernel(const uint16_t* __restrict__ x, int64_t n,
+                                                                   uint32_t* __restrict__ amax_bits) {
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t nvec = n >> 3;
+  uint32_t m = 0;
+  for (int64_t i = tid; i < nvec; i += nthreads) m = max(m, max_sane_mag8(ldg16(x + i * 8)));
+  for (int64_t i = (nvec << 3) + tid; i < n; i += nthreads) m = max(m, sane_mag(x[i]));
+  m = warp_max(m);
+  __shared__ uint32_t red[kQuantThreads / 32];
+  if (lane_id() == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0u;
+    m = warp_max(m);
+    // |bf16| << 16 is a non-negative fp32 bit pattern: integer order == value order.
+    if (threadIdx.x == 0 && m != 0u) atomicMax(amax_bits, m << 16);
+  }
+}
+
+__global__ void global_scale_kernel(const float* __restrict__ amax, float* gs, float* inv_gs) {
+  const float a = *amax;
+  const float g = (a > 0.0f) ? __fdiv_rn(2688.0f, a) : 1.0f;
+  if (gs) *gs = g;
+  if (inv_gs) *inv_gs = __fdiv_rn(1.0f, g);
+}
+
+__global__ void alpha_kernel(const float* __restrict__ gs_x, const float* __restrict__ gs_w, float* alpha) {
+  *alpha = __fdiv_rn(1.0f, __fmul_rn(*gs_x, *gs_w));
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostics.
+// ---------------------------------------------------------------------------
+__global__ void debug_e2m1_kernel(const float* __restrict__ v, int64_t n, uint8_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = static_cast<uint8_t>(cvt_e2m1x8(v[i], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xFu);
+}
+
+__global__ void debug_e4m3_kernel(const float* __restrict__ v, int64_t n, uint8_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = static_cast<uint8_t>(cvt_e4m3x2(v[i], 0.f) & 0xFFu);
+}
+
+__global__ void debug_wait_kernel(uint64_t limit_ns, uint32_t* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, nullptr, limit_ns)) raise_error(err, kErrTimeout);
+}
+
+int grid_for_rows(const DeviceInfo& dev, int64_t rows) {
+  const int64_t warps_per_block = kQuantThreads / 32;
+  int64_t blocks = ceil_div(rows, warps_per_block);
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;  // 8 blocks of 256 threads per SM
+  return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+}  // namespace
+}  // namespace bsp
+
+using namespace bsp;
+
+extern "C" {
+
+int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
+                   float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K) return BSP_ERR_INVALID_ARG;
+  if (sf_mode != BSP_SF_PER_TENSOR && sf_mode != BSP_SF_PER_ROW) return BSP_ERR_INVALID_ARG;
+  if (M == 0) return BSP_OK;
+  if (!x || !codes || !sf || (sf_mode == BSP_SF_PER_TENSOR && !global_sf)) return BSP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || ld_x % 8 != 0) return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  const int64_t Mp = round_up(M, 128);
+  const int grid = grid_for_rows(dev, Mp);
+  const bool per_row = sf_mode == BSP_SF_PER_ROW;
+  if (K % 64 == 0) {
+    if (per_row)
+      nvfp4_quant_k64_kernel<true><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs,
+                                                                       row_inv_gs, codes, sf);
+    else
+      nvfp4_quant_k64_kernel<false><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr,
+                                                                        nullptr, codes, sf);
+  } else {
+    if (per_row)
+      nvfp4_quant_generic_kernel<true><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs,
+                                                                           row_inv_gs, codes, sf);
+    else
+      nvfp4_quant_generic_kernel<false><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr,
+                                                                            nullptr, codes, sf);
+  }
+  return launch_status();
+}
+
+int mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, uint8_t* q, uint8_t* sf,
+                   bsp_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 32 != 0 || ld_x < K) return BSP_ERR_INVALID_ARG;
+  if (M == 0) return BSP_OK;
+  if (!x || !q || !sf) return BSP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || ld_x % 8 != 0) return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  const int64_t Mp = round_up(M, 128);
+  const int grid = grid_for_rows(dev, Mp);
+  if (K % 128 == 0)
+    mxfp8_quant_k128_kernel<<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, q, sf);
+  else
+    mxfp8_quant_generic_kernel<<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, q, sf);
+  return launch_status();
+}
+
+int bsp_amax_bf16(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
+  if (n < 0 || !amax || (n > 0 && !x)) return BSP_ERR_INVALID_ARG;
+  if ((x && !aligned16(x)) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  if (cudaMemsetAsync(amax, 0, sizeof(float), stream) != cudaSuccess) return launch_status();
+  if (n == 0) return BSP_OK;
+  int64_t blocks = ceil_div(ceil_div(n, 8), kQuantThreads);
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  amax_bf16_kernel<<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(x, n, reinterpret_cast<uint32_t*>(amax));
+  return launch_status();
+}
+
+int bsp_nvfp4_global_scale(const float* amax, float* gs, float* inv_gs, bsp_stream_t stream) {
+  if (!amax || (!gs && !inv_gs)) return BSP_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  global_scale_kernel<<<1, 1, 0, stream>>>(amax, gs, inv_gs);
+  return launch_status();
+}
+
+int bsp_nvfp4_alpha(const float* gs_x, const float* gs_w, float* alpha, bsp_stream_t stream) {
+  if (!gs_x || !gs_w || !alpha) return BSP_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  alpha_kernel<<<1, 1, 0, stream>>>(gs_x, gs_w, alpha);
+  return launch_status();
+}
+
+int bsp_debug_encode_e2m1(const float* v, int64_t n, uint8_t* codes, bsp_stream_t stream) {
+  if (n < 0 || (n > 0 && (!v || !codes))) return BSP_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  if (n == 0) return BSP_OK;
+  debug_e2m1_kernel<<<static_cast<int>(ceil_div(n, 256)), 256, 0, stream>>>(v, n, codes);
+  return launch_status();
+}
+
+int bsp_debug_encode_e4m3(const float* v, int64_t n, uint8_t* bytes, bsp_stream_t stream) {
+  if (n < 0 || (n > 0 && (!v || !bytes))) return BSP_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  if (n == 0) return BSP_OK;
+  debug_e4m3_kernel<<<static_cast<int>(ceil_div(n, 256)), 256, 0, stream>>>(v, n, bytes);
+  return launch_status();
+}
+
+int bsp_debug_wait_timeout(int64_t limit_ns, bsp_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return BSP_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  debug_wait_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_ns), dev.err_word);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,224 @@
+/*
+ * bsp.h -- C ABI of libbsp: block-scaled (NVFP4 W4A4 / MXFP8 W8A8) linear
+ * layers on NVIDIA B200 (sm_100a).
+ *
+ * The library is the hot path of a quantized linear layer:
+ *
+ *   codes, scales = quantize(x)                     (bf16 -> block-scaled)
+ *   D = alpha * (A (x) sfA) (B (x) sfB)^T + bias     (tensor cores, fp32 accumulate)
+ *
+ * Sources (page title, then the symbol or section on it):
+ *   hao-ai-lab-FastVideo  fastvideo/layers/quantization/nvfp4_qat_config.py
+ *       NVFP4QATQuantizeMethod.apply, convert_model_to_fp4
+ *   hao-ai-lab-FastVideo  fastvideo/layers/quantization/nvfp4_config.py
+ *       module docstring, _nvfp4_quantize, _mm_fp4, the fastvideo_fp4 custom
+ *       ops and their register_fake shape functions, NVFP4QuantizeMethod.apply
+ *   sgl-project sglang    python/sglang/srt/layers/quantization/nvfp4_online.py
+ *       ModelOptNvFp4OnlineFusedMoEMethod._quantize_weight_nvfp4,
+ *       NvFp4OnlineConfig (per-token activation scales)
+ *   vllm-omni             vllm_omni/quantization/mxfp8_config.py
+ *       DiffusionMXFP8Config, NPUMxfp8LinearMethod._quant_matmul
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless stated; the caller
+ *     allocates and owns every buffer.  The library never allocates, frees,
+ *     synchronises, or reads device memory from the host (except
+ *     bsp_device_status, which exists to do exactly that).  Calls are
+ *     asynchronous on `stream` (NULL = the legacy default stream).
+ *   - bf16 tensors are passed as `const uint16_t*` (their bit patterns).
+ *   - Matrices are row-major; `ld_*` is the row stride in ELEMENTS.
+ *   - Return value: a bsp_status.  Arguments are checked on the host first;
+ *     a non-zero status means nothing was launched.
+ *   - The current CUDA device must be an sm_100 GPU (B200/GB200), else
+ *     BSP_ERR_UNSUPPORTED_DEVICE.  (The pages gate NVFP4 on compute
+ *     capability 100: NVFP4QATConfig.get_min_capability.)
+ *   - Kernels bound every wait on the GPU.  A wait that runs out sets a
+ *     device error word instead of hanging; bsp_device_status reports it.
+ */
+#ifndef BSP_H
+#define BSP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (pointer to the runtime's opaque stream). */
+typedef struct CUstream_st *bsp_stream_t;
+
+typedef enum {
+    BSP_OK = 0,
+    BSP_ERR_INVALID_ARG = 1,        /* a size, mode or pointer argument is not allowed */
+    BSP_ERR_ALIGNMENT = 2,          /* a pointer or leading dimension is misaligned */
+    BSP_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 */
+    BSP_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    BSP_ERR_TIMEOUT = 5             /* a bounded wait on the GPU ran out (bsp_device_status) */
+} bsp_status;
+
+/* Scale modes of nvfp4_quantize. */
+enum {
+    BSP_SF_PER_TENSOR = 0, /* one fp32 encode scale for the whole tensor */
+    BSP_SF_PER_ROW = 1     /* one fp32 encode scale per row, computed in-kernel */
+};
+
+/* Output element types of the GEMMs. */
+enum {
+    BSP_OUT_BF16 = 0,
+    BSP_OUT_F32 = 1
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bsp_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int bsp_version(void);
+
+/* ------------------------------------------------------------------------
+ * Scale-factor buffer sizes.
+ * Scales are stored in the 128x4 tile layout the pages name ("layout_128x4
+ * scale layout", nvfp4_config.py module docstring; _nvfp4_quantize pads rows
+ * to 128 for it).  Logical scale (r, c) of a [rows, cols] scale matrix lives at
+ *   ((r/128) * (cols4/4) + c/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4
+ * with cols4 = cols rounded up to a multiple of 4; padding bytes are 0.
+ * The buffer holds round_up(rows,128) * round_up(cols,4) bytes.
+ * ---------------------------------------------------------------------- */
+
+/* NVFP4: cols = K/16 (one e4m3 scale per 16 elements).  0 if K % 16 != 0. */
+size_t bsp_nvfp4_sf_bytes(int64_t rows, int64_t K);
+/* MXFP8: cols = K/32 (one e8m0 scale per 32 elements).  0 if K % 32 != 0. */
+size_t bsp_mxfp8_sf_bytes(int64_t rows, int64_t K);
+
+/* ------------------------------------------------------------------------
+ * Global (per-tensor) scales.
+ * ---------------------------------------------------------------------- */
+
+/* amax = max |x_i| over n bf16 values, as the weight conversion computes it
+ * (x.abs().nan_to_num().amax(): NaN counts as 0, +-inf as the largest finite
+ * bf16).  nvfp4_qat_config.py, convert_model_to_fp4.
+ *   x     : bf16 [n], 16-byte aligned
+ *   amax  : fp32 [1], overwritten (the call zeroes it, then reduces into it)
+ * Errors: n < 0 -> INVALID_ARG; misaligned x -> ALIGNMENT. */
+int bsp_amax_bf16(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream);
+
+/* NVFP4 encode scale from an amax, on the device (no host sync):
+ *   gs = amax > 0 ? fl32(448*6 / amax) : 1.0     (convert_model_to_fp4; the
+ *        all-zero guard is nvfp4_online.py _quantize_weight_nvfp4)
+ *   inv_gs = fl32(1 / gs)                         (the decode scale)
+ * amax, gs, inv_gs: fp32 [1].  gs or inv_gs may be NULL. */
+int bsp_nvfp4_global_scale(const float *amax, float *gs, float *inv_gs, bsp_stream_t stream);
+
+/* alpha = fl32(1 / fl32(gs_x * gs_w)), the GEMM output scale of
+ * NVFP4QATQuantizeMethod.apply.  All fp32 [1]. */
+int bsp_nvfp4_alpha(const float *gs_x, const float *gs_w, float *alpha, bsp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * NVFP4 quantization (nvfp4_config.py: fastvideo_fp4::nvfp4_quantize and
+ * _nvfp4_quantize; module docstring: e2m1 elements, group size 16, e4m3
+ * scales, fp32 global scale, layout_128x4).
+ *
+ * Per row m and group g of 16 consecutive elements along K:
+ *   amax = max |x|;  s = fl32(fl32(amax / 6) * gs);  sfb = e4m3_rne_sat(s)
+ *   inv  = sfb == 0 ? 0 : fl32(gs / value(sfb))
+ *   code_i = e2m1_rne_sat(fl32(x_i * inv))  (sign kept)
+ *
+ *   x        : bf16 [M, K], row stride ld_x >= K elements; 16-byte aligned,
+ *              ld_x % 8 == 0
+ *   global_sf: PER_TENSOR -- fp32 [1], the encode scale gs (the caller passes
+ *              it, so there is no hidden reduction or host sync; activations
+ *              use a static 1.0 as NVFP4QATQuantizeMethod.__init__ does).
+ *              PER_ROW -- ignored (may be NULL).
+ *   sf_mode  : BSP_SF_PER_TENSOR or BSP_SF_PER_ROW.  PER_ROW computes
+ *              gs[m] = amax(row m) > 0 ? fl32(448*6/amax) : 1 in-kernel (the
+ *              dynamic per-token activation scales of nvfp4_online.py,
+ *              NvFp4OnlineConfig.use_per_token_activation).
+ *   row_gs   : PER_ROW: fp32 [M] receives gs[m] (may be NULL); else unused.
+ *   row_inv_gs: PER_ROW: fp32 [M] receives fl32(1/gs[m]), the per-row factor
+ *              nvfp4_gemm takes as row_scale (may be NULL); else unused.
+ *   codes    : uint8 [M, K/2] (dense), element 2j in the low nibble of byte j
+ *              (torch.float4_e2m1fn_x2 packing, _mm_fp4); 16-byte aligned.
+ *   sf       : uint8 [bsp_nvfp4_sf_bytes(M, K)] e4m3 bytes, 128x4 layout;
+ *              padding rows/columns are written as 0.  16-byte aligned.
+ * Rows are not padded in `codes` (the pages pad with F.pad and narrow back;
+ * here padding rows exist only in `sf`).
+ * Errors: K % 16 != 0, K <= 0, M < 0, ld_x < K, bad sf_mode, NULL required
+ * pointer -> INVALID_ARG; alignment -> ALIGNMENT.  M == 0 is a no-op. */
+int nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                   const float *global_sf, int sf_mode, float *row_gs, float *row_inv_gs,
+                   uint8_t *codes, uint8_t *sf, bsp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * NVFP4 GEMM (nvfp4_qat_config.py, NVFP4QATQuantizeMethod.apply:
+ * mm_fp4(x_fp4, w_fp4.T, x_scale, w_scale.T, 1/(gs_x*gs_w), bf16) then
+ * out + bias).  TN: both operands are K-major.
+ *
+ *   D[m, n] = alpha * row_scale[m] * sum_k A(m,k) sfA(m,k/16) B(n,k) sfB(n,k/16)
+ *             + bias[n]
+ * computed on tcgen05 block-scaled tensor cores with fp32 accumulation, then
+ * rounded once to the output type.
+ *
+ *   A, sfA    : nvfp4_quantize output for the activations, [M, K/2] + sf(M, K)
+ *   B, sfB    : nvfp4_quantize output for the weight, [N, K/2] + sf(N, K)
+ *   alpha     : fp32 [1] (device), or NULL for 1.0
+ *   row_scale : fp32 [M] per-row factor (1/gs[m] of PER_ROW quantization), or NULL
+ *   bias      : bf16 [N], 16-byte aligned, or NULL
+ *   D         : [M, ld_d] of d_dtype (BSP_OUT_BF16 or BSP_OUT_F32), 16-byte
+ *               aligned, ld_d >= N, ld_d * sizeof(elem) % 16 == 0
+ * Errors: M < 0, N < 0, K <= 0, K % 32 != 0 (the packed rows must be a
+ * multiple of 16 bytes for the tensor-memory-access engine), N % 8 != 0,
+ * ld_d < N, bad d_dtype, NULL A/B/sfA/sfB/D -> INVALID_ARG; alignment ->
+ * ALIGNMENT.  M == 0 or N == 0 is a no-op. */
+int nvfp4_gemm(const uint8_t *A, const uint8_t *sfA, const uint8_t *B, const uint8_t *sfB,
+               int64_t M, int64_t N, int64_t K, const float *alpha, const float *row_scale,
+               const uint16_t *bias, void *D, int d_dtype, int64_t ld_d, bsp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 quantization (mxfp8_config.py, DiffusionMXFP8Config: groups of 32
+ * K-elements share one float8_e8m0fnu scale, e4m3 elements, OCP MX).
+ * Per group: E = floor(log2 amax) (-inf for amax 0), e = clamp(E - 8, -127, 127),
+ * scale byte = e + 127, q_i = e4m3_rne_sat(x_i * 2^-e).
+ *   x  : bf16 [M, K], ld_x as for nvfp4_quantize
+ *   q  : uint8 e4m3 [M, K] (dense), 16-byte aligned
+ *   sf : uint8 [bsp_mxfp8_sf_bytes(M, K)] e8m0 bytes, 128x4 layout, padding 0
+ * Errors: K % 32 != 0 and the rest as nvfp4_quantize. */
+int mxfp8_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                   uint8_t *q, uint8_t *sf, bsp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 GEMM (mxfp8_config.py, NPUMxfp8LinearMethod._quant_matmul: per-group
+ * e8m0 scales on both operands, bias, output in the activation dtype).
+ *   D[m, n] = alpha * sum_k A(m,k) 2^eA(m,k/32) B(n,k) 2^eB(n,k/32) + bias[n]
+ * Arguments as nvfp4_gemm, with A [M, K] / B [N, K] e4m3 bytes and e8m0
+ * scales from mxfp8_quantize.  K % 32 != 0 -> INVALID_ARG. */
+int mxfp8_gemm(const uint8_t *A, const uint8_t *sfA, const uint8_t *B, const uint8_t *sfB,
+               int64_t M, int64_t N, int64_t K, const float *alpha,
+               const uint16_t *bias, void *D, int d_dtype, int64_t ld_d, bsp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Device error word.
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns BSP_OK, BSP_ERR_TIMEOUT if a kernel's bounded wait ran out
+ * since the last call, or BSP_ERR_CUDA if the synchronisation failed.
+ * ---------------------------------------------------------------------- */
+int bsp_device_status(bsp_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Diagnostics (used by the tests to pin the hardware conversions that the
+ * quantize kernels use).  All buffers are device buffers of n elements.
+ * ---------------------------------------------------------------------- */
+
+/* codes[i] = e2m1 code (0..15) of v[i] by the kernels' conversion path. */
+int bsp_debug_encode_e2m1(const float *v, int64_t n, uint8_t *codes, bsp_stream_t stream);
+/* bytes[i] = e4m3 byte of v[i] by the kernels' conversion path. */
+int bsp_debug_encode_e4m3(const float *v, int64_t n, uint8_t *bytes, bsp_stream_t stream);
+/* Launches one block that waits on a shared-memory barrier nobody arrives at,
+ * with a limit of `limit_ns` nanoseconds (1e3 .. 1e10).  The wait runs out and
+ * sets the error word, so bsp_device_status then returns BSP_ERR_TIMEOUT. */
+int bsp_debug_wait_timeout(int64_t limit_ns, bsp_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSP_H */

@@ -1,0 +1,77 @@
+"""The C-ABI library loads, exports every function include/bsp.h declares, and
+rejects bad arguments on the host (no GPU needed: validation happens before any
+device call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_scaled_precision_05_b200 import _native as nat
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bsp.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", src)) - {"if", "sizeof"})
+
+
+def test_header_and_binding_agree():
+    assert sorted(nat.SIGNATURES) == _declared_functions()
+
+
+def test_library_exports_every_declared_symbol():
+    L = nat.lib()
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for s in range(6):
+        assert nat.status_string(s).startswith("BSP_")
+    assert "UNKNOWN" in nat.status_string(99)
+    assert nat.lib().bsp_version() >= 100
+
+
+@pytest.mark.parametrize("rows,K,nv,mx", [(1, 16, 512, 0), (128, 256, 128 * 16, 128 * 8), (129, 64, 256 * 4, 256 * 4),
+                                          (32760, 5120, 32768 * 320, 32768 * 160), (0, 32, 0, 0), (5, 24, 0, 0)])
+def test_sf_bytes(rows, K, nv, mx):
+    import oracle
+    assert nat.lib().bsp_nvfp4_sf_bytes(rows, K) == nv
+    assert nat.lib().bsp_mxfp8_sf_bytes(rows, K) == mx
+    if K % 16 == 0:
+        assert nv == oracle.sf_bytes(rows, K // 16)
+
+
+def test_host_validation_rejects_bad_arguments():
+    L = nat.lib()
+    p = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(0x10008)
+    assert L.nvfp4_quantize(p, 4, 24, 24, p, 0, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG  # K % 16
+    assert L.nvfp4_quantize(p, 4, 32, 16, p, 0, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG  # ld < K
+    assert L.nvfp4_quantize(p, 4, 32, 32, p, 7, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG  # mode
+    assert L.nvfp4_quantize(p, 4, 32, 32, None, 0, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG  # no gs
+    assert L.nvfp4_quantize(odd, 4, 32, 32, p, 0, None, None, p, p, None) == nat.BSP_ERR_ALIGNMENT
+    assert L.nvfp4_quantize(p, 0, 32, 32, p, 0, None, None, p, p, None) == nat.BSP_OK  # empty is a no-op
+    assert L.mxfp8_quantize(p, 4, 48, 48, p, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.nvfp4_gemm(p, p, p, p, 4, 8, 48, None, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG  # K%32
+    assert L.nvfp4_gemm(p, p, p, p, 4, 12, 64, None, None, None, p, 0, 12, None) == nat.BSP_ERR_INVALID_ARG  # N%8
+    assert L.nvfp4_gemm(p, p, p, p, 4, 8, 64, None, None, None, p, 5, 8, None) == nat.BSP_ERR_INVALID_ARG  # dtype
+    assert L.nvfp4_gemm(p, p, p, p, 4, 8, 64, None, None, None, odd, 0, 8, None) == nat.BSP_ERR_ALIGNMENT
+    assert L.nvfp4_gemm(p, p, p, p, 4, 8, 64, None, None, None, p, 0, 12, None) == nat.BSP_ERR_ALIGNMENT  # ld_d
+    assert L.nvfp4_gemm(p, p, p, p, 0, 8, 64, None, None, None, p, 0, 8, None) == nat.BSP_OK
+    assert L.mxfp8_gemm(p, p, p, p, 4, 8, 48, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.bsp_amax_bf16(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.bsp_debug_wait_timeout(10, None) == nat.BSP_ERR_INVALID_ARG
+
+
+def test_no_gpu_means_an_error_not_a_fallback():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    L = nat.lib()
+    p = ctypes.c_void_p(0x10000)
+    st = L.nvfp4_quantize(p, 4, 32, 32, p, 0, None, None, p, p, None)
+    assert st in (nat.BSP_ERR_CUDA, nat.BSP_ERR_UNSUPPORTED_DEVICE)
