@@ -18,14 +18,18 @@
 //               block-scaled MMAs (K = 64 fp4 / 32 fp8 each) accumulating into
 //               a 128 x 256 fp32 accumulator in tensor memory, and releases the
 //               stage with tcgen05.commit.
-//   warps 2..5  epilogue: read the accumulator (tcgen05.ld), release it to the
-//               MMA warp as soon as the last columns are read, apply alpha,
-//               row scale and bias in fp32, round once, store.
+//   warps 2..9  epilogue, two warps per 32-lane quarter of tensor memory, each
+//               owning 128 accumulator columns: read them into registers
+//               (tcgen05.ld), hand the accumulator back to the MMA warp at once
+//               (so the next tile's MMAs overlap this tile's stores), apply
+//               alpha, row scale and bias in fp32, round once, stage 32 rows x
+//               32 bytes in swizzled shared memory and write them with TMA
+//               stores (full 32-byte sectors; rows/columns past M/N clipped).
 // Tensor memory: columns [0, 256) accumulator; then, per pipeline stage, the
 // stage's scale factors (a scale column may only be rewritten once the stage's
 // MMAs have completed, which the stage's empty barrier already guarantees).
 // Ragged M / N / K edges: TMA fills out-of-range rows, K bytes and scale tiles
-// with zeros (zero codes times zero scales add nothing); stores are masked.
+// with zeros (zero codes times zero scales add nothing); TMA stores clip.
 // Every wait is bounded; a wait that runs out raises the device error word and
 // the CTA drains its outstanding copies and MMAs, frees tensor memory and exits.
 #include "bsp_device.cuh"
@@ -55,10 +59,12 @@ struct Cfg {
   static constexpr int ACC_COLS = BN;
   static constexpr int TMEM_COLS = 512;
   static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
-  static constexpr int EPI_WARPS = 4;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_COLS = BN / 2;           // accumulator columns per epilogue warp
+  static constexpr int STAGING_BYTES = 1024;        // per epilogue warp: 32 rows x 32 bytes
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES + 1024 + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -96,11 +102,12 @@ template <int KIND>
 __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
     blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                            const GemmParams p) {
+                            const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   using C = Cfg<KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::EPI_WARPS * C::STAGING_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
@@ -127,6 +134,7 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmSFA);
     prefetch_tensormap(&tmSFB);
+    prefetch_tensormap(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -236,8 +244,17 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // this warp's quarter of the tensor-memory lanes
+    const int ew = warp - 2;               // 0..7
+    const int q = warp & 3;                // tensor-memory lane quarter this warp may read
+    const int half = ew >> 2;              // which 128 accumulator columns
+    uint8_t* stage_buf = staging + ew * C::STAGING_BYTES;
     const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+    // One staging row = 32 bytes = W output elements; the two 16-byte halves
+    // are swapped on rows 4..7 of every 8 (TMA's 32-byte swizzle), which keeps
+    // the 32 lanes' shared-memory writes at the minimum of 4 wavefronts.
+    constexpr int W_BF16 = 16, W_F32 = 8;
+    uint8_t* my_row = stage_buf + lane * 32;
+    const uint32_t swz = (lane >> 2) & 1u;
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       int mb, nb;
@@ -248,57 +265,91 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
         break;
       }
       tc_fence_after_sync();
-      const int row = mb * C::BM + q * 32 + static_cast<int>(lane);
-      const bool row_ok = row < p.M;
-      float scale = alpha;
-      if (p.row_scale != nullptr && row_ok) scale = __fmul_rn(alpha, __ldg(p.row_scale + row));
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < C::BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32cols(taddr + static_cast<uint32_t>(c), r);
-        tmem_ld_wait();
-        if (c == C::BN - 32) {
-          // accumulator fully read: hand it back to the MMA warp
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
-        }
-        const int n0 = nb * C::BN + c;
-        if (n0 >= p.N) continue;
-        float b[32];
+      uint32_t acc[4][32];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * C::EPI_COLS);
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
+      for (int k = 0; k < 4; ++k) tmem_ld_32cols(taddr + 32u * k, acc[k]);
+      tmem_ld_wait();
+      // accumulator is in registers: hand tensor memory back to the MMA warp
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+
+      const int row0 = mb * C::BM + q * 32;
+      const int row = row0 + static_cast<int>(lane);
+      float scale = alpha;
+      if (p.row_scale != nullptr && row < p.M) scale = __fmul_rn(alpha, __ldg(p.row_scale + row));
+      const int col0 = nb * C::BN + half * C::EPI_COLS;
+      if (p.out_f32) {
+#pragma unroll
+        for (int j = 0; j < C::EPI_COLS / W_F32; ++j) {
+          const int n0 = col0 + j * W_F32;
+          if (n0 >= p.N) break;
+          float b[W_F32];
           uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-          if (p.bias != nullptr && n0 + 8 * h < p.N) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * h));
-          const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+          if (p.bias != nullptr) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0));
+          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            b[8 * h + 2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-            b[8 * h + 2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+            b[2 * i] = bf16_bits_to_f32(bw[i] & 0xFFFFu);
+            b[2 * i + 1] = bf16_bits_to_f32(bw[i] >> 16);
+          }
+          float y[W_F32];
+#pragma unroll
+          for (int i = 0; i < W_F32; ++i) {
+            const int c = j * W_F32 + i;
+            y[i] = __fmaf_rn(__uint_as_float(acc[c >> 5][c & 31]), scale, b[i]);
+          }
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          *reinterpret_cast<float4*>(my_row + 16 * (0u ^ swz)) = make_float4(y[0], y[1], y[2], y[3]);
+          *reinterpret_cast<float4*>(my_row + 16 * (1u ^ swz)) = make_float4(y[4], y[5], y[6], y[7]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmD, stage_buf, n0, row0);
+            bulk_commit_group();
           }
         }
-        float y[32];
+      } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) y[i] = __fmaf_rn(__uint_as_float(r[i]), scale, b[i]);
-        if (!row_ok) continue;
-        if (p.out_f32) {
-          float* dst = static_cast<float*>(p.D) + static_cast<int64_t>(row) * p.ld_d + n0;
+        for (int j = 0; j < C::EPI_COLS / W_BF16; ++j) {
+          const int n0 = col0 + j * W_BF16;
+          if (n0 >= p.N) break;
+          float b[W_BF16];
 #pragma unroll
-          for (int h = 0; h < 8; ++h)
-            if (n0 + 4 * h < p.N)
-              *reinterpret_cast<float4*>(dst + 4 * h) = make_float4(y[4 * h], y[4 * h + 1], y[4 * h + 2], y[4 * h + 3]);
-        } else {
-          uint16_t* dst = static_cast<uint16_t*>(p.D) + static_cast<int64_t>(row) * p.ld_d + n0;
+          for (int h = 0; h < 2; ++h) {
+            uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+            if (p.bias != nullptr && n0 + 8 * h < p.N) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * h));
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-          for (int h = 0; h < 4; ++h)
-            if (n0 + 8 * h < p.N)
-              *reinterpret_cast<uint4*>(dst + 8 * h) =
-                  make_uint4(pack_bf16x2(y[8 * h], y[8 * h + 1]), pack_bf16x2(y[8 * h + 2], y[8 * h + 3]),
-                             pack_bf16x2(y[8 * h + 4], y[8 * h + 5]), pack_bf16x2(y[8 * h + 6], y[8 * h + 7]));
+            for (int i = 0; i < 4; ++i) {
+              b[8 * h + 2 * i] = bf16_bits_to_f32(bw[i] & 0xFFFFu);
+              b[8 * h + 2 * i + 1] = bf16_bits_to_f32(bw[i] >> 16);
+            }
+          }
+          uint32_t packed[W_BF16 / 2];
+#pragma unroll
+          for (int i = 0; i < W_BF16 / 2; ++i) {
+            const int c = j * W_BF16 + 2 * i;
+            packed[i] = pack_bf16x2(__fmaf_rn(__uint_as_float(acc[c >> 5][c & 31]), scale, b[2 * i]),
+                                    __fmaf_rn(__uint_as_float(acc[(c + 1) >> 5][(c + 1) & 31]), scale, b[2 * i + 1]));
+          }
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          *reinterpret_cast<uint4*>(my_row + 16 * (0u ^ swz)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          *reinterpret_cast<uint4*>(my_row + 16 * (1u ^ swz)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmD, stage_buf, n0, row0);
+            bulk_commit_group();
+          }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before_sync();
@@ -336,6 +387,19 @@ int encode_scales(CUtensorMap* m, const void* base, int64_t bands, int64_t tiles
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
 
+// Row-major output [rows, ld] of bf16 or fp32, boxes of 32 rows x 32 bytes, 32-byte swizzle.
+int encode_output(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+  const int64_t esize = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esize)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(32 / esize), 32u};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = encode_tiled_fn()(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+                                 dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
+}
+
 template <int KIND>
 int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, int64_t M, int64_t N,
              int64_t K, const float* alpha, const float* row_scale, const uint16_t* bias, void* D, int d_dtype,
@@ -360,11 +424,12 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
 
   const int64_t row_bytes = KIND == kNVF4 ? K / 2 : K;
   const int64_t tiles_per_band = round_up(K / group, 4) / 4;
-  CUtensorMap tmA, tmB, tmSFA, tmSFB;
+  CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
   if ((st = encode_operand(&tmA, A, M, row_bytes, C::BM)) != BSP_OK) return st;
   if ((st = encode_operand(&tmB, B, N, row_bytes, C::BN)) != BSP_OK) return st;
   if ((st = encode_scales(&tmSFA, sfA, ceil_div(M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
   if ((st = encode_scales(&tmSFB, sfB, ceil_div(N, 128), tiles_per_band, C::ATOMS, 2)) != BSP_OK) return st;
+  if ((st = encode_output(&tmD, D, M, N, ld_d, d_dtype == BSP_OUT_F32)) != BSP_OK) return st;
 
   static bool attr_set[64] = {};
   if (!attr_set[dev.id]) {
@@ -390,7 +455,7 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   p.err = dev.err_word;
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
   const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  blockscaled_gemm_kernel<KIND><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+  blockscaled_gemm_kernel<KIND><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, tmD, p);
   return launch_status();
 }
 

@@ -107,6 +107,31 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
 // NVFP4, K % 64 == 0.  Rows [M, Mp) are the scale padding (zeros).
 // A "quad" is 64 elements = one 128x4 tile row = 8 lanes; a warp step is 4 quads.
 // ---------------------------------------------------------------------------
+// U warp steps of one row: U 16-byte loads in flight per lane, then the
+// quantization of each.  `lp`, `cp`, `sp` point at this lane's first element,
+// code word and (for j == 0) scale word of the first step.
+template <int U>
+__device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uint8_t* sp, bool live, float gs,
+                                            uint32_t j) {
+  uint4 v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) v[u] = live ? ldg16(lp + u * 256) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    uint32_t mag = max_mag8(v[u]);
+    mag = max(mag, __shfl_xor_sync(kFull, mag, 1));  // lanes 2g, 2g+1 hold group g
+    uint32_t sfb;
+    float inv;
+    nvfp4_scale(mag, gs, sfb, inv);
+    const uint32_t word = nvfp4_codes8(v[u], inv);
+    const uint32_t s1 = __shfl_down_sync(kFull, sfb, 2);
+    const uint32_t s2 = __shfl_down_sync(kFull, sfb, 4);
+    const uint32_t s3 = __shfl_down_sync(kFull, sfb, 6);
+    if (live) *reinterpret_cast<uint32_t*>(cp + u * 128) = word;
+    if (j == 0) *reinterpret_cast<uint32_t*>(sp + u * 2048) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
 template <bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
@@ -114,6 +139,8 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
   const uint32_t lane = lane_id();
   const uint32_t sub = lane >> 3, j = lane & 7u;
   const int64_t quads = K >> 6;
+  const int64_t steps = quads >> 2;  // full warp steps (4 quads) per row
+  const int64_t rem = quads & 3;     // quads of a last, partial step
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
@@ -123,35 +150,19 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
     if (kPerRow && live) gs = row_scale_pass(row, K, r, row_gs, row_inv);
-    uint8_t* crow = codes + r * (K >> 1);
-    const int64_t sfb_row = sf_row_base(r, quads);
-
-    for (int64_t q0 = 0; q0 < quads; q0 += 4 * kUnroll) {
-      uint4 v[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t q = q0 + 4 * u + sub;
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (live && q < quads) v[u] = ldg16(row + q * 64 + j * 8);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t q = q0 + 4 * u + sub;
-        uint32_t mag = max_mag8(v[u]);
-        mag = max(mag, __shfl_xor_sync(kFull, mag, 1));  // lanes 2g, 2g+1 hold group g
-        uint32_t sfb;
-        float inv;
-        nvfp4_scale(mag, gs, sfb, inv);
-        const uint32_t word = nvfp4_codes8(v[u], inv);
-        const uint32_t s1 = __shfl_down_sync(kFull, sfb, 2);
-        const uint32_t s2 = __shfl_down_sync(kFull, sfb, 4);
-        const uint32_t s3 = __shfl_down_sync(kFull, sfb, 6);
-        if (q < quads) {
-          if (live) *reinterpret_cast<uint32_t*>(crow + q * 32 + j * 4) = word;
-          if (j == 0)
-            *reinterpret_cast<uint32_t*>(sf + sfb_row + q * 512) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
-        }
-      }
+    // this lane's element, code word and scale word in the row's first step
+    const uint16_t* lp = row + sub * 64 + j * 8;
+    uint8_t* cp = codes + r * (K >> 1) + sub * 32 + j * 4;
+    uint8_t* sp = sf + sf_row_base(r, quads) + sub * 512;
+    int64_t st = 0;
+    for (; st + kUnroll <= steps; st += kUnroll)
+      nvfp4_steps<kUnroll>(lp + st * 256, cp + st * 128, sp + st * 2048, live, gs, j);
+    for (; st < steps; ++st) nvfp4_steps<1>(lp + st * 256, cp + st * 128, sp + st * 2048, live, gs, j);
+    if (rem) {
+      // last partial step: quads beyond the row end are predicated off
+      const bool in = sub < rem;
+      nvfp4_steps<1>(in ? lp + st * 256 : lp, in ? cp + st * 128 : cp, in ? sp + st * 2048 : sp, live && in, gs,
+                     in ? j : 1u);
     }
   }
 }
@@ -358,11 +369,20 @@ __global__ void debug_wait_kernel(uint64_t limit_ns, uint32_t* err) {
   if (threadIdx.x == 0 && !mbar_wait(&bar, 0, nullptr, limit_ns)) raise_error(err, kErrTimeout);
 }
 
-int grid_for_rows(const DeviceInfo& dev, int64_t rows) {
+// Persistent grid: exactly the blocks that are resident at once (rows are
+// spread over warps by a grid-stride loop), so no block starts in a second,
+// partial wave.
+template <typename Kernel>
+int grid_for_rows(const DeviceInfo& dev, Kernel kernel, int64_t rows) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, 0) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
   const int64_t warps_per_block = kQuantThreads / 32;
-  int64_t blocks = ceil_div(rows, warps_per_block);
-  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;  // 8 blocks of 256 threads per SM
-  return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+  const int64_t needed = ceil_div(rows, warps_per_block);
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * per_sm;
+  return static_cast<int>(needed < cap ? (needed > 0 ? needed : 1) : cap);
 }
 
 }  // namespace
@@ -383,22 +403,27 @@ int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const 
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
   const int64_t Mp = round_up(M, 128);
-  const int grid = grid_for_rows(dev, Mp);
   const bool per_row = sf_mode == BSP_SF_PER_ROW;
   if (K % 64 == 0) {
-    if (per_row)
-      nvfp4_quant_k64_kernel<true><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs,
-                                                                       row_inv_gs, codes, sf);
-    else
-      nvfp4_quant_k64_kernel<false><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr,
-                                                                        nullptr, codes, sf);
+    if (per_row) {
+      auto k = nvfp4_quant_k64_kernel<true>;
+      k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
+                                                                 codes, sf);
+    } else {
+      auto k = nvfp4_quant_k64_kernel<false>;
+      k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
+                                                                 codes, sf);
+    }
   } else {
-    if (per_row)
-      nvfp4_quant_generic_kernel<true><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs,
-                                                                           row_inv_gs, codes, sf);
-    else
-      nvfp4_quant_generic_kernel<false><<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr,
-                                                                            nullptr, codes, sf);
+    if (per_row) {
+      auto k = nvfp4_quant_generic_kernel<true>;
+      k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
+                                                                 codes, sf);
+    } else {
+      auto k = nvfp4_quant_generic_kernel<false>;
+      k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
+                                                                 codes, sf);
+    }
   }
   return launch_status();
 }
@@ -413,11 +438,12 @@ int mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, uint8_
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
   const int64_t Mp = round_up(M, 128);
-  const int grid = grid_for_rows(dev, Mp);
   if (K % 128 == 0)
-    mxfp8_quant_k128_kernel<<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, q, sf);
+    mxfp8_quant_k128_kernel<<<grid_for_rows(dev, mxfp8_quant_k128_kernel, Mp), kQuantThreads, 0, stream>>>(
+        x, M, Mp, K, ld_x, q, sf);
   else
-    mxfp8_quant_generic_kernel<<<grid, kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, q, sf);
+    mxfp8_quant_generic_kernel<<<grid_for_rows(dev, mxfp8_quant_generic_kernel, Mp), kQuantThreads, 0, stream>>>(
+        x, M, Mp, K, ld_x, q, sf);
   return launch_status();
 }
 
