@@ -9,15 +9,22 @@
 // MXFP8: e4m3 operands, e8m0 scales per 32 (kind::mxf8f6f4, scale_vec::1X) --
 //   vllm-omni mxfp8_config.py, NPUMxfp8LinearMethod._quant_matmul.
 //
-// Design (one CTA per SM, persistent over output tiles of 128 x 256):
-//   warp 0      TMA producer: per stage, 128 rows of A and 256 rows of B (128
-//               bytes of K each, 128-byte swizzle) and the matching 128x4
-//               scale tiles, all into shared memory, completion on an mbarrier.
-//   warp 1      MMA issuer (one thread): copies the stage's scale tiles from
-//               shared memory into tensor memory (tcgen05.cp), issues four
-//               block-scaled MMAs (K = 64 fp4 / 32 fp8 each) accumulating into
-//               a 128 x 256 fp32 accumulator in tensor memory, and releases the
-//               stage with tcgen05.commit.
+// Design (persistent, one CTA per SM, warp-specialised):
+//   warp 0      TMA producer: per stage, this CTA's 128 rows of A and its rows
+//               of B (128 bytes of K each, 128-byte swizzle) plus the matching
+//               128x4 scale tiles, into shared memory; completion is counted on
+//               an mbarrier (the pair leader's one in the 2-SM form).
+//   warp 1      MMA issuer (one thread of the leader CTA): once a stage's data
+//               and scale factors are ready, issues four block-scaled MMAs
+//               (K = 64 fp4 / 32 fp8 each) accumulating fp32 in tensor memory,
+//               and releases the stage (tcgen05.commit).
+//   warps 10-13 scale-factor warps, one per 32-lane quarter of tensor memory:
+//               read the stage's 128x4 scale tiles from shared memory and write
+//               them into the stage's scale columns of tensor memory
+//               (tcgen05.st; each quarter holds the scales of all rows, which is
+//               the replicated layout the block-scaled MMA reads).  Keeping the
+//               scale traffic off the tensor pipe lets it overlap the MMAs of
+//               the previous stages.
 //   warps 2..9  epilogue, two warps per 32-lane quarter of tensor memory, each
 //               owning 128 accumulator columns: read them into registers
 //               (tcgen05.ld), hand the accumulator back to the MMA warp at once
@@ -25,6 +32,15 @@
 //               alpha, row scale and bias in fp32, round once, stage 32 rows x
 //               32 bytes in swizzled shared memory and write them with TMA
 //               stores (full 32-byte sectors; rows/columns past M/N clipped).
+//   (roles by warp index: 0 producer, 1 MMA, 2-9 epilogue, 10-13 scales)
+// Two forms:
+//   1-SM   128 x 256 output tiles, each CTA loads 128 rows of A and 256 of B.
+//   2-SM   256 x 256 output tiles per cluster of two CTAs (cta_group::2): each
+//          CTA loads its own 128 rows of A and 128 of the 256 rows of B, and
+//          the B scale tiles of all 256 rows; the leader's MMAs read both CTAs'
+//          shared memory and write each CTA's 128 accumulator rows into its own
+//          tensor memory; both CTAs' scale warps report to the leader.  Half
+//          the B traffic per SM and smaller stages.  (No TMA multicast.)
 // Tensor memory: columns [0, 256) accumulator; then, per pipeline stage, the
 // stage's scale factors (a scale column may only be rewritten once the stage's
 // MMAs have completed, which the stage's empty barrier already guarantees).
@@ -35,36 +51,68 @@
 #include "bsp_device.cuh"
 #include "bsp_internal.h"
 
+// Tuning knobs (compile-time): pipeline depth, and how the epilogue writes D --
+// 1: 32x32-byte swizzled shared-memory staging + TMA stores, with
+// BSP_GEMM_STAGING_BUFS buffers per epilogue warp; 0: 16-byte stores straight
+// from registers.
+#ifndef BSP_GEMM_STAGES
+#define BSP_GEMM_STAGES 8  // upper bound; the stages that fit shared and tensor memory are used
+#endif
+#ifndef BSP_GEMM_EPI_TMA
+#define BSP_GEMM_EPI_TMA 1
+#endif
+#ifndef BSP_GEMM_STAGING_BUFS
+#define BSP_GEMM_STAGING_BUFS 1
+#endif
+// Smallest M for which the 2-SM (CTA pair) form is used.  Off by default: on
+// B200 the pair form measured slower than the 1-SM form with scale-factor
+// warps on every workload here (its per-stage handshakes cross the pair).
+#ifndef BSP_GEMM_PAIR_MIN_M
+#define BSP_GEMM_PAIR_MIN_M (1 << 30)
+#endif
+
 namespace bsp {
 namespace {
 
 enum Kind : int { kNVF4 = 0, kMXF8 = 1 };
 
-template <int KIND>
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+template <int KIND, int CG>
 struct Cfg {
-  static constexpr int BM = 128, BN = 256;
+  static constexpr int BM = 128;                        // accumulator rows per CTA
+  static constexpr int BN = 256;                        // output tile columns
+  static constexpr int TILE_M = BM * CG;                // output tile rows
+  static constexpr int B_ROWS = BN / CG;                // rows of B each CTA loads
   static constexpr int ROW_BYTES = 128;                 // K bytes per operand row per stage
-  static constexpr int MMAS = 4;                         // per stage, 32 bytes of K each
-  static constexpr int ATOMS = KIND == kNVF4 ? 4 : 1;    // 128x4 scale tiles per 128 rows per stage
+  static constexpr int MMAS = 4;                        // per stage, 32 bytes of K each
+  static constexpr int ATOMS = KIND == kNVF4 ? 4 : 1;   // 128x4 scale tiles per 128 rows per stage
   static constexpr int A_BYTES = BM * ROW_BYTES;
-  static constexpr int B_BYTES = BN * ROW_BYTES;
+  static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
   static constexpr int SFA_BYTES = ATOMS * 512;
-  static constexpr int SFB_BYTES = 2 * ATOMS * 512;
-  static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int SFB_BYTES = 2 * ATOMS * 512;     // both 128-row bands of the 256 columns
+  static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // per CTA per stage
   static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
-  static constexpr int STAGES = 4;
   static constexpr int SFA_COLS = ATOMS * 4;
   static constexpr int SFB_COLS = ATOMS * 8;
-  static constexpr int SF_COLS = SFA_COLS + SFB_COLS;
+  static constexpr int SF_COLS = SFA_COLS + SFB_COLS;   // 48 (fp4) / 12 (fp8) per stage
   static constexpr int ACC_COLS = BN;
   static constexpr int TMEM_COLS = 512;
-  static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
   static constexpr int EPI_WARPS = 8;
-  static constexpr int EPI_COLS = BN / 2;           // accumulator columns per epilogue warp
-  static constexpr int STAGING_BYTES = 1024;        // per epilogue warp: 32 rows x 32 bytes
-  static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  static constexpr int EPI_COLS = BN / 2;  // accumulator columns per epilogue warp
+  static constexpr bool EPI_TMA = BSP_GEMM_EPI_TMA != 0;
+  static constexpr int STAGING_BUFS = EPI_TMA ? BSP_GEMM_STAGING_BUFS : 0;
+  static constexpr int STAGING_BYTES = 1024 * STAGING_BUFS;  // per epilogue warp: buffers of 32 rows x 32 bytes
+  static constexpr int SF_WARPS = 4;
+  static constexpr int FIRST_SF_WARP = 2 + EPI_WARPS;
+  static constexpr int THREADS = 64 + (EPI_WARPS + SF_WARPS) * 32;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES + 1024 + BAR_BYTES;
+  static constexpr int FIXED_BYTES = EPI_WARPS * STAGING_BYTES + 1024 + BAR_BYTES;
+  static constexpr int STAGES = cmin(cmin((232448 - FIXED_BYTES) / STAGE_BYTES, (TMEM_COLS - ACC_COLS) / SF_COLS),
+                                     BSP_GEMM_STAGES);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+  static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -98,18 +146,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int KIND>
-__global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
+template <int KIND, int CG>
+__global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                             const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-  using C = Cfg<KIND>;
+  using C = Cfg<KIND, CG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::EPI_WARPS * C::STAGING_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* sf_ready = empty + C::STAGES;
+  uint64_t* acc_full = sf_ready + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -117,14 +166,17 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;  // position in the CTA pair
+  const bool leader = rank == 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], C::SF_WARPS * CG);  // the scale warps of both CTAs report to the leader
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, C::EPI_WARPS);
+    mbar_init(acc_empty, C::EPI_WARPS * CG);  // the epilogue warps of both CTAs arrive on the leader's
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -137,14 +189,24 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
     prefetch_tensormap(&tmD);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (CG == 2)
+    cluster_sync();  // the peer's barriers are initialised before anyone signals them
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int num_tiles = p.num_m * p.num_n;
+  const int first_tile = static_cast<int>(blockIdx.x) / CG;
+  const int tile_step = static_cast<int>(gridDim.x) / CG;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -153,9 +215,12 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
       uint32_t issued[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
         int mb, nb;
         tile_coords(t, p.num_m, p.num_n, mb, nb);
+        const int a_row = mb * C::TILE_M + static_cast<int>(rank) * C::BM;
+        const int b_row = nb * C::BN + static_cast<int>(rank) * C::B_ROWS;
+        const int a_band = mb * CG + static_cast<int>(rank);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -163,9 +228,9 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
           }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-          tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, mb * C::BM);
-          tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, nb * C::BN);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, mb);
+          tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, a_row);
+          tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, b_row);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, a_band);
           tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, &full[stage], 0, kb * C::ATOMS, nb * 2);
           ++issued[stage];
           if (++stage == C::STAGES) {
@@ -184,18 +249,20 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int it = 0;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+      constexpr uint16_t kPair = 0x3;
+      for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
         if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          // the scale warps signal after their CTA's stage landed and its scales are in tensor memory
+          if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
@@ -203,60 +270,177 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
           const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sfa_t = tmem + C::ACC_COLS + stage * C::SF_COLS;
           const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-          const uint32_t sfa_s = sbase + C::A_BYTES + C::B_BYTES;
-          const uint32_t sfb_s = sfa_s + C::SFA_BYTES;
-#pragma unroll
-          for (int a = 0; a < C::ATOMS; ++a) tc_cp_32x128b_warpx4(sfa_t + 4 * a, desc_sf_block(sfa_s + 512 * a));
-#pragma unroll
-          for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-            for (int a = 0; a < C::ATOMS; ++a)
-              tc_cp_32x128b_warpx4(sfb_t + 8 * a + 4 * rt, desc_sf_block(sfb_s + 512 * (rt * C::ATOMS + a)));
           const uint64_t adesc = desc_kmajor_sw128(sbase);
           const uint64_t bdesc = desc_kmajor_sw128(sbase + C::A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::MMAS; ++kk) {
             const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
             // 32 bytes of K per MMA: advance the start address by 32 >> 4.
-            if constexpr (KIND == kNVF4)
-              tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_nvf4(C::BM, C::BN), sfa_t + 4u * kk,
-                          sfb_t + 8u * kk, accumulate);
-            else
-              tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8(C::BM, C::BN, static_cast<uint32_t>(kk)),
-                          sfa_t, sfb_t, accumulate);
+            if constexpr (KIND == kNVF4) {
+              const uint32_t idesc = idesc_nvf4(C::TILE_M, C::BN);
+              if constexpr (CG == 2)
+                tc_mma_nvf4_pair(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t + 4u * kk, sfb_t + 8u * kk,
+                                 accumulate);
+              else
+                tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t + 4u * kk, sfb_t + 8u * kk,
+                            accumulate);
+            } else {
+              const uint32_t idesc = idesc_mxf8(C::TILE_M, C::BN, static_cast<uint32_t>(kk));
+              if constexpr (CG == 2)
+                tc_mma_mxf8_pair(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t, sfb_t, accumulate);
+              else
+                tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t, sfb_t, accumulate);
+            }
           }
-          tc_commit(&empty[stage]);
+          if constexpr (CG == 2)
+            tc_commit_pair(&empty[stage], kPair);
+          else
+            tc_commit(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        if constexpr (CG == 2)
+          tc_commit_pair(acc_full, kPair);
+        else
+          tc_commit(acc_full);
       }
       if (!ok) {
         *abort_flag = 1u;
         raise_error(p.err, kErrTimeout);
       }
       // No MMA may still be running when tensor memory is freed.
-      tc_commit(drain);
+      if constexpr (CG == 2)
+        tc_commit_pair(drain, kPair);
+      else
+        tc_commit(drain);
       if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
+    } else if (lane == 0) {
+      // pair follower: its MMAs are issued by the leader; wait for their end
+      if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
+    }
+  } else if (warp >= C::FIRST_SF_WARP) {
+    // ------------------------------------------------------------ scale factors
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sf_ready_leader = CG == 2 ? mapa_shared(smem_u32(sf_ready), 0u) : smem_u32(sf_ready);
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          ok = false;
+          break;
+        }
+        // Line `lane` of each 512-byte scale tile (the scales of rows lane,
+        // lane+32, lane+64, lane+96 for 4 K-groups) becomes 4 consecutive
+        // columns of this lane; every lane quarter gets the same copy.
+        const uint8_t* sfa_s = smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+        const uint8_t* sfb_s = sfa_s + C::SFA_BYTES;
+        uint32_t v[C::SF_COLS];
+#pragma unroll
+        for (int a = 0; a < C::ATOMS; ++a) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sfa_s + 512 * a + lane * 16);
+          v[4 * a + 0] = w.x;
+          v[4 * a + 1] = w.y;
+          v[4 * a + 2] = w.z;
+          v[4 * a + 3] = w.w;
+        }
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+          for (int a = 0; a < C::ATOMS; ++a) {
+            const uint4 w = *reinterpret_cast<const uint4*>(sfb_s + 512 * (rt * C::ATOMS + a) + lane * 16);
+            v[C::SFA_COLS + 8 * a + 4 * rt + 0] = w.x;
+            v[C::SFA_COLS + 8 * a + 4 * rt + 1] = w.y;
+            v[C::SFA_COLS + 8 * a + 4 * rt + 2] = w.z;
+            v[C::SFA_COLS + 8 * a + 4 * rt + 3] = w.w;
+          }
+        const uint32_t taddr = tmem + lane_base + C::ACC_COLS + stage * C::SF_COLS;
+        if constexpr (C::SF_COLS == 48) {
+          tmem_st_16cols(taddr, v);
+          tmem_st_16cols(taddr + 16, v + 16);
+          tmem_st_16cols(taddr + 32, v + 32);
+        } else {
+          static_assert(C::SF_COLS == 12, "scale columns per stage");
+          tmem_st_4cols(taddr, v);
+          tmem_st_8cols(taddr + 4, v + 4);
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CG == 2)
+            mbar_arrive_cluster(sf_ready_leader + 8u * stage);
+          else
+            mbar_arrive(&sf_ready[stage]);
+        }
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1u;
+      raise_error(p.err, kErrTimeout);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;               // 0..7
-    const int q = warp & 3;                // tensor-memory lane quarter this warp may read
-    const int half = ew >> 2;              // which 128 accumulator columns
+    const int ew = warp - 2;   // 0..7
+    const int q = warp & 3;    // tensor-memory lane quarter this warp may read
+    const int half = ew >> 2;  // which 128 accumulator columns
     uint8_t* stage_buf = staging + ew * C::STAGING_BYTES;
     const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+    const uint32_t acc_empty_leader = CG == 2 ? mapa_shared(smem_u32(acc_empty), 0u) : smem_u32(acc_empty);
     // One staging row = 32 bytes = W output elements; the two 16-byte halves
     // are swapped on rows 4..7 of every 8 (TMA's 32-byte swizzle), which keeps
     // the 32 lanes' shared-memory writes at the minimum of 4 wavefronts.
     constexpr int W_BF16 = 16, W_F32 = 8;
-    uint8_t* my_row = stage_buf + lane * 32;
     const uint32_t swz = (lane >> 2) & 1u;
+    uint32_t store_seq = 0;  // TMA stores issued by this warp (picks the staging buffer)
+
+    // Writes 32 bytes of this lane's row into the staging buffer, then one
+    // lane stores the 32 x 32-byte box at (n0, row0).
+    auto stage_and_store = [&](int n0, int row0, uint4 lo, uint4 hi) {
+      if constexpr (C::EPI_TMA) {
+        uint8_t* buf = stage_buf + (store_seq % C::STAGING_BUFS) * 1024;
+        if (lane == 0) bulk_wait_read_allow(C::STAGING_BUFS - 1);
+        __syncwarp();
+        *reinterpret_cast<uint4*>(buf + lane * 32 + 16 * (0u ^ swz)) = lo;
+        *reinterpret_cast<uint4*>(buf + lane * 32 + 16 * (1u ^ swz)) = hi;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmD, buf, n0, row0);
+          bulk_commit_group();
+        }
+        ++store_seq;
+      } else {
+        const int row = row0 + static_cast<int>(lane);
+        if (row < p.M) {
+          const int64_t esize = p.out_f32 ? 4 : 2;
+          uint8_t* dst = static_cast<uint8_t*>(p.D) + (static_cast<int64_t>(row) * p.ld_d + n0) * esize;
+          *reinterpret_cast<uint4*>(dst) = lo;
+          if (n0 + 16 / esize < p.N) *reinterpret_cast<uint4*>(dst + 16) = hi;
+        }
+      }
+    };
+
+    auto release_accumulator = [&]() {
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (CG == 2)
+          mbar_arrive_cluster(acc_empty_leader);
+        else
+          mbar_arrive(acc_empty);
+      }
+    };
+
     int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+    for (int t = first_tile; t < num_tiles; t += tile_step, ++it) {
       int mb, nb;
       tile_coords(t, p.num_m, p.num_n, mb, nb);
       if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
@@ -265,99 +449,95 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
         break;
       }
       tc_fence_after_sync();
-      uint32_t acc[4][32];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * C::EPI_COLS);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) tmem_ld_32cols(taddr + 32u * k, acc[k]);
-      tmem_ld_wait();
-      // accumulator is in registers: hand tensor memory back to the MMA warp
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-
-      const int row0 = mb * C::BM + q * 32;
+      const int row0 = mb * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
       const int row = row0 + static_cast<int>(lane);
       float scale = alpha;
       if (p.row_scale != nullptr && row < p.M) scale = __fmul_rn(alpha, __ldg(p.row_scale + row));
       const int col0 = nb * C::BN + half * C::EPI_COLS;
-      if (p.out_f32) {
+
+      if (!p.out_f32) {
+        // bf16: read all 128 columns, applying the epilogue and packing as they
+        // arrive, release tensor memory, then store from registers.
+        uint32_t packed[C::EPI_COLS / 2];
 #pragma unroll
-        for (int j = 0; j < C::EPI_COLS / W_F32; ++j) {
-          const int n0 = col0 + j * W_F32;
-          if (n0 >= p.N) break;
-          float b[W_F32];
-          uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-          if (p.bias != nullptr) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0));
-          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+        for (int k = 0; k < C::EPI_COLS / 16; ++k) {
+          uint32_t r[16];
+          tmem_ld_16cols(taddr + 16u * k, r);
+          uint32_t bw[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            b[2 * i] = bf16_bits_to_f32(bw[i] & 0xFFFFu);
-            b[2 * i + 1] = bf16_bits_to_f32(bw[i] >> 16);
+          for (int h = 0; h < 2; ++h) {
+            const int n = col0 + 16 * k + 8 * h;
+            uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+            if (p.bias != nullptr && n < p.N) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+            bw[4 * h + 0] = bv.x;
+            bw[4 * h + 1] = bv.y;
+            bw[4 * h + 2] = bv.z;
+            bw[4 * h + 3] = bv.w;
           }
-          float y[W_F32];
+          tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < W_F32; ++i) {
-            const int c = j * W_F32 + i;
-            y[i] = __fmaf_rn(__uint_as_float(acc[c >> 5][c & 31]), scale, b[i]);
-          }
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
-          *reinterpret_cast<float4*>(my_row + 16 * (0u ^ swz)) = make_float4(y[0], y[1], y[2], y[3]);
-          *reinterpret_cast<float4*>(my_row + 16 * (1u ^ swz)) = make_float4(y[4], y[5], y[6], y[7]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmD, stage_buf, n0, row0);
-            bulk_commit_group();
-          }
+          for (int i = 0; i < 8; ++i)
+            packed[8 * k + i] =
+                pack_bf16x2(__fmaf_rn(__uint_as_float(r[2 * i]), scale, bf16_bits_to_f32(bw[i] & 0xFFFFu)),
+                            __fmaf_rn(__uint_as_float(r[2 * i + 1]), scale, bf16_bits_to_f32(bw[i] >> 16)));
         }
-      } else {
+        release_accumulator();
 #pragma unroll
         for (int j = 0; j < C::EPI_COLS / W_BF16; ++j) {
           const int n0 = col0 + j * W_BF16;
           if (n0 >= p.N) break;
-          float b[W_BF16];
+          stage_and_store(n0, row0, make_uint4(packed[8 * j], packed[8 * j + 1], packed[8 * j + 2], packed[8 * j + 3]),
+                          make_uint4(packed[8 * j + 4], packed[8 * j + 5], packed[8 * j + 6], packed[8 * j + 7]));
+        }
+      } else {
+        // fp32: 16 columns at a time, tensor memory released at the end.
+#pragma unroll 1
+        for (int k = 0; k < C::EPI_COLS / 16; ++k) {
+          uint32_t r[16];
+          tmem_ld_16cols(taddr + 16u * k, r);
+          tmem_ld_wait();
+          const int nk = col0 + 16 * k;
+          if (nk >= p.N) continue;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
+            const int n0 = nk + W_F32 * h;
+            if (n0 >= p.N) break;
             uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-            if (p.bias != nullptr && n0 + 8 * h < p.N) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * h));
+            if (p.bias != nullptr) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0));
             const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+            float y[W_F32];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              b[8 * h + 2 * i] = bf16_bits_to_f32(bw[i] & 0xFFFFu);
-              b[8 * h + 2 * i + 1] = bf16_bits_to_f32(bw[i] >> 16);
+              y[2 * i] = __fmaf_rn(__uint_as_float(r[8 * h + 2 * i]), scale, bf16_bits_to_f32(bw[i] & 0xFFFFu));
+              y[2 * i + 1] = __fmaf_rn(__uint_as_float(r[8 * h + 2 * i + 1]), scale, bf16_bits_to_f32(bw[i] >> 16));
             }
-          }
-          uint32_t packed[W_BF16 / 2];
-#pragma unroll
-          for (int i = 0; i < W_BF16 / 2; ++i) {
-            const int c = j * W_BF16 + 2 * i;
-            packed[i] = pack_bf16x2(__fmaf_rn(__uint_as_float(acc[c >> 5][c & 31]), scale, b[2 * i]),
-                                    __fmaf_rn(__uint_as_float(acc[(c + 1) >> 5][(c + 1) & 31]), scale, b[2 * i + 1]));
-          }
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
-          *reinterpret_cast<uint4*>(my_row + 16 * (0u ^ swz)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          *reinterpret_cast<uint4*>(my_row + 16 * (1u ^ swz)) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmD, stage_buf, n0, row0);
-            bulk_commit_group();
+            stage_and_store(n0, row0,
+                            make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                                       __float_as_uint(y[3])),
+                            make_uint4(__float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
+                                       __float_as_uint(y[7])));
           }
         }
+        release_accumulator();
       }
     }
-    if (lane == 0) bulk_wait_all();
+    if constexpr (C::EPI_TMA) {
+      if (lane == 0) bulk_wait_all();
+    }
     __syncwarp();
   }
 
   tc_fence_before_sync();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (CG == 2)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -400,11 +580,62 @@ int encode_output(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
 
+template <int KIND, int CG>
+int launch_gemm(const DeviceInfo& dev, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSFA,
+                const CUtensorMap& tmSFB, const CUtensorMap& tmD, GemmParams p, cudaStream_t stream) {
+  using C = Cfg<KIND, CG>;
+  auto kernel = blockscaled_gemm_kernel<KIND, CG>;
+  static bool attr_set[64] = {};
+  static int max_clusters[64] = {};
+  if (!attr_set[dev.id]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return launch_status();
+    int units = dev.sm_count / CG;
+    if constexpr (CG == 2) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * units, 1, 1);
+      cfg.blockDim = dim3(C::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) units = n;
+      cudaGetLastError();
+    }
+    max_clusters[dev.id] = units;
+    attr_set[dev.id] = true;
+  }
+  p.num_m = static_cast<int>(ceil_div(p.M, C::TILE_M));
+  p.num_n = static_cast<int>(ceil_div(p.N, C::BN));
+  const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
+  const int units = static_cast<int>(tiles < max_clusters[dev.id] ? tiles : max_clusters[dev.id]);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  if constexpr (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmSFA, tmSFB, tmD, p) != cudaSuccess) return launch_status();
+  return launch_status();
+}
+
 template <int KIND>
 int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, int64_t M, int64_t N,
              int64_t K, const float* alpha, const float* row_scale, const uint16_t* bias, void* D, int d_dtype,
              int64_t ld_d, cudaStream_t stream) {
-  using C = Cfg<KIND>;
   const int64_t group = KIND == kNVF4 ? 16 : 32;
   if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return BSP_ERR_INVALID_ARG;
   if (d_dtype != BSP_OUT_BF16 && d_dtype != BSP_OUT_F32) return BSP_ERR_INVALID_ARG;
@@ -414,38 +645,31 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   if (!A || !B || !sfA || !sfB || !D) return BSP_ERR_INVALID_ARG;
   const int64_t esize = d_dtype == BSP_OUT_F32 ? 4 : 2;
   if (!aligned16(A) || !aligned16(B) || !aligned16(sfA) || !aligned16(sfB) || !aligned16(D) ||
-      (bias && !aligned16(bias)) || (ld_d * esize) % 16 != 0 || (row_scale && (reinterpret_cast<uintptr_t>(row_scale) & 3u)) ||
-      (alpha && (reinterpret_cast<uintptr_t>(alpha) & 3u)))
+      (bias && !aligned16(bias)) || (ld_d * esize) % 16 != 0 ||
+      (row_scale && (reinterpret_cast<uintptr_t>(row_scale) & 3u)) || (alpha && (reinterpret_cast<uintptr_t>(alpha) & 3u)))
     return BSP_ERR_ALIGNMENT;
   DeviceInfo dev;
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
   if (encode_tiled_fn() == nullptr) return BSP_ERR_CUDA;
 
+  const bool pair = M >= BSP_GEMM_PAIR_MIN_M;
   const int64_t row_bytes = KIND == kNVF4 ? K / 2 : K;
   const int64_t tiles_per_band = round_up(K / group, 4) / 4;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
-  if ((st = encode_operand(&tmA, A, M, row_bytes, C::BM)) != BSP_OK) return st;
-  if ((st = encode_operand(&tmB, B, N, row_bytes, C::BN)) != BSP_OK) return st;
-  if ((st = encode_scales(&tmSFA, sfA, ceil_div(M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
-  if ((st = encode_scales(&tmSFB, sfB, ceil_div(N, 128), tiles_per_band, C::ATOMS, 2)) != BSP_OK) return st;
+  if ((st = encode_operand(&tmA, A, M, row_bytes, 128)) != BSP_OK) return st;
+  if ((st = encode_operand(&tmB, B, N, row_bytes, pair ? 128 : 256)) != BSP_OK) return st;
+  if ((st = encode_scales(&tmSFA, sfA, ceil_div(M, 128), tiles_per_band, KIND == kNVF4 ? 4 : 1, 1)) != BSP_OK)
+    return st;
+  if ((st = encode_scales(&tmSFB, sfB, ceil_div(N, 128), tiles_per_band, KIND == kNVF4 ? 4 : 1, 2)) != BSP_OK)
+    return st;
   if ((st = encode_output(&tmD, D, M, N, ld_d, d_dtype == BSP_OUT_F32)) != BSP_OK) return st;
-
-  static bool attr_set[64] = {};
-  if (!attr_set[dev.id]) {
-    if (cudaFuncSetAttribute(blockscaled_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return launch_status();
-    attr_set[dev.id] = true;
-  }
 
   GemmParams p;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.num_m = static_cast<int>(ceil_div(M, C::BM));
-  p.num_n = static_cast<int>(ceil_div(N, C::BN));
-  p.num_kb = static_cast<int>(ceil_div(row_bytes, C::ROW_BYTES));
+  p.num_kb = static_cast<int>(ceil_div(row_bytes, 128));
   p.alpha = alpha;
   p.row_scale = row_scale;
   p.bias = bias;
@@ -453,10 +677,8 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   p.ld_d = ld_d;
   p.out_f32 = d_dtype == BSP_OUT_F32;
   p.err = dev.err_word;
-  const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
-  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  blockscaled_gemm_kernel<KIND><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, tmD, p);
-  return launch_status();
+  return pair ? launch_gemm<KIND, 2>(dev, tmA, tmB, tmSFA, tmSFB, tmD, p, stream)
+              : launch_gemm<KIND, 1>(dev, tmA, tmB, tmSFA, tmSFB, tmD, p, stream);
 }
 
 }  // namespace

@@ -14,10 +14,11 @@
 //   ((r/128)*(cols4/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4
 //
 // HBM-bound streaming kernels.  Fast paths (K % 64 == 0 for NVFP4, K % 128 ==
-// 0 for MXFP8): one warp per row, every lane one 16-byte bf16 load per step
-// (a warp step reads 512 contiguous bytes), group amax by warp shuffles in the
-// integer domain (|bf16| bit patterns order like their values), hardware cvt
-// with round-to-nearest-even and saturation, 4-byte code stores, and the four
+// 0 for MXFP8): one warp per row, one lane per group (16 or 32 elements read
+// with adjacent 16-byte loads, so a warp step reads 1 or 2 KB of one row and
+// the scale arithmetic is paid once per group), group amax in the integer
+// domain (|bf16| bit patterns order like their values), hardware cvt with
+// round-to-nearest-even and saturation, 8- or 32-byte code stores, and the four
 // scale bytes of a 128x4 tile row gathered by shuffles into one 4-byte store.
 #include "bsp_device.cuh"
 #include "bsp_internal.h"
@@ -26,7 +27,7 @@ namespace bsp {
 namespace {
 
 constexpr int kQuantThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;  // warp steps in flight per row iteration
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
@@ -107,28 +108,33 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
 // NVFP4, K % 64 == 0.  Rows [M, Mp) are the scale padding (zeros).
 // A "quad" is 64 elements = one 128x4 tile row = 8 lanes; a warp step is 4 quads.
 // ---------------------------------------------------------------------------
-// U warp steps of one row: U 16-byte loads in flight per lane, then the
-// quantization of each.  `lp`, `cp`, `sp` point at this lane's first element,
-// code word and (for j == 0) scale word of the first step.
+// One lane quantizes one group of 16 (two adjacent 16-byte loads); a warp step
+// covers 32 groups = 512 elements of one row.  U steps: 2U loads in flight per
+// lane, then the quantization of each.  `lp`, `cp`, `sp` point at this lane's
+// group, its 8 code bytes, and (for lanes with g % 4 == 0) its 4 scale bytes in
+// the first step.
 template <int U>
 __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uint8_t* sp, bool live, float gs,
-                                            uint32_t j) {
-  uint4 v[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) v[u] = live ? ldg16(lp + u * 256) : make_uint4(0u, 0u, 0u, 0u);
+                                            bool store_sf) {
+  uint4 v[U][2];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    uint32_t mag = max_mag8(v[u]);
-    mag = max(mag, __shfl_xor_sync(kFull, mag, 1));  // lanes 2g, 2g+1 hold group g
+    v[u][0] = live ? ldg16(lp + u * 512) : make_uint4(0u, 0u, 0u, 0u);
+    v[u][1] = live ? ldg16(lp + u * 512 + 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
     uint32_t sfb;
     float inv;
-    nvfp4_scale(mag, gs, sfb, inv);
-    const uint32_t word = nvfp4_codes8(v[u], inv);
-    const uint32_t s1 = __shfl_down_sync(kFull, sfb, 2);
-    const uint32_t s2 = __shfl_down_sync(kFull, sfb, 4);
-    const uint32_t s3 = __shfl_down_sync(kFull, sfb, 6);
-    if (live) *reinterpret_cast<uint32_t*>(cp + u * 128) = word;
-    if (j == 0) *reinterpret_cast<uint32_t*>(sp + u * 2048) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    nvfp4_scale(max(max_mag8(v[u][0]), max_mag8(v[u][1])), gs, sfb, inv);
+    uint2 w;
+    w.x = nvfp4_codes8(v[u][0], inv);
+    w.y = nvfp4_codes8(v[u][1], inv);
+    const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
+    const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
+    const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
+    if (live) *reinterpret_cast<uint2*>(cp + u * 256) = w;
+    if (store_sf) *reinterpret_cast<uint32_t*>(sp + u * 4096) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
   }
 }
 
@@ -137,32 +143,31 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
   const uint32_t lane = lane_id();
-  const uint32_t sub = lane >> 3, j = lane & 7u;
-  const int64_t quads = K >> 6;
-  const int64_t steps = quads >> 2;  // full warp steps (4 quads) per row
-  const int64_t rem = quads & 3;     // quads of a last, partial step
+  const int64_t groups = K >> 4;
+  const int64_t steps = groups >> 5;  // full warp steps (32 groups) per row
+  const int64_t rem = groups & 31;    // groups of a last, partial step (a multiple of 4)
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+  const bool quad_lead = (lane & 3u) == 0u;
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const bool live = r < M;
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
     if (kPerRow && live) gs = row_scale_pass(row, K, r, row_gs, row_inv);
-    // this lane's element, code word and scale word in the row's first step
-    const uint16_t* lp = row + sub * 64 + j * 8;
-    uint8_t* cp = codes + r * (K >> 1) + sub * 32 + j * 4;
-    uint8_t* sp = sf + sf_row_base(r, quads) + sub * 512;
+    // group g = 32 * step + lane: elements 16 g, code bytes 8 g, scale tile g / 4
+    const uint16_t* lp = row + lane * 16;
+    uint8_t* cp = codes + r * (K >> 1) + lane * 8;
+    uint8_t* sp = sf + sf_row_base(r, groups >> 2) + (lane >> 2) * 512;
     int64_t st = 0;
     for (; st + kUnroll <= steps; st += kUnroll)
-      nvfp4_steps<kUnroll>(lp + st * 256, cp + st * 128, sp + st * 2048, live, gs, j);
-    for (; st < steps; ++st) nvfp4_steps<1>(lp + st * 256, cp + st * 128, sp + st * 2048, live, gs, j);
+      nvfp4_steps<kUnroll>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
+    for (; st < steps; ++st) nvfp4_steps<1>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
     if (rem) {
-      // last partial step: quads beyond the row end are predicated off
-      const bool in = sub < rem;
-      nvfp4_steps<1>(in ? lp + st * 256 : lp, in ? cp + st * 128 : cp, in ? sp + st * 2048 : sp, live && in, gs,
-                     in ? j : 1u);
+      const bool in = lane < rem;  // groups beyond the row end are predicated off
+      nvfp4_steps<1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * 4096 : sp, live && in, gs,
+                     in && quad_lead);
     }
   }
 }
@@ -231,50 +236,59 @@ __device__ __forceinline__ uint2 mx_elems8(const uint4& v, float mul) {
   return o;
 }
 
-// K % 128 == 0: a quad is 128 elements (4 groups of 32, one 128x4 tile row) =
-// 16 lanes; a warp step is 2 quads.
+// K % 128 == 0: one lane quantizes one group of 32 (four adjacent 16-byte
+// loads); a warp step covers 32 groups = 1024 elements of one row.
+template <int U>
+__device__ __forceinline__ void mxfp8_steps(const uint16_t* lp, uint8_t* qp, uint8_t* sp, bool live, bool store_sf) {
+  uint4 v[U][4];
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[u][i] = live ? ldg16(lp + u * 1024 + i * 8) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const uint32_t mag = max(max(max_mag8(v[u][0]), max_mag8(v[u][1])), max(max_mag8(v[u][2]), max_mag8(v[u][3])));
+    uint32_t sfb;
+    float mul;
+    mx_scale(mag, sfb, mul);
+    const uint2 o0 = mx_elems8(v[u][0], mul), o1 = mx_elems8(v[u][1], mul);
+    const uint2 o2 = mx_elems8(v[u][2], mul), o3 = mx_elems8(v[u][3], mul);
+    const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
+    const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
+    const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
+    if (live) {
+      *reinterpret_cast<uint4*>(qp + u * 1024) = make_uint4(o0.x, o0.y, o1.x, o1.y);
+      *reinterpret_cast<uint4*>(qp + u * 1024 + 16) = make_uint4(o2.x, o2.y, o3.x, o3.y);
+    }
+    if (store_sf) *reinterpret_cast<uint32_t*>(sp + u * 4096) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
 __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_k128_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                                           int64_t Mp, int64_t K, int64_t ld_x,
                                                                           uint8_t* __restrict__ q,
                                                                           uint8_t* __restrict__ sf) {
   const uint32_t lane = lane_id();
-  const uint32_t sub = lane >> 4, j = lane & 15u;
-  const int64_t quads = K >> 7;
+  const int64_t groups = K >> 5;
+  const int64_t steps = groups >> 5;
+  const int64_t rem = groups & 31;  // a multiple of 4
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const bool quad_lead = (lane & 3u) == 0u;
+  constexpr int kU = 2;
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const bool live = r < M;
-    const uint16_t* row = x + r * ld_x;
-    uint8_t* qrow = q + r * K;
-    const int64_t sfb_row = sf_row_base(r, quads);
-    for (int64_t q0 = 0; q0 < quads; q0 += 2 * kUnroll) {
-      uint4 v[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t qq = q0 + 2 * u + sub;
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (live && qq < quads) v[u] = ldg16(row + qq * 128 + j * 8);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t qq = q0 + 2 * u + sub;
-        uint32_t mag = max_mag8(v[u]);
-        mag = max(mag, __shfl_xor_sync(kFull, mag, 1));
-        mag = max(mag, __shfl_xor_sync(kFull, mag, 2));  // lanes 4g..4g+3 hold group g
-        uint32_t sfb;
-        float mul;
-        mx_scale(mag, sfb, mul);
-        const uint2 o = mx_elems8(v[u], mul);
-        const uint32_t s1 = __shfl_down_sync(kFull, sfb, 4);
-        const uint32_t s2 = __shfl_down_sync(kFull, sfb, 8);
-        const uint32_t s3 = __shfl_down_sync(kFull, sfb, 12);
-        if (qq < quads) {
-          if (live) *reinterpret_cast<uint2*>(qrow + qq * 128 + j * 8) = o;
-          if (j == 0)
-            *reinterpret_cast<uint32_t*>(sf + sfb_row + qq * 512) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
-        }
-      }
+    const uint16_t* lp = x + r * ld_x + lane * 32;
+    uint8_t* qp = q + r * K + lane * 32;
+    uint8_t* sp = sf + sf_row_base(r, groups >> 2) + (lane >> 2) * 512;
+    int64_t st = 0;
+    for (; st + kU <= steps; st += kU) mxfp8_steps<kU>(lp + st * 1024, qp + st * 1024, sp + st * 4096, live, quad_lead);
+    for (; st < steps; ++st) mxfp8_steps<1>(lp + st * 1024, qp + st * 1024, sp + st * 4096, live, quad_lead);
+    if (rem) {
+      const bool in = lane < rem;
+      mxfp8_steps<1>(in ? lp + st * 1024 : lp, in ? qp + st * 1024 : qp, in ? sp + st * 4096 : sp, live && in,
+                     in && quad_lead);
     }
   }
 }
