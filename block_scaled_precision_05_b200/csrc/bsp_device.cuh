@@ -125,15 +125,28 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                : "memory");
 }
 
+// L2 policy that marks lines for early eviction (streamed outputs).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// Same as tma_store_2d with an L2 cache policy.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
-// Waits until at most `pending` (0 or 1) committed bulk stores are still
-// reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_allow(int pending) {
-  if (pending <= 0)
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-  else
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+// Waits until at most N committed bulk stores are still reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_allow() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 // Waits until every committed bulk store has completed.

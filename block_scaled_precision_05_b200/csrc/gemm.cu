@@ -64,6 +64,15 @@
 #ifndef BSP_GEMM_STAGING_BUFS
 #define BSP_GEMM_STAGING_BUFS 1
 #endif
+// Rasterisation: m-blocks per tile group; 0 chooses by operand size (see
+// launch_gemm).
+#ifndef BSP_GEMM_GROUP_M
+#define BSP_GEMM_GROUP_M 0
+#endif
+// 1: output TMA stores carry an L2 evict-first hint.
+#ifndef BSP_GEMM_STORE_EVICT_FIRST
+#define BSP_GEMM_STORE_EVICT_FIRST 1
+#endif
 // Smallest M for which the 2-SM (CTA pair) form is used.  Off by default: on
 // B200 the pair form measured slower than the 1-SM form with scale-factor
 // warps on every workload here (its per-stage handshakes cross the pair).
@@ -119,6 +128,7 @@ struct Cfg {
 struct GemmParams {
   int M, N, K;
   int num_m, num_n, num_kb;
+  int group_m;  // m-blocks per rasterisation group
   const float* alpha;
   const float* row_scale;
   const uint16_t* bias;
@@ -128,10 +138,10 @@ struct GemmParams {
   uint32_t* err;
 };
 
-// Output tile t -> (m block, n block), grouped 16 m-blocks at a time so that
-// concurrently running CTAs share A and B panels in L2.
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
-  constexpr int G = 16;
+// Output tile t -> (m block, n block), grouped G m-blocks at a time so that
+// concurrently running CTAs share A and B panels in L2 (G is chosen on the host
+// so that a group's A panel stays well inside L2 while B streams past it).
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int G, int& mb, int& nb) {
   const int per_group = G * num_n;
   const int g = t / per_group;
   const int first = g * G;
@@ -217,7 +227,7 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
       bool ok = true;
       for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
         int mb, nb;
-        tile_coords(t, p.num_m, p.num_n, mb, nb);
+        tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
         const int a_row = mb * C::TILE_M + static_cast<int>(rank) * C::BM;
         const int b_row = nb * C::BN + static_cast<int>(rank) * C::B_ROWS;
         const int a_band = mb * CG + static_cast<int>(rank);
@@ -400,20 +410,24 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     constexpr int W_BF16 = 16, W_F32 = 8;
     const uint32_t swz = (lane >> 2) & 1u;
     uint32_t store_seq = 0;  // TMA stores issued by this warp (picks the staging buffer)
+    const uint64_t evict_first = l2_policy_evict_first();
 
     // Writes 32 bytes of this lane's row into the staging buffer, then one
     // lane stores the 32 x 32-byte box at (n0, row0).
     auto stage_and_store = [&](int n0, int row0, uint4 lo, uint4 hi) {
       if constexpr (C::EPI_TMA) {
         uint8_t* buf = stage_buf + (store_seq % C::STAGING_BUFS) * 1024;
-        if (lane == 0) bulk_wait_read_allow(C::STAGING_BUFS - 1);
+        if (lane == 0) bulk_wait_read_allow<C::STAGING_BUFS - 1>();
         __syncwarp();
         *reinterpret_cast<uint4*>(buf + lane * 32 + 16 * (0u ^ swz)) = lo;
         *reinterpret_cast<uint4*>(buf + lane * 32 + 16 * (1u ^ swz)) = hi;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmD, buf, n0, row0);
+          if constexpr (BSP_GEMM_STORE_EVICT_FIRST)
+            tma_store_2d_hint(&tmD, buf, n0, row0, evict_first);
+          else
+            tma_store_2d(&tmD, buf, n0, row0);
           bulk_commit_group();
         }
         ++store_seq;
@@ -442,7 +456,7 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     int it = 0;
     for (int t = first_tile; t < num_tiles; t += tile_step, ++it) {
       int mb, nb;
-      tile_coords(t, p.num_m, p.num_n, mb, nb);
+      tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
       if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
         *abort_flag = 1u;
         raise_error(p.err, kErrTimeout);
@@ -627,6 +641,24 @@ int launch_gemm(const DeviceInfo& dev, const CUtensorMap& tmA, const CUtensorMap
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+  }
+  if (BSP_GEMM_GROUP_M > 0) {
+    p.group_m = BSP_GEMM_GROUP_M < p.num_m ? BSP_GEMM_GROUP_M : p.num_m;
+  } else {
+    // B (codes and scales) well inside L2: group just enough m-blocks that the
+    // CTAs running at once cover every n-block, so each A panel is read from
+    // DRAM once.  Large B: about 24 MiB of A per group, so the group's A panel
+    // stays in L2 while B streams past it once per group.
+    const int64_t b_bytes = static_cast<int64_t>(p.N) * p.num_kb * 128 * 17 / 16;
+    int64_t g;
+    if (b_bytes < (32ll << 20)) {
+      g = ceil_div(2ll * max_clusters[dev.id], p.num_n);
+    } else {
+      const int64_t a_panel = static_cast<int64_t>(C::TILE_M) * p.num_kb * 128 * 17 / 16;
+      g = (24ll << 20) / (a_panel > 0 ? a_panel : 1);
+    }
+    g = g < 8 ? 8 : g;
+    p.group_m = static_cast<int>(g < p.num_m ? g : p.num_m);
   }
   if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmSFA, tmSFB, tmD, p) != cudaSuccess) return launch_status();
   return launch_status();

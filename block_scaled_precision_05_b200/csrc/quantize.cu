@@ -94,7 +94,12 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
                                                 float* row_gs, float* row_inv) {
   const uint32_t lane = lane_id();
   uint32_t m = 0;
-  for (int64_t c = lane * 8; c < K; c += 256) m = max(m, max_sane_mag8(ldg16(row + c)));
+  int64_t c = lane * 8;
+  for (; c + 768 < K; c += 1024) {  // four independent 16-byte loads in flight
+    const uint4 a = ldg16(row + c), b = ldg16(row + c + 256), d = ldg16(row + c + 512), e = ldg16(row + c + 768);
+    m = max(max(m, max(max_sane_mag8(a), max_sane_mag8(b))), max(max_sane_mag8(d), max_sane_mag8(e)));
+  }
+  for (; c < K; c += 256) m = max(m, max_sane_mag8(ldg16(row + c)));
   m = warp_max(m);
   const float gs = global_scale_from_mag(m);
   if (lane == 0) {
@@ -135,6 +140,57 @@ __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uin
     const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
     if (live) *reinterpret_cast<uint2*>(cp + u * 256) = w;
     if (store_sf) *reinterpret_cast<uint32_t*>(sp + u * 4096) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
+// Per-tensor scale, short rows (K = 512 * S, S <= 3): a warp quantizes two rows
+// per iteration with all 4S 16-byte loads of both rows issued up front, so the
+// memory pipeline stays full although each row is only S warp steps long.
+template <int S>
+__global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const float* __restrict__ gs_ptr,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  constexpr int64_t K = 512 * S;
+  const uint32_t lane = lane_id();
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float gs = __ldg(gs_ptr);
+  const bool quad_lead = (lane & 3u) == 0u;
+  for (int64_t r0 = 2 * warp; r0 < Mp; r0 += 2 * nwarps) {
+    uint4 v[2][S][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t r = r0 + h;
+      const bool live = r < M;
+      const uint16_t* lp = x + r * ld_x + lane * 16;
+#pragma unroll
+      for (int st = 0; st < S; ++st) {
+        v[h][st][0] = live ? ldg16(lp + st * 512) : make_uint4(0u, 0u, 0u, 0u);
+        v[h][st][1] = live ? ldg16(lp + st * 512 + 8) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t r = r0 + h;
+      if (r >= Mp) break;
+      const bool live = r < M;
+      uint8_t* cp = codes + r * (K >> 1) + lane * 8;
+      uint8_t* sp = sf + sf_row_base(r, K >> 6) + (lane >> 2) * 512;
+#pragma unroll
+      for (int st = 0; st < S; ++st) {
+        uint32_t sfb;
+        float inv;
+        nvfp4_scale(max(max_mag8(v[h][st][0]), max_mag8(v[h][st][1])), gs, sfb, inv);
+        uint2 w;
+        w.x = nvfp4_codes8(v[h][st][0], inv);
+        w.y = nvfp4_codes8(v[h][st][1], inv);
+        const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
+        const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
+        const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
+        if (live) *reinterpret_cast<uint2*>(cp + st * 256) = w;
+        if (quad_lead) *reinterpret_cast<uint32_t*>(sp + st * 4096) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
+    }
   }
 }
 
@@ -423,6 +479,15 @@ int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const 
       auto k = nvfp4_quant_k64_kernel<true>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
                                                                  codes, sf);
+    } else if (K == 1024 || K == 1536) {
+      const int64_t pairs = ceil_div(Mp, 2);
+      if (K == 1024) {
+        auto k = nvfp4_quant_short_kernel<2>;
+        k<<<grid_for_rows(dev, k, pairs), kQuantThreads, 0, stream>>>(x, M, Mp, ld_x, global_sf, codes, sf);
+      } else {
+        auto k = nvfp4_quant_short_kernel<3>;
+        k<<<grid_for_rows(dev, k, pairs), kQuantThreads, 0, stream>>>(x, M, Mp, ld_x, global_sf, codes, sf);
+      }
     } else {
       auto k = nvfp4_quant_k64_kernel<false>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
