@@ -73,6 +73,10 @@
 #ifndef BSP_GEMM_STORE_EVICT_FIRST
 #define BSP_GEMM_STORE_EVICT_FIRST 1
 #endif
+// Largest M for which the transposed skinny-M kernel is used.
+#ifndef BSP_GEMM_SKINNY_MAX_M
+#define BSP_GEMM_SKINNY_MAX_M 64
+#endif
 // Smallest M for which the 2-SM (CTA pair) form is used.  Off by default: on
 // B200 the pair form measured slower than the 1-SM form with scale-factor
 // warps on every workload here (its per-stage handshakes cross the pair).
@@ -555,6 +559,303 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Skinny M (M <= 128, e.g. per-token decode-like batches against a large
+// weight): the GEMM is bound by streaming the weight from HBM, so it is run
+// transposed, D^T = B A^T.  The weight is the MMA's 128-row operand (tiles of
+// 128 weight rows, so ~N/128 CTAs stream disjoint weight panels through a deep
+// pipeline of small stages) and the BNA <= 128 activation rows are the MMA's N
+// side.  Same roles as the main kernel: warp 0 producer, warp 1 MMA issuer,
+// warps 2-5 scale factors, warps 6-9 epilogue (lane = output column n, one
+// TMEM column per activation row m; each warp writes 32 consecutive n of a
+// row of D per instruction).
+// ---------------------------------------------------------------------------
+template <int KIND, int BNA>
+struct SkCfg {
+  static constexpr int BM = 128;                         // weight rows per tile (MMA M)
+  static constexpr int ROW_BYTES = 128;
+  static constexpr int MMAS = 4;
+  static constexpr int ATOMS = KIND == kNVF4 ? 4 : 1;
+  static constexpr int W_BYTES = BM * ROW_BYTES;
+  static constexpr int X_BYTES = BNA * ROW_BYTES;
+  static constexpr int SFW_BYTES = ATOMS * 512;
+  static constexpr int SFX_BYTES = ATOMS * 512;         // one 128-row band of activation scales
+  static constexpr int TX_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
+  static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
+  static constexpr int SFW_COLS = ATOMS * 4;
+  static constexpr int SFX_COLS = ATOMS * 4;            // N <= 128: one column group per K step
+  static constexpr int SF_COLS = SFW_COLS + SFX_COLS;
+  static constexpr int ACC_COLS = BNA;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SF_WARPS = 4, EPI_WARPS = 4;
+  static constexpr int THREADS = 64 + (SF_WARPS + EPI_WARPS) * 32;
+  static constexpr int FIXED_BYTES = 1024 + 256;
+  static constexpr int STAGES =
+      cmin(cmin((232448 - FIXED_BYTES) / STAGE_BYTES, (TMEM_COLS - ACC_COLS) / SF_COLS), 8);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+  static_assert(STAGES >= 2 && ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "budget");
+};
+
+template <int KIND, int BNA>
+__global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
+    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmSFW, const __grid_constant__ CUtensorMap tmSFX,
+                       const GemmParams p) {
+  using C = SkCfg<KIND, BNA>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* sf_ready = empty + C::STAGES;
+  uint64_t* acc_full = sf_ready + C::STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], C::SF_WARPS);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, C::EPI_WARPS);
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmSFW);
+    prefetch_tensormap(&tmSFX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  // tile t: weight panel nb = t % num_n (fastest), activation block mb = t / num_n
+  const int num_tiles = p.num_m * p.num_n;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued[C::STAGES];
+      for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int nb = t % p.num_n, mb = t / p.num_n;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+          tma_load_2d(st, &tmW, &full[stage], kb * C::ROW_BYTES, nb * C::BM);
+          tma_load_2d(st + C::W_BYTES, &tmX, &full[stage], kb * C::ROW_BYTES, mb * BNA);
+          tma_load_3d(st + C::W_BYTES + C::X_BYTES, &tmSFW, &full[stage], 0, kb * C::ATOMS, nb);
+          tma_load_3d(st + C::W_BYTES + C::X_BYTES + C::SFW_BYTES, &tmSFX, &full[stage], 0, kb * C::ATOMS,
+                      (mb * BNA) >> 7);
+          ++issued[stage];
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1u;
+        raise_error(p.err, kErrTimeout);
+      }
+      for (int s = 0; s < C::STAGES; ++s)
+        if (issued[s] && !mbar_wait(&full[s], (issued[s] - 1u) & 1u, nullptr)) raise_error(p.err, kErrTimeout);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+        if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sfw_t = tmem + C::ACC_COLS + stage * C::SF_COLS;
+          const uint32_t sfx_t = sfw_t + C::SFW_COLS;
+          const uint64_t wdesc = desc_kmajor_sw128(sbase);
+          const uint64_t xdesc = desc_kmajor_sw128(sbase + C::W_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::MMAS; ++kk) {
+            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (KIND == kNVF4)
+              tc_mma_nvf4(tmem, wdesc + 2u * kk, xdesc + 2u * kk, idesc_nvf4(C::BM, BNA), sfw_t + 4u * kk,
+                          sfx_t + 4u * kk, accumulate);
+            else
+              tc_mma_mxf8(tmem, wdesc + 2u * kk, xdesc + 2u * kk, idesc_mxf8(C::BM, BNA, static_cast<uint32_t>(kk)),
+                          sfw_t, sfx_t, accumulate);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+      }
+      if (!ok) {
+        *abort_flag = 1u;
+        raise_error(p.err, kErrTimeout);
+      }
+      tc_commit(drain);
+      if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
+    }
+  } else if (warp < 2 + C::SF_WARPS) {
+    // scale warps: stage tiles -> replicated scale columns (see the main kernel)
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* sfw_s = smem + stage * C::STAGE_BYTES + C::W_BYTES + C::X_BYTES;
+        const uint8_t* sfx_s = sfw_s + C::SFW_BYTES;
+        uint32_t v[C::SF_COLS];
+#pragma unroll
+        for (int a = 0; a < C::ATOMS; ++a) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sfw_s + 512 * a + lane * 16);
+          const uint4 x = *reinterpret_cast<const uint4*>(sfx_s + 512 * a + lane * 16);
+          v[4 * a + 0] = w.x;
+          v[4 * a + 1] = w.y;
+          v[4 * a + 2] = w.z;
+          v[4 * a + 3] = w.w;
+          v[C::SFW_COLS + 4 * a + 0] = x.x;
+          v[C::SFW_COLS + 4 * a + 1] = x.y;
+          v[C::SFW_COLS + 4 * a + 2] = x.z;
+          v[C::SFW_COLS + 4 * a + 3] = x.w;
+        }
+        const uint32_t taddr = tmem + lane_base + C::ACC_COLS + stage * C::SF_COLS;
+        if constexpr (C::SF_COLS == 32) {
+          tmem_st_16cols(taddr, v);
+          tmem_st_16cols(taddr + 16, v + 16);
+        } else {
+          static_assert(C::SF_COLS == 8, "scale columns per stage");
+          tmem_st_8cols(taddr, v);
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready[stage]);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1u;
+      raise_error(p.err, kErrTimeout);
+    }
+  } else {
+    // epilogue: lane = output column n, TMEM column c = activation row m
+    const int q = warp & 3;
+    const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int nb = t % p.num_n, mb = t / p.num_n;
+      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
+        *abort_flag = 1u;
+        raise_error(p.err, kErrTimeout);
+        break;
+      }
+      tc_fence_after_sync();
+      const int n = nb * C::BM + q * 32 + static_cast<int>(lane);
+      const bool n_ok = n < p.N;
+      float b = 0.0f;
+      if (p.bias != nullptr && n_ok) b = bf16_bits_to_f32(p.bias[n]);
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BNA; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_16cols(taddr + static_cast<uint32_t>(c0), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int m = mb * BNA + c0 + i;
+          if (m >= p.M) break;
+          float scale = alpha;
+          if (p.row_scale != nullptr) scale = __fmul_rn(alpha, __ldg(p.row_scale + m));
+          const float y = __fmaf_rn(__uint_as_float(r[i]), scale, b);
+          if (n_ok) {
+            if (p.out_f32)
+              static_cast<float*>(p.D)[static_cast<int64_t>(m) * p.ld_d + n] = y;
+            else
+              static_cast<__nv_bfloat16*>(p.D)[static_cast<int64_t>(m) * p.ld_d + n] = __float2bfloat16_rn(y);
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows);
+int encode_scales(CUtensorMap* m, const void* base, int64_t bands, int64_t tiles_per_band, int atoms, int box_bands);
+
+template <int KIND, int BNA>
+int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                  int64_t row_bytes, int64_t tiles_per_band, GemmParams p, cudaStream_t stream) {
+  using C = SkCfg<KIND, BNA>;
+  auto kernel = skinny_gemm_kernel<KIND, BNA>;
+  static bool attr_set[64] = {};
+  if (!attr_set[dev.id]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return launch_status();
+    attr_set[dev.id] = true;
+  }
+  CUtensorMap tmW, tmX, tmSFW, tmSFX;
+  int st;
+  if ((st = encode_operand(&tmW, B, p.N, row_bytes, C::BM)) != BSP_OK) return st;
+  if ((st = encode_operand(&tmX, A, p.M, row_bytes, BNA)) != BSP_OK) return st;
+  if ((st = encode_scales(&tmSFW, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
+  if ((st = encode_scales(&tmSFX, sfA, ceil_div(p.M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
+  p.num_n = static_cast<int>(ceil_div(p.N, C::BM));
+  p.num_m = static_cast<int>(ceil_div(p.M, BNA));
+  const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmW, tmX, tmSFW, tmSFX, p);
+  return launch_status();
+}
+
 // Row-major uint8 matrix [rows, row_bytes], boxes of box_rows x 128 bytes, 128-byte swizzle.
 int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
@@ -686,6 +987,7 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   if (encode_tiled_fn() == nullptr) return BSP_ERR_CUDA;
 
   const bool pair = M >= BSP_GEMM_PAIR_MIN_M;
+  const bool skinny = M <= BSP_GEMM_SKINNY_MAX_M;
   const int64_t row_bytes = KIND == kNVF4 ? K / 2 : K;
   const int64_t tiles_per_band = round_up(K / group, 4) / 4;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
@@ -709,6 +1011,12 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   p.ld_d = ld_d;
   p.out_f32 = d_dtype == BSP_OUT_F32;
   p.err = dev.err_word;
+  if (skinny) {
+    if (M <= 16) return launch_skinny<KIND, 16>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    if (M <= 32) return launch_skinny<KIND, 32>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    if (M <= 64) return launch_skinny<KIND, 64>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    return launch_skinny<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+  }
   return pair ? launch_gemm<KIND, 2>(dev, tmA, tmB, tmSFA, tmSFB, tmD, p, stream)
               : launch_gemm<KIND, 1>(dev, tmA, tmB, tmSFA, tmSFB, tmD, p, stream);
 }
