@@ -287,6 +287,18 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Same for rows of 64 or 128 bytes (TMA's 64- or 128-byte swizzle); 8-row
+// groups are 8 * row_bytes apart.
+__device__ __forceinline__ uint64_t desc_kmajor_swizzled(uint32_t saddr, int row_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((8u * row_bytes) >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(row_bytes == 128 ? 2u : 4u) << 61;  // 128-byte : 64-byte swizzle
+  return d;
+}
+
 // Descriptor of a 32-row x 16-byte scale-factor block (rows 16 bytes apart,
 // no swizzle), the source of tc_cp_32x128b_warpx4.
 __device__ __forceinline__ uint64_t desc_sf_block(uint32_t saddr) {

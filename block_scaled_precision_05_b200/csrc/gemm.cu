@@ -77,6 +77,11 @@
 #ifndef BSP_GEMM_SKINNY_MAX_M
 #define BSP_GEMM_SKINNY_MAX_M 64
 #endif
+// K bytes per operand row per pipeline stage of the NVFP4 main kernel (128 or
+// 64; 64 halves the stage size and doubles the stage count).
+#ifndef BSP_GEMM_NVF4_ROW_BYTES
+#define BSP_GEMM_NVF4_ROW_BYTES 128
+#endif
 // Smallest M for which the 2-SM (CTA pair) form is used.  Off by default: on
 // B200 the pair form measured slower than the 1-SM form with scale-factor
 // warps on every workload here (its per-stage handshakes cross the pair).
@@ -97,9 +102,10 @@ struct Cfg {
   static constexpr int BN = 256;                        // output tile columns
   static constexpr int TILE_M = BM * CG;                // output tile rows
   static constexpr int B_ROWS = BN / CG;                // rows of B each CTA loads
-  static constexpr int ROW_BYTES = 128;                 // K bytes per operand row per stage
-  static constexpr int MMAS = 4;                        // per stage, 32 bytes of K each
-  static constexpr int ATOMS = KIND == kNVF4 ? 4 : 1;   // 128x4 scale tiles per 128 rows per stage
+  static constexpr int ROW_BYTES = KIND == kNVF4 ? BSP_GEMM_NVF4_ROW_BYTES : 128;  // K bytes per row per stage
+  static constexpr int MMAS = ROW_BYTES / 32;                                    // per stage, 32 bytes of K each
+  static constexpr int ATOMS = KIND == kNVF4 ? ROW_BYTES / 32 : 1;  // 128x4 scale tiles per 128 rows per stage
+  static_assert(ROW_BYTES == 128 || ROW_BYTES == 64, "stage row width");
   static constexpr int A_BYTES = BM * ROW_BYTES;
   static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
   static constexpr int SFA_BYTES = ATOMS * 512;
@@ -284,8 +290,8 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
           const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sfa_t = tmem + C::ACC_COLS + stage * C::SF_COLS;
           const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-          const uint64_t adesc = desc_kmajor_sw128(sbase);
-          const uint64_t bdesc = desc_kmajor_sw128(sbase + C::A_BYTES);
+          const uint64_t adesc = desc_kmajor_swizzled(sbase, C::ROW_BYTES);
+          const uint64_t bdesc = desc_kmajor_swizzled(sbase + C::A_BYTES, C::ROW_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::MMAS; ++kk) {
             const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
@@ -376,6 +382,9 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
           tmem_st_16cols(taddr, v);
           tmem_st_16cols(taddr + 16, v + 16);
           tmem_st_16cols(taddr + 32, v + 32);
+        } else if constexpr (C::SF_COLS == 24) {
+          tmem_st_16cols(taddr, v);
+          tmem_st_8cols(taddr + 16, v + 16);
         } else {
           static_assert(C::SF_COLS == 12, "scale columns per stage");
           tmem_st_4cols(taddr, v);
@@ -828,7 +837,8 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
   }
 }
 
-int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows);
+int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows,
+                   int box_bytes = 128);
 int encode_scales(CUtensorMap* m, const void* base, int64_t bands, int64_t tiles_per_band, int atoms, int box_bands);
 
 template <int KIND, int BNA>
@@ -856,14 +866,16 @@ int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, c
   return launch_status();
 }
 
-// Row-major uint8 matrix [rows, row_bytes], boxes of box_rows x 128 bytes, 128-byte swizzle.
-int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+// Row-major uint8 matrix [rows, row_bytes], boxes of box_rows x box_bytes (128
+// or 64) with the matching TMA swizzle.
+int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows, int box_bytes) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1u, 1u};
   CUresult r = encode_tiled_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
-                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
@@ -896,9 +908,17 @@ int encode_output(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
 }
 
 template <int KIND, int CG>
-int launch_gemm(const DeviceInfo& dev, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSFA,
-                const CUtensorMap& tmSFB, const CUtensorMap& tmD, GemmParams p, cudaStream_t stream) {
+int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                int64_t row_bytes, int64_t tiles_per_band, const CUtensorMap& tmD, GemmParams p,
+                cudaStream_t stream) {
   using C = Cfg<KIND, CG>;
+  CUtensorMap tmA, tmB, tmSFA, tmSFB;
+  int st;
+  if ((st = encode_operand(&tmA, A, p.M, row_bytes, C::BM, C::ROW_BYTES)) != BSP_OK) return st;
+  if ((st = encode_operand(&tmB, B, p.N, row_bytes, C::B_ROWS, C::ROW_BYTES)) != BSP_OK) return st;
+  if ((st = encode_scales(&tmSFA, sfA, ceil_div(p.M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
+  if ((st = encode_scales(&tmSFB, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, 2)) != BSP_OK) return st;
+  p.num_kb = static_cast<int>(ceil_div(row_bytes, C::ROW_BYTES));
   auto kernel = blockscaled_gemm_kernel<KIND, CG>;
   static bool attr_set[64] = {};
   static int max_clusters[64] = {};
@@ -950,12 +970,12 @@ int launch_gemm(const DeviceInfo& dev, const CUtensorMap& tmA, const CUtensorMap
     // CTAs running at once cover every n-block, so each A panel is read from
     // DRAM once.  Large B: about 24 MiB of A per group, so the group's A panel
     // stays in L2 while B streams past it once per group.
-    const int64_t b_bytes = static_cast<int64_t>(p.N) * p.num_kb * 128 * 17 / 16;
+    const int64_t b_bytes = static_cast<int64_t>(p.N) * row_bytes * 17 / 16;
     int64_t g;
     if (b_bytes < (32ll << 20)) {
       g = ceil_div(2ll * max_clusters[dev.id], p.num_n);
     } else {
-      const int64_t a_panel = static_cast<int64_t>(C::TILE_M) * p.num_kb * 128 * 17 / 16;
+      const int64_t a_panel = static_cast<int64_t>(C::TILE_M) * row_bytes * 17 / 16;
       g = (24ll << 20) / (a_panel > 0 ? a_panel : 1);
     }
     g = g < 8 ? 8 : g;
@@ -990,13 +1010,7 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   const bool skinny = M <= BSP_GEMM_SKINNY_MAX_M;
   const int64_t row_bytes = KIND == kNVF4 ? K / 2 : K;
   const int64_t tiles_per_band = round_up(K / group, 4) / 4;
-  CUtensorMap tmA, tmB, tmSFA, tmSFB, tmD;
-  if ((st = encode_operand(&tmA, A, M, row_bytes, 128)) != BSP_OK) return st;
-  if ((st = encode_operand(&tmB, B, N, row_bytes, pair ? 128 : 256)) != BSP_OK) return st;
-  if ((st = encode_scales(&tmSFA, sfA, ceil_div(M, 128), tiles_per_band, KIND == kNVF4 ? 4 : 1, 1)) != BSP_OK)
-    return st;
-  if ((st = encode_scales(&tmSFB, sfB, ceil_div(N, 128), tiles_per_band, KIND == kNVF4 ? 4 : 1, 2)) != BSP_OK)
-    return st;
+  CUtensorMap tmD;
   if ((st = encode_output(&tmD, D, M, N, ld_d, d_dtype == BSP_OUT_F32)) != BSP_OK) return st;
 
   GemmParams p;
@@ -1017,8 +1031,8 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
     if (M <= 64) return launch_skinny<KIND, 64>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
     return launch_skinny<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
   }
-  return pair ? launch_gemm<KIND, 2>(dev, tmA, tmB, tmSFA, tmSFB, tmD, p, stream)
-              : launch_gemm<KIND, 1>(dev, tmA, tmB, tmSFA, tmSFB, tmD, p, stream);
+  return pair ? launch_gemm<KIND, 2>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream)
+              : launch_gemm<KIND, 1>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
 }
 
 }  // namespace
