@@ -194,6 +194,78 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
   }
 }
 
+// Per-row (per-token) scale, K % 64 == 0 and K <= 16 * 256 * kRowG: one block
+// of 256 threads per row.  Thread t holds groups t, t+256, ... of the row in
+// registers (two adjacent 16-byte loads each, all issued at once), the row
+// amax is reduced through shared memory, and the row is quantized from the
+// registers, so each row costs one memory round trip.
+constexpr int kRowG = 4;
+
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, float* __restrict__ row_gs,
+    float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  __shared__ uint32_t red[kQuantThreads / 32];
+  __shared__ float gs_sh;
+  const uint32_t lane = lane_id();
+  const int t = static_cast<int>(threadIdx.x);
+  const int groups = static_cast<int>(K >> 4);
+  const int64_t tiles_per_band = groups >> 2;
+  for (int64_t r = blockIdx.x; r < Mp; r += gridDim.x) {
+    const bool live = r < M;
+    const uint16_t* row = x + r * ld_x;
+    uint4 v[kRowG][2];
+    uint32_t mag = 0;
+#pragma unroll
+    for (int i = 0; i < kRowG; ++i) {
+      const int g = t + i * kQuantThreads;
+      const bool in = live && g < groups;
+      v[i][0] = in ? ldg16(row + g * 16) : make_uint4(0u, 0u, 0u, 0u);
+      v[i][1] = in ? ldg16(row + g * 16 + 8) : make_uint4(0u, 0u, 0u, 0u);
+      mag = max(mag, max(max_sane_mag8(v[i][0]), max_sane_mag8(v[i][1])));
+    }
+    mag = warp_max(mag);
+    if (lane == 0) red[threadIdx.x >> 5] = mag;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      uint32_t m = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0u;
+      m = warp_max(m);
+      if (threadIdx.x == 0) {
+        const float gs = global_scale_from_mag(m);
+        gs_sh = gs;
+        if (live) {
+          if (row_gs) row_gs[r] = gs;
+          if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
+        }
+      }
+    }
+    __syncthreads();
+    const float gs = gs_sh;
+    uint8_t* crow = codes + r * (K >> 1);
+    const int64_t sbase = sf_row_base(r, tiles_per_band);
+#pragma unroll
+    for (int i = 0; i < kRowG; ++i) {
+      const int g = t + i * kQuantThreads;
+      // within a warp, groups are consecutive, so lanes 4j..4j+3 own one scale word
+      if (i * kQuantThreads + (t & ~31) >= groups) break;  // warp-uniform
+      uint32_t sfb;
+      float inv;
+      nvfp4_scale(max(max_mag8(v[i][0]), max_mag8(v[i][1])), gs, sfb, inv);
+      uint2 w;
+      w.x = nvfp4_codes8(v[i][0], inv);
+      w.y = nvfp4_codes8(v[i][1], inv);
+      const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
+      const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
+      const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
+      if (g < groups) {
+        if (live) *reinterpret_cast<uint2*>(crow + g * 8) = w;
+        if ((g & 3) == 0)
+          *reinterpret_cast<uint32_t*>(sf + sbase + (g >> 2) * 512) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
+    }
+    __syncthreads();  // red / gs_sh are reused by the next row
+  }
+}
+
 template <bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
@@ -475,7 +547,22 @@ int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const 
   const int64_t Mp = round_up(M, 128);
   const bool per_row = sf_mode == BSP_SF_PER_ROW;
   if (K % 64 == 0) {
-    if (per_row) {
+    int rowblock_cap = 0;  // rows the block-per-row kernel keeps resident at once
+    if (per_row && K <= 16 * kQuantThreads * kRowG) {
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_quant_rowblock_kernel, kQuantThreads, 0) !=
+              cudaSuccess ||
+          per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+      }
+      rowblock_cap = dev.sm_count * per_sm;
+    }
+    if (per_row && Mp <= rowblock_cap) {
+      // few rows: one block per row, all rows in one wave, one memory round trip
+      nvfp4_quant_rowblock_kernel<<<static_cast<int>(Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, row_gs,
+                                                                                      row_inv_gs, codes, sf);
+    } else if (per_row) {
       auto k = nvfp4_quant_k64_kernel<true>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
                                                                  codes, sf);
