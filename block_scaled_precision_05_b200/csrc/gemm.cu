@@ -470,44 +470,43 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     for (int t = first_tile; t < num_tiles; t += tile_step, ++it) {
       int mb, nb;
       tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
-      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
-        *abort_flag = 1u;
-        raise_error(p.err, kErrTimeout);
-        break;
-      }
-      tc_fence_after_sync();
+      // Row scale and bias are fetched before the accumulator is ready.  The
+      // bias of this warp's 128 columns is spread over the lanes, four columns
+      // each (lane j: columns col0 + 4j .. 4j + 3), and handed to every lane by
+      // shuffles while the accumulator is read.
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * C::EPI_COLS);
       const int row0 = mb * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
       const int row = row0 + static_cast<int>(lane);
       float scale = alpha;
       if (p.row_scale != nullptr && row < p.M) scale = __fmul_rn(alpha, __ldg(p.row_scale + row));
       const int col0 = nb * C::BN + half * C::EPI_COLS;
+      uint2 bias4 = make_uint2(0u, 0u);
+      if (p.bias != nullptr && col0 + 4 * static_cast<int>(lane) < p.N)
+        bias4 = __ldg(reinterpret_cast<const uint2*>(p.bias + col0 + 4 * static_cast<int>(lane)));
+      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
+        *abort_flag = 1u;
+        raise_error(p.err, kErrTimeout);
+        break;
+      }
+      tc_fence_after_sync();
 
       if (!p.out_f32) {
-        // bf16: read all 128 columns, applying the epilogue and packing as they
-        // arrive, release tensor memory, then store from registers.
+        // bf16: read the 128 columns 32 at a time, applying the epilogue and
+        // packing as they arrive, release tensor memory, then store from
+        // registers.
         uint32_t packed[C::EPI_COLS / 2];
 #pragma unroll
-        for (int k = 0; k < C::EPI_COLS / 16; ++k) {
-          uint32_t r[16];
-          tmem_ld_16cols(taddr + 16u * k, r);
-          uint32_t bw[8];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int n = col0 + 16 * k + 8 * h;
-            uint4 bv = make_uint4(0u, 0u, 0u, 0u);
-            if (p.bias != nullptr && n < p.N) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
-            bw[4 * h + 0] = bv.x;
-            bw[4 * h + 1] = bv.y;
-            bw[4 * h + 2] = bv.z;
-            bw[4 * h + 3] = bv.w;
-          }
+        for (int c = 0; c < C::EPI_COLS / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32cols(taddr + 32u * c, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            packed[8 * k + i] =
-                pack_bf16x2(__fmaf_rn(__uint_as_float(r[2 * i]), scale, bf16_bits_to_f32(bw[i] & 0xFFFFu)),
-                            __fmaf_rn(__uint_as_float(r[2 * i + 1]), scale, bf16_bits_to_f32(bw[i] >> 16)));
+          for (int i = 0; i < 16; ++i) {
+            // columns 32c + 2i, 2i + 1 are held by lane 8c + i/2
+            const uint32_t bw = __shfl_sync(0xFFFFFFFFu, (i & 1) ? bias4.y : bias4.x, 8 * c + (i >> 1));
+            packed[16 * c + i] = pack_bf16x2(__fmaf_rn(__uint_as_float(r[2 * i]), scale, bf16_bits_to_f32(bw & 0xFFFFu)),
+                                             __fmaf_rn(__uint_as_float(r[2 * i + 1]), scale, bf16_bits_to_f32(bw >> 16)));
+          }
         }
         release_accumulator();
 #pragma unroll
