@@ -224,6 +224,9 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // Set-up above overlaps the previous kernel under programmatic launch; every
+  // global access below comes after its completion.
+  grid_dependency_wait();
   const int num_tiles = p.num_m * p.num_n;
   const int first_tile = static_cast<int>(blockIdx.x) / CG;
   const int tile_step = static_cast<int>(gridDim.x) / CG;
@@ -649,6 +652,7 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();  // as in the main kernel
   // tile t: weight panel nb = t % num_n (fastest), activation block mb = t / num_n
   const int num_tiles = p.num_m * p.num_n;
 
@@ -861,7 +865,17 @@ int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, c
   p.num_m = static_cast<int>(ceil_div(p.M, BNA));
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
   const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmW, tmX, tmSFW, tmSFX, p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // as in launch_gemm
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, tmW, tmX, tmSFW, tmSFX, p) != cudaSuccess) return launch_status();
   return launch_status();
 }
 
@@ -949,18 +963,22 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
   const int units = static_cast<int>(tiles < max_clusters[dev.id] ? tiles : max_clusters[dev.id]);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
+  // programmatic launch: the kernel's set-up overlaps the previous kernel's tail
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if constexpr (CG == 2) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
   if (BSP_GEMM_GROUP_M > 0) {
     p.group_m = BSP_GEMM_GROUP_M < p.num_m ? BSP_GEMM_GROUP_M : p.num_m;

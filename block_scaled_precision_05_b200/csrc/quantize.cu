@@ -150,6 +150,7 @@ template <int S>
 __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const float* __restrict__ gs_ptr,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   constexpr int64_t K = 512 * S;
   const uint32_t lane = lane_id();
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -204,6 +205,7 @@ constexpr int kRowG = 4;
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, float* __restrict__ row_gs,
     float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   __shared__ uint32_t red[kQuantThreads / 32];
   __shared__ float gs_sh;
   const uint32_t lane = lane_id();
@@ -270,6 +272,7 @@ template <bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   const uint32_t lane = lane_id();
   const int64_t groups = K >> 4;
   const int64_t steps = groups >> 5;  // full warp steps (32 groups) per row
@@ -307,6 +310,7 @@ template <bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   const uint32_t lane = lane_id();
   const int64_t groups = K >> 4, cols4 = (groups + 3) & ~int64_t(3);
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -396,6 +400,7 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_k128_kernel(const u
                                                                           int64_t Mp, int64_t K, int64_t ld_x,
                                                                           uint8_t* __restrict__ q,
                                                                           uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   const uint32_t lane = lane_id();
   const int64_t groups = K >> 5;
   const int64_t steps = groups >> 5;
@@ -426,6 +431,7 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_generic_kernel(cons
                                                                              int64_t M, int64_t Mp, int64_t K,
                                                                              int64_t ld_x, uint8_t* __restrict__ q,
                                                                              uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   const uint32_t lane = lane_id();
   const int64_t groups = K >> 5, cols4 = (groups + 3) & ~int64_t(3);
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
