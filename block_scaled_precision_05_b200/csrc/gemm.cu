@@ -10,14 +10,14 @@
 //   vllm-omni mxfp8_config.py, NPUMxfp8LinearMethod._quant_matmul.
 //
 // Design (persistent, one CTA per SM, warp-specialised):
-//   warp 0      TMA producer: per stage, this CTA's 128 rows of A and its rows
+//   warp 0      TMA producer: per stage, the tile's 128 rows of A and BN rows
 //               of B (128 bytes of K each, 128-byte swizzle) plus the matching
 //               128x4 scale tiles, into shared memory; completion is counted on
-//               an mbarrier (the pair leader's one in the 2-SM form).
-//   warp 1      MMA issuer (one thread of the leader CTA): once a stage's data
-//               and scale factors are ready, issues four block-scaled MMAs
-//               (K = 64 fp4 / 32 fp8 each) accumulating fp32 in tensor memory,
-//               and releases the stage (tcgen05.commit).
+//               the stage's mbarrier.
+//   warp 1      MMA issuer (one thread): once a stage's data and scale factors
+//               are ready, issues four block-scaled MMAs (K = 64 fp4 / 32 fp8
+//               each) accumulating fp32 in tensor memory, and releases the
+//               stage (tcgen05.commit).
 //   warps 10-13 scale-factor warps, one per 32-lane quarter of tensor memory:
 //               read the stage's 128x4 scale tiles from shared memory and write
 //               them into the stage's scale columns of tensor memory
@@ -26,24 +26,21 @@
 //               scale traffic off the tensor pipe lets it overlap the MMAs of
 //               the previous stages.
 //   warps 2..9  epilogue, two warps per 32-lane quarter of tensor memory, each
-//               owning 128 accumulator columns: read them into registers
-//               (tcgen05.ld), hand the accumulator back to the MMA warp at once
-//               (so the next tile's MMAs overlap this tile's stores), apply
-//               alpha, row scale and bias in fp32, round once, stage 32 rows x
-//               32 bytes in swizzled shared memory and write them with TMA
-//               stores (full 32-byte sectors; rows/columns past M/N clipped).
+//               owning half of the tile's accumulator columns: read them into
+//               registers (tcgen05.ld), hand the accumulator back to the MMA
+//               warp at once, apply alpha, row scale and bias in fp32, round
+//               once, stage 32 rows x 32 bytes in swizzled shared memory and
+//               write them with TMA stores (full 32-byte sectors; rows/columns
+//               past M/N clipped).
 //   (roles by warp index: 0 producer, 1 MMA, 2-9 epilogue, 10-13 scales)
-// Two forms:
-//   1-SM   128 x 256 output tiles, each CTA loads 128 rows of A and 256 of B.
-//   2-SM   256 x 256 output tiles per cluster of two CTAs (cta_group::2): each
-//          CTA loads its own 128 rows of A and 128 of the 256 rows of B, and
-//          the B scale tiles of all 256 rows; the leader's MMAs read both CTAs'
-//          shared memory and write each CTA's 128 accumulator rows into its own
-//          tensor memory; both CTAs' scale warps report to the leader.  Half
-//          the B traffic per SM and smaller stages.  (No TMA multicast.)
-// Tensor memory: columns [0, 256) accumulator; then, per pipeline stage, the
-// stage's scale factors (a scale column may only be rewritten once the stage's
-// MMAs have completed, which the stage's empty barrier already guarantees).
+// Output tiles are 128 x 256 with one accumulator (256 tensor-memory
+// columns): two accumulators of 256 columns would leave no room for the stages'
+// scale factors, and 128-column tiles measured slower (an N = 128 block-scaled
+// MMA takes about as long to issue as an N = 256 one), so the next tile's MMAs
+// wait until the epilogue has read the accumulator, which it does first thing.
+// Tensor memory: the accumulator; then, per pipeline stage, the stage's
+// scale factors (a scale column may only be rewritten once the stage's MMAs
+// have completed, which the stage's empty barrier already guarantees).
 // Ragged M / N / K edges: TMA fills out-of-range rows, K bytes and scale tiles
 // with zeros (zero codes times zero scales add nothing); TMA stores clip.
 // Every wait is bounded; a wait that runs out raises the device error word and
@@ -82,12 +79,6 @@
 #ifndef BSP_GEMM_NVF4_ROW_BYTES
 #define BSP_GEMM_NVF4_ROW_BYTES 128
 #endif
-// Smallest M for which the 2-SM (CTA pair) form is used.  Off by default: on
-// B200 the pair form measured slower than the 1-SM form with scale-factor
-// warps on every workload here (its per-stage handshakes cross the pair).
-#ifndef BSP_GEMM_PAIR_MIN_M
-#define BSP_GEMM_PAIR_MIN_M (1 << 30)
-#endif
 
 namespace bsp {
 namespace {
@@ -96,26 +87,25 @@ enum Kind : int { kNVF4 = 0, kMXF8 = 1 };
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
-template <int KIND, int CG>
+template <int KIND>
 struct Cfg {
-  static constexpr int BM = 128;                        // accumulator rows per CTA
+  static constexpr int BM = 128;                        // accumulator rows (tensor-memory lanes)
   static constexpr int BN = 256;                        // output tile columns
-  static constexpr int TILE_M = BM * CG;                // output tile rows
-  static constexpr int B_ROWS = BN / CG;                // rows of B each CTA loads
   static constexpr int ROW_BYTES = KIND == kNVF4 ? BSP_GEMM_NVF4_ROW_BYTES : 128;  // K bytes per row per stage
   static constexpr int MMAS = ROW_BYTES / 32;                                    // per stage, 32 bytes of K each
   static constexpr int ATOMS = KIND == kNVF4 ? ROW_BYTES / 32 : 1;  // 128x4 scale tiles per 128 rows per stage
   static_assert(ROW_BYTES == 128 || ROW_BYTES == 64, "stage row width");
+  static constexpr int B_BANDS = BN / 128;              // 128-row bands of B per tile
   static constexpr int A_BYTES = BM * ROW_BYTES;
-  static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
+  static constexpr int B_BYTES = BN * ROW_BYTES;
   static constexpr int SFA_BYTES = ATOMS * 512;
-  static constexpr int SFB_BYTES = 2 * ATOMS * 512;     // both 128-row bands of the 256 columns
-  static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // per CTA per stage
+  static constexpr int SFB_BYTES = B_BANDS * ATOMS * 512;
+  static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // per stage
   static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
-  static constexpr int SFA_COLS = ATOMS * 4;
-  static constexpr int SFB_COLS = ATOMS * 8;
-  static constexpr int SF_COLS = SFA_COLS + SFB_COLS;   // 48 (fp4) / 12 (fp8) per stage
-  static constexpr int ACC_COLS = BN;
+  static constexpr int SFA_COLS = ATOMS * 4;            // per stage, replicated layout
+  static constexpr int SFB_COLS = ATOMS * 4 * B_BANDS;
+  static constexpr int SF_COLS = SFA_COLS + SFB_COLS;   // 48 (fp4) / 12 (fp8)
+  static constexpr int SFB_COLS_PER_MMA = KIND == kNVF4 ? 4 * B_BANDS : 0;  // fp8: one scale set per stage
   static constexpr int TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_COLS = BN / 2;  // accumulator columns per epilogue warp
@@ -127,12 +117,14 @@ struct Cfg {
   static constexpr int THREADS = 64 + (EPI_WARPS + SF_WARPS) * 32;
   static constexpr int BAR_BYTES = 256;
   static constexpr int FIXED_BYTES = EPI_WARPS * STAGING_BYTES + 1024 + BAR_BYTES;
+  static constexpr int ACC_COLS = BN;  // one fp32 accumulator
   static constexpr int STAGES = cmin(cmin((232448 - FIXED_BYTES) / STAGE_BYTES, (TMEM_COLS - ACC_COLS) / SF_COLS),
                                      BSP_GEMM_STAGES);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
   static_assert(STAGES >= 2, "pipeline depth");
   static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(3 * STAGES + 3 <= BAR_BYTES / 8 - 1, "barrier space");
 };
 
 struct GemmParams {
@@ -166,12 +158,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int KIND, int CG>
-__global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
+template <int KIND>
+__global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
     blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                             const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-  using C = Cfg<KIND, CG>;
+  using C = Cfg<KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
@@ -186,17 +178,15 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
-  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;  // position in the CTA pair
-  const bool leader = rank == 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_ready[s], C::SF_WARPS * CG);  // the scale warps of both CTAs report to the leader
+      mbar_init(&sf_ready[s], C::SF_WARPS);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, C::EPI_WARPS * CG);  // the epilogue warps of both CTAs arrive on the leader's
+    mbar_init(acc_empty, C::EPI_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -209,27 +199,19 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     prefetch_tensormap(&tmD);
   }
   if (warp == 1) {
-    if constexpr (CG == 2) {
-      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, C::TMEM_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before_sync();
-  if constexpr (CG == 2)
-    cluster_sync();  // the peer's barriers are initialised before anyone signals them
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   // Set-up above overlaps the previous kernel under programmatic launch; every
   // global access below comes after its completion.
   grid_dependency_wait();
   const int num_tiles = p.num_m * p.num_n;
-  const int first_tile = static_cast<int>(blockIdx.x) / CG;
-  const int tile_step = static_cast<int>(gridDim.x) / CG;
+  const int first_tile = static_cast<int>(blockIdx.x);
+  const int tile_step = static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -241,9 +223,6 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
       for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
         int mb, nb;
         tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
-        const int a_row = mb * C::TILE_M + static_cast<int>(rank) * C::BM;
-        const int b_row = nb * C::BN + static_cast<int>(rank) * C::B_ROWS;
-        const int a_band = mb * CG + static_cast<int>(rank);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -251,10 +230,11 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
           }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-          tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, a_row);
-          tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, b_row);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, a_band);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, &full[stage], 0, kb * C::ATOMS, nb * 2);
+          tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, mb * C::BM);
+          tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, nb * C::BN);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, mb);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, &full[stage], 0, kb * C::ATOMS,
+                      nb * C::B_BANDS);
           ++issued[stage];
           if (++stage == C::STAGES) {
             stage = 0;
@@ -272,19 +252,19 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && leader) {
+    if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int it = 0;
-      constexpr uint16_t kPair = 0x3;
       for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
+        // the epilogue has read the previous tile's accumulator
         if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          // the scale warps signal after their CTA's stage landed and its scales are in tensor memory
+          // the scale warps signal after the stage landed and its scales are in tensor memory
           if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -299,55 +279,33 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
           for (int kk = 0; kk < C::MMAS; ++kk) {
             const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
             // 32 bytes of K per MMA: advance the start address by 32 >> 4.
-            if constexpr (KIND == kNVF4) {
-              const uint32_t idesc = idesc_nvf4(C::TILE_M, C::BN);
-              if constexpr (CG == 2)
-                tc_mma_nvf4_pair(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t + 4u * kk, sfb_t + 8u * kk,
-                                 accumulate);
-              else
-                tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t + 4u * kk, sfb_t + 8u * kk,
-                            accumulate);
-            } else {
-              const uint32_t idesc = idesc_mxf8(C::TILE_M, C::BN, static_cast<uint32_t>(kk));
-              if constexpr (CG == 2)
-                tc_mma_mxf8_pair(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t, sfb_t, accumulate);
-              else
-                tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t, sfb_t, accumulate);
-            }
+            if constexpr (KIND == kNVF4)
+              tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_nvf4(C::BM, C::BN), sfa_t + 4u * kk,
+                          sfb_t + static_cast<uint32_t>(C::SFB_COLS_PER_MMA * kk), accumulate);
+            else
+              tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8(C::BM, C::BN, static_cast<uint32_t>(kk)),
+                          sfa_t, sfb_t, accumulate);
           }
-          if constexpr (CG == 2)
-            tc_commit_pair(&empty[stage], kPair);
-          else
-            tc_commit(&empty[stage]);
+          tc_commit(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        if constexpr (CG == 2)
-          tc_commit_pair(acc_full, kPair);
-        else
-          tc_commit(acc_full);
+        tc_commit(acc_full);
       }
       if (!ok) {
         *abort_flag = 1u;
         raise_error(p.err, kErrTimeout);
       }
       // No MMA may still be running when tensor memory is freed.
-      if constexpr (CG == 2)
-        tc_commit_pair(drain, kPair);
-      else
-        tc_commit(drain);
-      if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
-    } else if (lane == 0) {
-      // pair follower: its MMAs are issued by the leader; wait for their end
+      tc_commit(drain);
       if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
     }
   } else if (warp >= C::FIRST_SF_WARP) {
     // ------------------------------------------------------------ scale factors
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t sf_ready_leader = CG == 2 ? mapa_shared(smem_u32(sf_ready), 0u) : smem_u32(sf_ready);
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
@@ -358,7 +316,8 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
         }
         // Line `lane` of each 512-byte scale tile (the scales of rows lane,
         // lane+32, lane+64, lane+96 for 4 K-groups) becomes 4 consecutive
-        // columns of this lane; every lane quarter gets the same copy.
+        // columns of this lane; every lane quarter gets the same copy.  Per
+        // MMA step: 4 columns of A scales, then 4 per 128-row band of B.
         const uint8_t* sfa_s = smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
         const uint8_t* sfb_s = sfa_s + C::SFA_BYTES;
         uint32_t v[C::SF_COLS];
@@ -371,37 +330,35 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
           v[4 * a + 3] = w.w;
         }
 #pragma unroll
-        for (int rt = 0; rt < 2; ++rt)
+        for (int rt = 0; rt < C::B_BANDS; ++rt)
 #pragma unroll
           for (int a = 0; a < C::ATOMS; ++a) {
             const uint4 w = *reinterpret_cast<const uint4*>(sfb_s + 512 * (rt * C::ATOMS + a) + lane * 16);
-            v[C::SFA_COLS + 8 * a + 4 * rt + 0] = w.x;
-            v[C::SFA_COLS + 8 * a + 4 * rt + 1] = w.y;
-            v[C::SFA_COLS + 8 * a + 4 * rt + 2] = w.z;
-            v[C::SFA_COLS + 8 * a + 4 * rt + 3] = w.w;
+            constexpr int kPerAtom = 4 * C::B_BANDS;
+            v[C::SFA_COLS + kPerAtom * a + 4 * rt + 0] = w.x;
+            v[C::SFA_COLS + kPerAtom * a + 4 * rt + 1] = w.y;
+            v[C::SFA_COLS + kPerAtom * a + 4 * rt + 2] = w.z;
+            v[C::SFA_COLS + kPerAtom * a + 4 * rt + 3] = w.w;
           }
         const uint32_t taddr = tmem + lane_base + C::ACC_COLS + stage * C::SF_COLS;
         if constexpr (C::SF_COLS == 48) {
           tmem_st_16cols(taddr, v);
           tmem_st_16cols(taddr + 16, v + 16);
           tmem_st_16cols(taddr + 32, v + 32);
-        } else if constexpr (C::SF_COLS == 24) {
+        } else if constexpr (C::SF_COLS == 32) {
           tmem_st_16cols(taddr, v);
-          tmem_st_8cols(taddr + 16, v + 16);
-        } else {
-          static_assert(C::SF_COLS == 12, "scale columns per stage");
+          tmem_st_16cols(taddr + 16, v + 16);
+        } else if constexpr (C::SF_COLS == 12) {
           tmem_st_4cols(taddr, v);
           tmem_st_8cols(taddr + 4, v + 4);
+        } else {
+          static_assert(C::SF_COLS == 8, "scale columns per stage");
+          tmem_st_8cols(taddr, v);
         }
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) {
-          if constexpr (CG == 2)
-            mbar_arrive_cluster(sf_ready_leader + 8u * stage);
-          else
-            mbar_arrive(&sf_ready[stage]);
-        }
+        if (lane == 0) mbar_arrive(&sf_ready[stage]);
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -416,10 +373,9 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;   // 0..7
     const int q = warp & 3;    // tensor-memory lane quarter this warp may read
-    const int half = ew >> 2;  // which 128 accumulator columns
+    const int half = ew >> 2;  // which half of the tile's columns
     uint8_t* stage_buf = staging + ew * C::STAGING_BYTES;
     const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
-    const uint32_t acc_empty_leader = CG == 2 ? mapa_shared(smem_u32(acc_empty), 0u) : smem_u32(acc_empty);
     // One staging row = 32 bytes = W output elements; the two 16-byte halves
     // are swapped on rows 4..7 of every 8 (TMA's 32-byte swizzle), which keeps
     // the 32 lanes' shared-memory writes at the minimum of 4 wavefronts.
@@ -461,12 +417,7 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
     auto release_accumulator = [&]() {
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) {
-        if constexpr (CG == 2)
-          mbar_arrive_cluster(acc_empty_leader);
-        else
-          mbar_arrive(acc_empty);
-      }
+      if (lane == 0) mbar_arrive(acc_empty);
     };
 
     int it = 0;
@@ -474,11 +425,11 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
       int mb, nb;
       tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
       // Row scale and bias are fetched before the accumulator is ready.  The
-      // bias of this warp's 128 columns is spread over the lanes, four columns
-      // each (lane j: columns col0 + 4j .. 4j + 3), and handed to every lane by
+      // bias of this warp's columns is spread over the lanes, four columns each
+      // (lane j: columns col0 + 4j .. 4j + 3), and handed to every lane by
       // shuffles while the accumulator is read.
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * C::EPI_COLS);
-      const int row0 = mb * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
+      const int row0 = mb * C::BM + q * 32;
       const int row = row0 + static_cast<int>(lane);
       float scale = alpha;
       if (p.row_scale != nullptr && row < p.M) scale = __fmul_rn(alpha, __ldg(p.row_scale + row));
@@ -494,7 +445,7 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
       tc_fence_after_sync();
 
       if (!p.out_f32) {
-        // bf16: read the 128 columns 32 at a time, applying the epilogue and
+        // bf16: read the columns 32 at a time, applying the epilogue and
         // packing as they arrive, release tensor memory, then store from
         // registers.
         uint32_t packed[C::EPI_COLS / 2];
@@ -559,14 +510,10 @@ __global__ void __launch_bounds__(Cfg<KIND, CG>::THREADS, 1)
 
   tc_fence_before_sync();
   __syncthreads();
-  if constexpr (CG == 2) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    if constexpr (CG == 2)
-      tmem_dealloc_pair(tmem, C::TMEM_COLS);
-    else
-      tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -920,51 +867,33 @@ int encode_output(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
 
-template <int KIND, int CG>
+template <int KIND>
 int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                 int64_t row_bytes, int64_t tiles_per_band, const CUtensorMap& tmD, GemmParams p,
                 cudaStream_t stream) {
-  using C = Cfg<KIND, CG>;
+  using C = Cfg<KIND>;
   CUtensorMap tmA, tmB, tmSFA, tmSFB;
   int st;
   if ((st = encode_operand(&tmA, A, p.M, row_bytes, C::BM, C::ROW_BYTES)) != BSP_OK) return st;
-  if ((st = encode_operand(&tmB, B, p.N, row_bytes, C::B_ROWS, C::ROW_BYTES)) != BSP_OK) return st;
+  if ((st = encode_operand(&tmB, B, p.N, row_bytes, C::BN, C::ROW_BYTES)) != BSP_OK) return st;
   if ((st = encode_scales(&tmSFA, sfA, ceil_div(p.M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
-  if ((st = encode_scales(&tmSFB, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, 2)) != BSP_OK) return st;
+  if ((st = encode_scales(&tmSFB, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, C::B_BANDS)) != BSP_OK)
+    return st;
   p.num_kb = static_cast<int>(ceil_div(row_bytes, C::ROW_BYTES));
-  auto kernel = blockscaled_gemm_kernel<KIND, CG>;
+  auto kernel = blockscaled_gemm_kernel<KIND>;
   static bool attr_set[64] = {};
-  static int max_clusters[64] = {};
   if (!attr_set[dev.id]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return launch_status();
-    int units = dev.sm_count / CG;
-    if constexpr (CG == 2) {
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 2;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(2 * units, 1, 1);
-      cfg.blockDim = dim3(C::THREADS, 1, 1);
-      cfg.dynamicSmemBytes = C::SMEM_BYTES;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) units = n;
-      cudaGetLastError();
-    }
-    max_clusters[dev.id] = units;
     attr_set[dev.id] = true;
   }
-  p.num_m = static_cast<int>(ceil_div(p.M, C::TILE_M));
+  p.num_m = static_cast<int>(ceil_div(p.M, C::BM));
   p.num_n = static_cast<int>(ceil_div(p.N, C::BN));
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
-  const int units = static_cast<int>(tiles < max_clusters[dev.id] ? tiles : max_clusters[dev.id]);
+  const int ctas = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -973,13 +902,6 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if constexpr (CG == 2) {
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = 2;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.numAttrs = 2;
-  }
   if (BSP_GEMM_GROUP_M > 0) {
     p.group_m = BSP_GEMM_GROUP_M < p.num_m ? BSP_GEMM_GROUP_M : p.num_m;
   } else {
@@ -990,9 +912,9 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
     const int64_t b_bytes = static_cast<int64_t>(p.N) * row_bytes * 17 / 16;
     int64_t g;
     if (b_bytes < (32ll << 20)) {
-      g = ceil_div(2ll * max_clusters[dev.id], p.num_n);
+      g = ceil_div(2ll * ctas, p.num_n);
     } else {
-      const int64_t a_panel = static_cast<int64_t>(C::TILE_M) * row_bytes * 17 / 16;
+      const int64_t a_panel = static_cast<int64_t>(C::BM) * row_bytes * 17 / 16;
       g = (24ll << 20) / (a_panel > 0 ? a_panel : 1);
     }
     g = g < 8 ? 8 : g;
@@ -1023,7 +945,6 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   if (st != BSP_OK) return st;
   if (encode_tiled_fn() == nullptr) return BSP_ERR_CUDA;
 
-  const bool pair = M >= BSP_GEMM_PAIR_MIN_M;
   const bool skinny = M <= BSP_GEMM_SKINNY_MAX_M;
   const int64_t row_bytes = KIND == kNVF4 ? K / 2 : K;
   const int64_t tiles_per_band = round_up(K / group, 4) / 4;
@@ -1048,8 +969,7 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
     if (M <= 64) return launch_skinny<KIND, 64>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
     return launch_skinny<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
   }
-  return pair ? launch_gemm<KIND, 2>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream)
-              : launch_gemm<KIND, 1>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
+  return launch_gemm<KIND>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
 }
 
 }  // namespace
