@@ -741,28 +741,36 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int nb = t % p.num_n, mb = t / p.num_n;
+      const int n = nb * C::BM + q * 32 + static_cast<int>(lane);
+      const bool n_ok = n < p.N;
+      float b = 0.0f;
+      if (p.bias != nullptr && n_ok) b = bf16_bits_to_f32(p.bias[n]);
+      // alpha x row scale of this tile's activation rows, one row per lane,
+      // fetched before the accumulator is ready and handed out by shuffles
+      float rs[(BNA + 31) / 32];
+#pragma unroll
+      for (int j = 0; j < (BNA + 31) / 32; ++j) {
+        const int m = mb * BNA + 32 * j + static_cast<int>(lane);
+        rs[j] = (p.row_scale != nullptr && m < p.M) ? __fmul_rn(alpha, __ldg(p.row_scale + m)) : alpha;
+      }
       if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
         *abort_flag = 1u;
         raise_error(p.err, kErrTimeout);
         break;
       }
       tc_fence_after_sync();
-      const int n = nb * C::BM + q * 32 + static_cast<int>(lane);
-      const bool n_ok = n < p.N;
-      float b = 0.0f;
-      if (p.bias != nullptr && n_ok) b = bf16_bits_to_f32(p.bias[n]);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
+#pragma unroll
       for (int c0 = 0; c0 < BNA; c0 += 16) {
+        if (mb * BNA + c0 >= p.M) break;  // warp-uniform
         uint32_t r[16];
         tmem_ld_16cols(taddr + static_cast<uint32_t>(c0), r);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int m = mb * BNA + c0 + i;
-          if (m >= p.M) break;
-          float scale = alpha;
-          if (p.row_scale != nullptr) scale = __fmul_rn(alpha, __ldg(p.row_scale + m));
+          if (m >= p.M) break;  // warp-uniform
+          const float scale = __shfl_sync(0xFFFFFFFFu, rs[(c0 + i) >> 5], (c0 + i) & 31);
           const float y = __fmaf_rn(__uint_as_float(r[i]), scale, b);
           if (n_ok) {
             if (p.out_f32)

@@ -41,21 +41,39 @@ __device__ __forceinline__ uint32_t sane_mag(uint32_t b16) {
   return m;
 }
 
-__device__ __forceinline__ uint32_t max_mag8(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
-  return m;
+__device__ __forceinline__ __nv_bfloat162 u32_as_bf162(uint32_t u) {
+  __nv_bfloat162 r;
+  memcpy(&r, &u, 4);
+  return r;
 }
 
-__device__ __forceinline__ uint32_t max_sane_mag8(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m = max(m, max(sane_mag(w[i] & 0xFFFFu), sane_mag(w[i] >> 16)));
-  return m;
+// Packed maxima of |x| over the 8 bf16 of a 16-byte chunk (two lanes of 4),
+// with the packed bf16 max instruction, which ignores a NaN operand.
+__device__ __forceinline__ __nv_bfloat162 absmax8_x2(const uint4& v) {
+  const __nv_bfloat162 a = u32_as_bf162(v.x & 0x7FFF7FFFu), b = u32_as_bf162(v.y & 0x7FFF7FFFu);
+  const __nv_bfloat162 c = u32_as_bf162(v.z & 0x7FFF7FFFu), d = u32_as_bf162(v.w & 0x7FFF7FFFu);
+  return __hmax2(__hmax2(a, b), __hmax2(c, d));
 }
+
+// Bit pattern of the larger of the two packed maxima; NaN elements are
+// ignored (a group of NaNs only gives 0).  Values are non-negative, so bit
+// patterns order like the values.
+__device__ __forceinline__ uint32_t max_of_halves(__nv_bfloat162 m) {
+  const __nv_bfloat16 h = __hmax(__low2bfloat16(m), __high2bfloat16(m));
+  uint16_t u;
+  memcpy(&u, &h, 2);
+  return u > 0x7F80u ? 0u : static_cast<uint32_t>(u);
+}
+
+// amax bit pattern of one 16-element group (two 16-byte chunks).
+__device__ __forceinline__ uint32_t group_mag16(const uint4& a, const uint4& b) {
+  return max_of_halves(__hmax2(absmax8_x2(a), absmax8_x2(b)));
+}
+
+__device__ __forceinline__ uint32_t max_mag8(const uint4& v) { return max_of_halves(absmax8_x2(v)); }
+
+// As max_mag8, with +-inf counted as the largest finite bf16 (sane_mag).
+__device__ __forceinline__ uint32_t max_sane_mag8(const uint4& v) { return min(max_mag8(v), 0x7F7Fu); }
 
 __device__ __forceinline__ uint32_t warp_max(uint32_t m) {
 #pragma unroll
@@ -77,11 +95,14 @@ __device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sf
 }
 
 // Eight bf16 (one 16-byte chunk) times inv -> eight e2m1 codes in one word.
+// The products are fp32 multiplies, two per packed instruction.
 __device__ __forceinline__ uint32_t nvfp4_codes8(const uint4& v, float inv) {
-  return cvt_e2m1x8(__fmul_rn(bf16_bits_to_f32(v.x & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.x >> 16), inv),
-                    __fmul_rn(bf16_bits_to_f32(v.y & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.y >> 16), inv),
-                    __fmul_rn(bf16_bits_to_f32(v.z & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.z >> 16), inv),
-                    __fmul_rn(bf16_bits_to_f32(v.w & 0xFFFFu), inv), __fmul_rn(bf16_bits_to_f32(v.w >> 16), inv));
+  const float2 i2 = make_float2(inv, inv);
+  const float2 p0 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.x & 0xFFFFu), __uint_as_float(v.x & 0xFFFF0000u)), i2);
+  const float2 p1 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.y & 0xFFFFu), __uint_as_float(v.y & 0xFFFF0000u)), i2);
+  const float2 p2 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.z & 0xFFFFu), __uint_as_float(v.z & 0xFFFF0000u)), i2);
+  const float2 p3 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.w & 0xFFFFu), __uint_as_float(v.w & 0xFFFF0000u)), i2);
+  return cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y);
 }
 
 // Byte offset of the first of the four scale bytes (r, 4*tile_col .. +3).
@@ -131,7 +152,7 @@ __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uin
   for (int u = 0; u < U; ++u) {
     uint32_t sfb;
     float inv;
-    nvfp4_scale(max(max_mag8(v[u][0]), max_mag8(v[u][1])), gs, sfb, inv);
+    nvfp4_scale(group_mag16(v[u][0], v[u][1]), gs, sfb, inv);
     uint2 w;
     w.x = nvfp4_codes8(v[u][0], inv);
     w.y = nvfp4_codes8(v[u][1], inv);
@@ -181,7 +202,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
       for (int st = 0; st < S; ++st) {
         uint32_t sfb;
         float inv;
-        nvfp4_scale(max(max_mag8(v[h][st][0]), max_mag8(v[h][st][1])), gs, sfb, inv);
+        nvfp4_scale(group_mag16(v[h][st][0], v[h][st][1]), gs, sfb, inv);
         uint2 w;
         w.x = nvfp4_codes8(v[h][st][0], inv);
         w.y = nvfp4_codes8(v[h][st][1], inv);
@@ -251,7 +272,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
       if (i * kQuantThreads + (t & ~31) >= groups) break;  // warp-uniform
       uint32_t sfb;
       float inv;
-      nvfp4_scale(max(max_mag8(v[i][0]), max_mag8(v[i][1])), gs, sfb, inv);
+      nvfp4_scale(group_mag16(v[i][0], v[i][1]), gs, sfb, inv);
       uint2 w;
       w.x = nvfp4_codes8(v[i][0], inv);
       w.y = nvfp4_codes8(v[i][1], inv);
@@ -328,7 +349,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
       if (live && c < groups) {
         const uint4 a = ldg16(row + c * 16), b = ldg16(row + c * 16 + 8);
         float inv;
-        nvfp4_scale(max(max_mag8(a), max_mag8(b)), gs, sfb, inv);
+        nvfp4_scale(group_mag16(a, b), gs, sfb, inv);
         uint2 w;
         w.x = nvfp4_codes8(a, inv);
         w.y = nvfp4_codes8(b, inv);
@@ -379,7 +400,8 @@ __device__ __forceinline__ void mxfp8_steps(const uint16_t* lp, uint8_t* qp, uin
     for (int i = 0; i < 4; ++i) v[u][i] = live ? ldg16(lp + u * 1024 + i * 8) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    const uint32_t mag = max(max(max_mag8(v[u][0]), max_mag8(v[u][1])), max(max_mag8(v[u][2]), max_mag8(v[u][3])));
+    const uint32_t mag = max_of_halves(__hmax2(__hmax2(absmax8_x2(v[u][0]), absmax8_x2(v[u][1])),
+                                               __hmax2(absmax8_x2(v[u][2]), absmax8_x2(v[u][3]))));
     uint32_t sfb;
     float mul;
     mx_scale(mag, sfb, mul);
