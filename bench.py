@@ -196,7 +196,7 @@ def run_ours(args, rank, world, local_rank):
     W = up(lin.W)
     bias = None if lin.bias is None else up(lin.bias)
     if kind == "nvfp4":
-        layer = api.NVFP4Linear(W, bias, per_token=lin.per_token)
+        layer = api.NVFP4Linear(W, bias, per_token=lin.per_token, four_over_six=args.four_over_six)
     else:
         layer = api.MXFP8Linear(W, bias)
     del W
@@ -354,6 +354,8 @@ def run_ours(args, rank, world, local_rank):
 
     cfg = describe(lin, kind)
     cfg["parallelism"] = f"replicas x{world}"
+    if kind == "nvfp4":
+        cfg["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -371,7 +373,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = oracle_baseline(lin, kind, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = oracle_baseline(lin, kind, budget_s=args.cpu_budget, four_over_six=args.four_over_six)
     return out
 
 
@@ -484,10 +486,10 @@ def oracle_step(lin, kind, rows, wq):
     return oracle.bf16_round(y)
 
 
-def oracle_weights(lin, kind):
+def oracle_weights(lin, kind, four_over_six=False):
     import oracle
     if kind == "nvfp4":
-        gs_w = oracle.nvfp4_global_scale(oracle.amax_bf16(lin.W))
+        gs_w = oracle.nvfp4_global_scale(oracle.amax_bf16(lin.W), 1536.0 if four_over_six else 2688.0)
         cb, sb = oracle.nvfp4_quantize(lin.W, gs_w)
         return gs_w, cb, sb, oracle.nvfp4_dequantize(cb, sb, lin.K)
     qb, sb = oracle.mxfp8_quantize(lin.W)
@@ -502,9 +504,9 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_baseline(lin, kind, budget_s=10.0):
+def oracle_baseline(lin, kind, budget_s=10.0, four_over_six=False):
     """Times the oracle on a bounded row sample, scaled to TFLOP/s."""
-    wq = oracle_weights(lin, kind)
+    wq = oracle_weights(lin, kind, four_over_six)
     rng = np.random.default_rng(123)
     rows = np.sort(rng.choice(lin.M, size=min(lin.M, 128), replace=False))
     t0 = time.perf_counter()
@@ -559,7 +561,7 @@ def run_reference(args):
     if args.config == "loadtime":
         return run_reference_loadtime(args)
     lin, kind = make_workload(args.config)
-    wq = oracle_weights(lin, kind)
+    wq = oracle_weights(lin, kind, args.four_over_six)
     rng = np.random.default_rng(7)
     n = min(lin.M, args.ref_rows)
     for _ in range(args.warmup):
@@ -575,6 +577,8 @@ def run_reference(args):
               f"rounding; weight quantized beforehand (load time)")
     cfg = describe(lin, kind)
     cfg["parallelism"] = "host cores"
+    if kind == "nvfp4":
+        cfg["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -591,6 +595,8 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="wan13")
+    ap.add_argument("--four-over-six", action="store_true",
+                    help="NVFP4 weight global scale 256*6/amax (the 4over6 setting) instead of 448*6/amax")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=256, help="rows per oracle step for --impl reference")

@@ -30,7 +30,9 @@ SIGNATURES = {
     "bsp_nvfp4_sf_bytes": (_sz, [_i64, _i64]),
     "bsp_mxfp8_sf_bytes": (_sz, [_i64, _i64]),
     "bsp_amax_bf16": (_i32, [_vp, _i64, _vp, _vp]),
+    "bsp_amax_bf16_into": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_nvfp4_global_scale": (_i32, [_vp, _vp, _vp, _vp]),
+    "bsp_nvfp4_global_scale_max": (_i32, [_vp, ctypes.c_float, _vp, _vp, _vp]),
     "bsp_nvfp4_alpha": (_i32, [_vp, _vp, _vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),

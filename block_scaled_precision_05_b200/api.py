@@ -57,6 +57,13 @@ def mxfp8_sf_bytes(rows: int, K: int) -> int:
 
 
 # --------------------------------------------------------------------------- scales
+# e4m3_max * 6: the numerator of the NVFP4 global scale.  448 is the largest
+# e4m3 value; the 4over6 setting of nvfp4_online.py _quantize_weight_nvfp4 uses
+# 256 so that every group scale stays <= 256.
+FP8_FP4_MAX = 448.0 * 6.0
+FP8_FP4_MAX_4OVER6 = 256.0 * 6.0
+
+
 def amax(x: torch.Tensor) -> torch.Tensor:
     """fp32 [1] device tensor: max |x| over a bf16 tensor (NaN as 0, inf as bf16 max)."""
     _require_cuda(x)
@@ -67,14 +74,39 @@ def amax(x: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def nvfp4_global_scale(amax_t: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
-    """(gs, 1/gs) fp32 [1] device tensors with gs = 448*6/amax (1 for amax 0)."""
+def amax_into(x: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
+    """Folds max |x| into `out` (an fp32 [1] amax from `amax`) on the device."""
+    _require_cuda(x, out)
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("amax_into expects a contiguous bf16 tensor")
+    if out.dtype != torch.float32 or out.numel() != 1:
+        raise ValueError("amax_into expects an fp32 [1] accumulator")
+    nat.check(nat.lib().bsp_amax_bf16_into(_ptr(x), x.numel(), _ptr(out), _stream()), "bsp_amax_bf16_into")
+    return out
+
+
+def nvfp4_global_scale(amax_t: torch.Tensor, fp8_fp4_max: float = FP8_FP4_MAX) -> tuple[torch.Tensor, torch.Tensor]:
+    """(gs, 1/gs) fp32 [1] device tensors with gs = fp8_fp4_max/amax (1 for amax 0)."""
     _require_cuda(amax_t)
     gs = torch.empty(1, dtype=torch.float32, device=amax_t.device)
     inv = torch.empty_like(gs)
-    nat.check(nat.lib().bsp_nvfp4_global_scale(_ptr(amax_t), _ptr(gs), _ptr(inv), _stream()),
-              "bsp_nvfp4_global_scale")
+    nat.check(nat.lib().bsp_nvfp4_global_scale_max(_ptr(amax_t), float(fp8_fp4_max), _ptr(gs), _ptr(inv), _stream()),
+              "bsp_nvfp4_global_scale_max")
     return gs, inv
+
+
+def nvfp4_quantize_shared(weights, fp8_fp4_max: float = FP8_FP4_MAX):
+    """Quantizes several bf16 weights with one global scale from their joint
+    amax (the gated w1/w3 pair of nvfp4_online.py, quantized together so both
+    halves share one per-tensor scale).  Returns ([NVFP4Tensor], gs, 1/gs)."""
+    ws = [coerce_input(w).contiguous() for w in weights]
+    if not ws:
+        raise ValueError("nvfp4_quantize_shared needs at least one weight")
+    a = amax(ws[0])
+    for w in ws[1:]:
+        amax_into(w, a)
+    gs, inv = nvfp4_global_scale(a, fp8_fp4_max)
+    return [nvfp4_quantize(w, gs) for w in ws], gs, inv
 
 
 def nvfp4_alpha(gs_x: torch.Tensor, gs_w: torch.Tensor) -> torch.Tensor:
@@ -217,9 +249,14 @@ class NVFP4Linear:
     per_token=False: static activation scale gs_x = 1.0 (no reduction, no host
     sync, capturable in a CUDA graph).  per_token=True: per-row activation
     scales computed inside the quantize kernel and applied in the GEMM epilogue.
+    four_over_six=True: weight global scale 256*6/amax instead of 448*6/amax
+    (nvfp4_online.py, the 4over6 setting).  global_scale=(gs_w, 1/gs_w): use a
+    weight scale shared with other tensors (see shared_scale_group) instead of
+    this weight's own amax.
     """
 
-    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None, per_token: bool = False):
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None, per_token: bool = False,
+                 four_over_six: bool = False, global_scale: tuple[torch.Tensor, torch.Tensor] | None = None):
         if weight.dim() != 2:
             raise ValueError(f"expects a 2-D weight, got shape {tuple(weight.shape)}")
         if weight.shape[1] % 16 != 0:
@@ -227,7 +264,10 @@ class NVFP4Linear:
         w = coerce_input(weight).contiguous()
         self.out_features, self.in_features = w.shape
         self.per_token = per_token
-        self.gs_w, self.inv_gs_w = nvfp4_global_scale(amax(w))
+        if global_scale is None:
+            self.gs_w, self.inv_gs_w = nvfp4_global_scale(amax(w), FP8_FP4_MAX_4OVER6 if four_over_six else FP8_FP4_MAX)
+        else:
+            self.gs_w, self.inv_gs_w = global_scale
         self.weight = nvfp4_quantize(w, self.gs_w)
         self.gs_x = torch.ones(1, dtype=torch.float32, device=w.device)
         # per-token: the GEMM applies 1/gs_w here and 1/gs_x[m] as the row scale
@@ -245,6 +285,21 @@ class NVFP4Linear:
         y = nvfp4_gemm(xq, self.weight, self.alpha, xq.row_inv_gs if self.per_token else None, self.bias,
                        out_dtype=out_dtype)
         return y.view(*lead, self.out_features)
+
+
+    @classmethod
+    def shared_scale_group(cls, weights, biases=None, per_token: bool = False, four_over_six: bool = False):
+        """Linear layers whose weights share one global scale from their joint
+        amax (the gated w1/w3 pair of nvfp4_online.py)."""
+        ws = [coerce_input(w).contiguous() for w in weights]
+        if not ws:
+            raise ValueError("shared_scale_group needs at least one weight")
+        a = amax(ws[0])
+        for w in ws[1:]:
+            amax_into(w, a)
+        scale = nvfp4_global_scale(a, FP8_FP4_MAX_4OVER6 if four_over_six else FP8_FP4_MAX)
+        biases = [None] * len(ws) if biases is None else list(biases)
+        return [cls(w, b, per_token=per_token, global_scale=scale) for w, b in zip(ws, biases)]
 
 
 class MXFP8Linear:

@@ -505,9 +505,9 @@ __global__ void __launch_bounds__(kQuantThreads) amax_bf16_kernel(const uint16_t
   }
 }
 
-__global__ void global_scale_kernel(const float* __restrict__ amax, float* gs, float* inv_gs) {
+__global__ void global_scale_kernel(const float* __restrict__ amax, float fp8_fp4_max, float* gs, float* inv_gs) {
   const float a = *amax;
-  const float g = (a > 0.0f) ? __fdiv_rn(2688.0f, a) : 1.0f;
+  const float g = (a > 0.0f) ? __fdiv_rn(fp8_fp4_max, a) : 1.0f;
   if (gs) *gs = g;
   if (inv_gs) *inv_gs = __fdiv_rn(1.0f, g);
 }
@@ -553,6 +553,22 @@ int grid_for_rows(const DeviceInfo& dev, Kernel kernel, int64_t rows) {
   const int64_t needed = ceil_div(rows, warps_per_block);
   const int64_t cap = static_cast<int64_t>(dev.sm_count) * per_sm;
   return static_cast<int>(needed < cap ? (needed > 0 ? needed : 1) : cap);
+}
+
+// max|x| folded into *amax (zeroed first when `reset`).
+int amax_launch(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream, bool reset) {
+  if (n < 0 || !amax || (n > 0 && !x)) return BSP_ERR_INVALID_ARG;
+  if ((x && !aligned16(x)) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  if (reset && cudaMemsetAsync(amax, 0, sizeof(float), stream) != cudaSuccess) return launch_status();
+  if (n == 0) return BSP_OK;
+  int64_t blocks = ceil_div(ceil_div(n, 8), kQuantThreads);
+  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  amax_bf16_kernel<<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(x, n, reinterpret_cast<uint32_t*>(amax));
+  return launch_status();
 }
 
 }  // namespace
@@ -642,27 +658,26 @@ int mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, uint8_
 }
 
 int bsp_amax_bf16(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
-  if (n < 0 || !amax || (n > 0 && !x)) return BSP_ERR_INVALID_ARG;
-  if ((x && !aligned16(x)) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return BSP_ERR_ALIGNMENT;
+  return amax_launch(x, n, amax, stream, true);
+}
+
+int bsp_amax_bf16_into(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
+  return amax_launch(x, n, amax, stream, false);
+}
+
+int bsp_nvfp4_global_scale_max(const float* amax, float fp8_fp4_max, float* gs, float* inv_gs,
+                               bsp_stream_t stream) {
+  if (!amax || (!gs && !inv_gs)) return BSP_ERR_INVALID_ARG;
+  if (!(fp8_fp4_max > 0.0f) || !(fp8_fp4_max <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
   DeviceInfo dev;
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
-  if (cudaMemsetAsync(amax, 0, sizeof(float), stream) != cudaSuccess) return launch_status();
-  if (n == 0) return BSP_OK;
-  int64_t blocks = ceil_div(ceil_div(n, 8), kQuantThreads);
-  const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
-  if (blocks > cap) blocks = cap;
-  amax_bf16_kernel<<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(x, n, reinterpret_cast<uint32_t*>(amax));
+  global_scale_kernel<<<1, 1, 0, stream>>>(amax, fp8_fp4_max, gs, inv_gs);
   return launch_status();
 }
 
 int bsp_nvfp4_global_scale(const float* amax, float* gs, float* inv_gs, bsp_stream_t stream) {
-  if (!amax || (!gs && !inv_gs)) return BSP_ERR_INVALID_ARG;
-  DeviceInfo dev;
-  int st = current_device(&dev);
-  if (st != BSP_OK) return st;
-  global_scale_kernel<<<1, 1, 0, stream>>>(amax, gs, inv_gs);
-  return launch_status();
+  return bsp_nvfp4_global_scale_max(amax, 448.0f * 6.0f, gs, inv_gs, stream);
 }
 
 int bsp_nvfp4_alpha(const float* gs_x, const float* gs_w, float* alpha, bsp_stream_t stream) {

@@ -102,12 +102,33 @@ size_t bsp_mxfp8_sf_bytes(int64_t rows, int64_t K);
  * Errors: n < 0 -> INVALID_ARG; misaligned x -> ALIGNMENT. */
 int bsp_amax_bf16(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream);
 
+/* As bsp_amax_bf16, but folds max |x_i| into the caller's *amax (which must
+ * hold a previous amax, e.g. from bsp_amax_bf16) instead of overwriting it:
+ * the amax over several tensors that must share one global scale, such as the
+ * gated w1/w3 pair that nvfp4_online.py quantizes together
+ * (process_loaded_weight: torch.cat of the pair, one amax-derived scale).
+ *   x     : bf16 [n], 16-byte aligned
+ *   amax  : fp32 [1], read and updated on the device
+ * Errors as bsp_amax_bf16. */
+int bsp_amax_bf16_into(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream);
+
 /* NVFP4 encode scale from an amax, on the device (no host sync):
  *   gs = amax > 0 ? fl32(448*6 / amax) : 1.0     (convert_model_to_fp4; the
  *        all-zero guard is nvfp4_online.py _quantize_weight_nvfp4)
  *   inv_gs = fl32(1 / gs)                         (the decode scale)
  * amax, gs, inv_gs: fp32 [1].  gs or inv_gs may be NULL. */
 int bsp_nvfp4_global_scale(const float *amax, float *gs, float *inv_gs, bsp_stream_t stream);
+
+/* The same with the numerator as a parameter: gs = amax > 0 ?
+ * fl32(fp8_fp4_max / amax) : 1.0, inv_gs = fl32(1 / gs).  fp8_fp4_max is
+ * e4m3_max * 6: 448 * 6 = 2688 (bsp_nvfp4_global_scale) or, with the 4over6
+ * setting of nvfp4_online.py _quantize_weight_nvfp4 (e4m3_max = 256 so that
+ * every group scale stays <= 256), 256 * 6 = 1536.
+ *   fp8_fp4_max: host value, finite and > 0 (else INVALID_ARG, nothing
+ *                launched)
+ * Other arguments and errors as bsp_nvfp4_global_scale. */
+int bsp_nvfp4_global_scale_max(const float *amax, float fp8_fp4_max, float *gs, float *inv_gs,
+                               bsp_stream_t stream);
 
 /* alpha = fl32(1 / fl32(gs_x * gs_w)), the GEMM output scale of
  * NVFP4QATQuantizeMethod.apply.  All fp32 [1]. */

@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.bspo_amax_bf16.argtypes = [vp, i64]
         L.bspo_nvfp4_global_scale.restype = f32
         L.bspo_nvfp4_global_scale.argtypes = [f32]
+        L.bspo_nvfp4_global_scale_max.restype = f32
+        L.bspo_nvfp4_global_scale_max.argtypes = [f32, f32]
         L.bspo_row_global_scales.restype = None
         L.bspo_row_global_scales.argtypes = [vp, i64, i64, i64, vp, vp]
         L.bspo_nvfp4_quantize_group.restype = None
@@ -170,8 +172,11 @@ def amax_bf16(x: np.ndarray) -> float:
     return float(np.float32(lib().bspo_amax_bf16(_ptr(a), a.size)))
 
 
-def nvfp4_global_scale(amax: float) -> np.float32:
-    return np.float32(lib().bspo_nvfp4_global_scale(float(np.float32(amax))))
+def nvfp4_global_scale(amax: float, fp8_fp4_max: float | None = None) -> np.float32:
+    """gs = fp8_fp4_max / amax in fp32 (1 for amax 0); fp8_fp4_max defaults to 448*6."""
+    if fp8_fp4_max is None:
+        return np.float32(lib().bspo_nvfp4_global_scale(float(np.float32(amax))))
+    return np.float32(lib().bspo_nvfp4_global_scale_max(float(np.float32(amax)), float(np.float32(fp8_fp4_max))))
 
 
 def row_global_scales(x: np.ndarray):

@@ -215,13 +215,21 @@ float bspo_amax_bf16(const uint16_t *x, int64_t n)
     return (float)amax; /* exact: a bf16 value */
 }
 
-/* Encode global scale 448*6/amax in fp32; an all-zero tensor gets 1.0
- * (the guarded form of [SGL], where weight_scale_2 is 1 when amax is 0). */
-float bspo_nvfp4_global_scale(float amax)
+/* Encode global scale fp8_fp4_max/amax in fp32, fp8_fp4_max = e4m3_max * 6;
+ * an all-zero tensor gets 1.0 (the guarded form of [SGL], where
+ * weight_scale_2 is 1 when amax is 0).  [SGL] _quantize_weight_nvfp4 takes
+ * e4m3_max = 448 (the largest e4m3), or 256 with its 4over6 setting. */
+float bspo_nvfp4_global_scale_max(float amax, float fp8_fp4_max)
 {
     if (amax > 0.0f)
-        return 2688.0f / amax;
+        return fp8_fp4_max / amax;
     return 1.0f;
+}
+
+/* 448*6/amax: [FV-QAT] convert_model_to_fp4. */
+float bspo_nvfp4_global_scale(float amax)
+{
+    return bspo_nvfp4_global_scale_max(amax, 448.0f * 6.0f);
 }
 
 /* Per-row (per-token) scales: gs[m] from the row amax; inv[m] = fl32(1/gs[m]),

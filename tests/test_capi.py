@@ -64,6 +64,10 @@ def test_host_validation_rejects_bad_arguments():
     assert L.nvfp4_gemm(p, p, p, p, 0, 8, 64, None, None, None, p, 0, 8, None) == nat.BSP_OK
     assert L.mxfp8_gemm(p, p, p, p, 4, 8, 48, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_amax_bf16(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.bsp_amax_bf16_into(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
+    for bad in (0.0, -2688.0, float("inf"), float("nan")):
+        assert L.bsp_nvfp4_global_scale_max(p, bad, p, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.bsp_nvfp4_global_scale_max(p, 1536.0, None, None, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_debug_wait_timeout(10, None) == nat.BSP_ERR_INVALID_ARG
 
 
