@@ -31,10 +31,13 @@ SIGNATURES = {
     "bsp_mxfp8_sf_bytes": (_sz, [_i64, _i64]),
     "bsp_amax_bf16": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_amax_bf16_into": (_i32, [_vp, _i64, _vp, _vp]),
+    "bsp_amax_f16": (_i32, [_vp, _i64, _vp, _vp]),
+    "bsp_amax_f16_into": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_nvfp4_global_scale": (_i32, [_vp, _vp, _vp, _vp]),
     "bsp_nvfp4_global_scale_max": (_i32, [_vp, ctypes.c_float, _vp, _vp, _vp]),
     "bsp_nvfp4_alpha": (_i32, [_vp, _vp, _vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nvfp4_quantize_f16": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "mxfp8_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "mxfp8_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _i64, _vp]),

@@ -41,11 +41,22 @@ def _require_cuda(*ts: torch.Tensor | None) -> None:
 
 
 def coerce_input(x: torch.Tensor) -> torch.Tensor:
-    """Activation dtype rule of the pages: bf16 passes, other floats are cast to
-    bf16, anything else is an error."""
+    """Input dtype rule of the NVFP4 path (nvfp4_config.py,
+    _coerce_fp4_input_dtype): bf16 and fp16 pass as they are, other floats are
+    cast to bf16, anything else is an error."""
+    if not x.is_floating_point():
+        raise TypeError(f"block-scaled linear expects floating-point inputs, got {x.dtype}")
+    return x if x.dtype in (torch.bfloat16, torch.float16) else x.to(torch.bfloat16)
+
+
+def coerce_bf16(x: torch.Tensor) -> torch.Tensor:
+    """bf16 for the paths whose kernels read bf16 only (MXFP8, the bias)."""
     if not x.is_floating_point():
         raise TypeError(f"block-scaled linear expects floating-point inputs, got {x.dtype}")
     return x if x.dtype == torch.bfloat16 else x.to(torch.bfloat16)
+
+
+_HALF_TYPES = (torch.bfloat16, torch.float16)
 
 
 def nvfp4_sf_bytes(rows: int, K: int) -> int:
@@ -65,23 +76,26 @@ FP8_FP4_MAX_4OVER6 = 256.0 * 6.0
 
 
 def amax(x: torch.Tensor) -> torch.Tensor:
-    """fp32 [1] device tensor: max |x| over a bf16 tensor (NaN as 0, inf as bf16 max)."""
+    """fp32 [1] device tensor: max |x| over a bf16 or fp16 tensor (NaN as 0, inf
+    as the format's largest finite value)."""
     _require_cuda(x)
-    if x.dtype != torch.bfloat16 or not x.is_contiguous():
-        raise ValueError("amax expects a contiguous bf16 tensor")
+    if x.dtype not in _HALF_TYPES or not x.is_contiguous():
+        raise ValueError("amax expects a contiguous bf16 or fp16 tensor")
     out = torch.empty(1, dtype=torch.float32, device=x.device)
-    nat.check(nat.lib().bsp_amax_bf16(_ptr(x), x.numel(), _ptr(out), _stream()), "bsp_amax_bf16")
+    fn = "bsp_amax_bf16" if x.dtype == torch.bfloat16 else "bsp_amax_f16"
+    nat.check(getattr(nat.lib(), fn)(_ptr(x), x.numel(), _ptr(out), _stream()), fn)
     return out
 
 
 def amax_into(x: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
     """Folds max |x| into `out` (an fp32 [1] amax from `amax`) on the device."""
     _require_cuda(x, out)
-    if x.dtype != torch.bfloat16 or not x.is_contiguous():
-        raise ValueError("amax_into expects a contiguous bf16 tensor")
+    if x.dtype not in _HALF_TYPES or not x.is_contiguous():
+        raise ValueError("amax_into expects a contiguous bf16 or fp16 tensor")
     if out.dtype != torch.float32 or out.numel() != 1:
         raise ValueError("amax_into expects an fp32 [1] accumulator")
-    nat.check(nat.lib().bsp_amax_bf16_into(_ptr(x), x.numel(), _ptr(out), _stream()), "bsp_amax_bf16_into")
+    fn = "bsp_amax_bf16_into" if x.dtype == torch.bfloat16 else "bsp_amax_f16_into"
+    nat.check(getattr(nat.lib(), fn)(_ptr(x), x.numel(), _ptr(out), _stream()), fn)
     return out
 
 
@@ -153,10 +167,10 @@ def _as_2d(x: torch.Tensor) -> torch.Tensor:
 
 def nvfp4_quantize(x: torch.Tensor, global_sf: torch.Tensor | None = None, per_row: bool = False,
                    out: NVFP4Tensor | None = None) -> NVFP4Tensor:
-    """Quantize bf16 [..., K] to NVFP4 along K (leading dims flattened)."""
+    """Quantize bf16 or fp16 [..., K] to NVFP4 along K (leading dims flattened)."""
     _require_cuda(x, global_sf)
-    if x.dtype != torch.bfloat16:
-        raise TypeError("nvfp4_quantize expects bf16 input (use coerce_input first)")
+    if x.dtype not in _HALF_TYPES:
+        raise TypeError("nvfp4_quantize expects bf16 or fp16 input (use coerce_input first)")
     x2 = _as_2d(x)
     M, K = x2.shape
     dev = x2.device
@@ -168,12 +182,13 @@ def nvfp4_quantize(x: torch.Tensor, global_sf: torch.Tensor | None = None, per_r
             out.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
     if not per_row and global_sf is None:
         raise ValueError("per-tensor quantization needs global_sf (fp32 device tensor)")
-    st = nat.lib().nvfp4_quantize(
+    fn = nat.lib().nvfp4_quantize if x2.dtype == torch.bfloat16 else nat.lib().nvfp4_quantize_f16
+    st = fn(
         _ptr(x2), M, K, x2.stride(0), None if per_row else _ptr(global_sf),
         nat.BSP_SF_PER_ROW if per_row else nat.BSP_SF_PER_TENSOR,
         _ptr(out.row_gs) if per_row else None, _ptr(out.row_inv_gs) if per_row else None,
         _ptr(out.codes), _ptr(out.sf), _stream())
-    nat.check(st, "nvfp4_quantize")
+    nat.check(st, "nvfp4_quantize" if x2.dtype == torch.bfloat16 else "nvfp4_quantize_f16")
     return out
 
 
@@ -204,6 +219,14 @@ def _out(M: int, N: int, dtype: torch.dtype, device, out: torch.Tensor | None) -
     return out, (nat.BSP_OUT_F32 if dtype == torch.float32 else nat.BSP_OUT_BF16)
 
 
+def _check_epilogue_args(alpha, row_scale, bias, N: int) -> None:
+    for name, t in (("alpha", alpha), ("row_scale", row_scale)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise TypeError(f"{name} must be a contiguous fp32 device tensor")
+    if bias is not None and (bias.dtype != torch.bfloat16 or not bias.is_contiguous() or bias.numel() != N):
+        raise TypeError(f"bias must be a contiguous bf16 tensor of {N} elements")
+
+
 def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, alpha: torch.Tensor | None = None,
                row_scale: torch.Tensor | None = None, bias: torch.Tensor | None = None,
                out_dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
@@ -212,6 +235,7 @@ def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, alpha: torch.Tensor | None = None
         raise ValueError("A and B disagree on K")
     _require_cuda(a.codes, b.codes, alpha, row_scale, bias)
     M, N = a.rows, b.rows
+    _check_epilogue_args(alpha, row_scale, bias, N)
     out, d_dtype = _out(M, N, out_dtype, a.codes.device, out)
     st = nat.lib().nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, a.K,
                               _ptr(alpha), _ptr(row_scale), _ptr(bias), _ptr(out), d_dtype, out.stride(0),
@@ -228,6 +252,7 @@ def mxfp8_gemm(a: MXFP8Tensor, b: MXFP8Tensor, alpha: torch.Tensor | None = None
         raise ValueError("A and B disagree on K")
     _require_cuda(a.q, b.q, alpha, bias)
     M, N = a.rows, b.rows
+    _check_epilogue_args(alpha, None, bias, N)
     out, d_dtype = _out(M, N, out_dtype, a.q.device, out)
     st = nat.lib().mxfp8_gemm(_ptr(a.q), _ptr(a.sf), _ptr(b.q), _ptr(b.sf), M, N, a.K, _ptr(alpha), _ptr(bias),
                               _ptr(out), d_dtype, out.stride(0), _stream())
@@ -272,7 +297,7 @@ class NVFP4Linear:
         self.gs_x = torch.ones(1, dtype=torch.float32, device=w.device)
         # per-token: the GEMM applies 1/gs_w here and 1/gs_x[m] as the row scale
         self.alpha = self.inv_gs_w if per_token else nvfp4_alpha(self.gs_x, self.gs_w)
-        self.bias = None if bias is None else coerce_input(bias).contiguous()
+        self.bias = None if bias is None else coerce_bf16(bias).contiguous()
 
     def quantize_input(self, x: torch.Tensor) -> NVFP4Tensor:
         x = coerce_input(x)
@@ -308,12 +333,12 @@ class MXFP8Linear:
     def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None):
         if weight.dim() != 2 or weight.shape[1] % 32 != 0:
             raise ValueError(f"expects a 2-D weight with K % 32 == 0, got {tuple(weight.shape)}")
-        w = coerce_input(weight).contiguous()
+        w = coerce_bf16(weight).contiguous()
         self.out_features, self.in_features = w.shape
         self.weight = mxfp8_quantize(w)
-        self.bias = None if bias is None else coerce_input(bias).contiguous()
+        self.bias = None if bias is None else coerce_bf16(bias).contiguous()
 
     def __call__(self, x: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
         lead = x.shape[:-1]
-        xq = mxfp8_quantize(coerce_input(x))
+        xq = mxfp8_quantize(coerce_bf16(x))
         return mxfp8_gemm(xq, self.weight, None, self.bias, out_dtype=out_dtype).view(*lead, self.out_features)

@@ -20,6 +20,8 @@
 // domain (|bf16| bit patterns order like their values), hardware cvt with
 // round-to-nearest-even and saturation, 8- or 32-byte code stores, and the four
 // scale bytes of a 128x4 tile row gathered by shuffles into one 4-byte store.
+#include <cuda_fp16.h>
+
 #include "bsp_device.cuh"
 #include "bsp_internal.h"
 
@@ -32,48 +34,94 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
-// |x| bit pattern of a bf16 for the amax reductions: NaN counts as 0 and
-// +-inf as the largest finite bf16 (x.abs().nan_to_num()).
+// Input element formats (16-bit floats, two per 32-bit word, the element at
+// the lower address in the low half).  In both, the bit pattern of |x| orders
+// like its value.
+struct InBf16 {
+  using T2 = __nv_bfloat162;
+  static constexpr uint32_t kInf = 0x7F80u, kMaxFinite = 0x7F7Fu;
+  static __device__ __forceinline__ float value(uint32_t bits) { return __uint_as_float(bits << 16); }
+  static __device__ __forceinline__ float2 values2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  }
+  static __device__ __forceinline__ T2 abs2(uint32_t w) {
+    T2 r;
+    const uint32_t u = w & 0x7FFF7FFFu;
+    memcpy(&r, &u, 4);
+    return r;
+  }
+  static __device__ __forceinline__ uint32_t larger_half(T2 m) {
+    const __nv_bfloat16 h = __hmax(__low2bfloat16(m), __high2bfloat16(m));
+    uint16_t u;
+    memcpy(&u, &h, 2);
+    return u;
+  }
+};
+
+struct InF16 {
+  using T2 = __half2;
+  static constexpr uint32_t kInf = 0x7C00u, kMaxFinite = 0x7BFFu;
+  static __device__ __forceinline__ float value(uint32_t bits) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+  }
+  static __device__ __forceinline__ float2 values2(uint32_t w) {
+    __half2 h;
+    memcpy(&h, &w, 4);
+    return __half22float2(h);
+  }
+  static __device__ __forceinline__ T2 abs2(uint32_t w) {
+    T2 r;
+    const uint32_t u = w & 0x7FFF7FFFu;
+    memcpy(&r, &u, 4);
+    return r;
+  }
+  static __device__ __forceinline__ uint32_t larger_half(T2 m) {
+    const __half h = __hmax(__low2half(m), __high2half(m));
+    return __half_as_ushort(h);
+  }
+};
+
+// |x| bit pattern for the tensor / row amax: NaN counts as 0 and +-inf as the
+// largest finite value (x.abs().nan_to_num()).
+template <class In>
 __device__ __forceinline__ uint32_t sane_mag(uint32_t b16) {
-  uint32_t m = b16 & 0x7FFFu;
-  if (m > 0x7F80u) return 0u;
-  if (m == 0x7F80u) return 0x7F7Fu;
+  const uint32_t m = b16 & 0x7FFFu;
+  if (m > In::kInf) return 0u;
+  if (m == In::kInf) return In::kMaxFinite;
   return m;
 }
 
-__device__ __forceinline__ __nv_bfloat162 u32_as_bf162(uint32_t u) {
-  __nv_bfloat162 r;
-  memcpy(&r, &u, 4);
-  return r;
+// Packed maxima of |x| over the 8 elements of a 16-byte chunk, with the packed
+// max instruction, which ignores a NaN operand.
+template <class In>
+__device__ __forceinline__ typename In::T2 absmax8_x2(const uint4& v) {
+  return __hmax2(__hmax2(In::abs2(v.x), In::abs2(v.y)), __hmax2(In::abs2(v.z), In::abs2(v.w)));
 }
 
-// Packed maxima of |x| over the 8 bf16 of a 16-byte chunk (two lanes of 4),
-// with the packed bf16 max instruction, which ignores a NaN operand.
-__device__ __forceinline__ __nv_bfloat162 absmax8_x2(const uint4& v) {
-  const __nv_bfloat162 a = u32_as_bf162(v.x & 0x7FFF7FFFu), b = u32_as_bf162(v.y & 0x7FFF7FFFu);
-  const __nv_bfloat162 c = u32_as_bf162(v.z & 0x7FFF7FFFu), d = u32_as_bf162(v.w & 0x7FFF7FFFu);
-  return __hmax2(__hmax2(a, b), __hmax2(c, d));
-}
-
-// Bit pattern of the larger of the two packed maxima; NaN elements are
-// ignored (a group of NaNs only gives 0).  Values are non-negative, so bit
-// patterns order like the values.
-__device__ __forceinline__ uint32_t max_of_halves(__nv_bfloat162 m) {
-  const __nv_bfloat16 h = __hmax(__low2bfloat16(m), __high2bfloat16(m));
-  uint16_t u;
-  memcpy(&u, &h, 2);
-  return u > 0x7F80u ? 0u : static_cast<uint32_t>(u);
+// Bit pattern of the larger of two packed maxima; NaN elements are ignored (a
+// group of NaNs only gives 0).
+template <class In>
+__device__ __forceinline__ uint32_t max_of_halves(typename In::T2 m) {
+  const uint32_t u = In::larger_half(m);
+  return u > In::kInf ? 0u : u;
 }
 
 // amax bit pattern of one 16-element group (two 16-byte chunks).
+template <class In>
 __device__ __forceinline__ uint32_t group_mag16(const uint4& a, const uint4& b) {
-  return max_of_halves(__hmax2(absmax8_x2(a), absmax8_x2(b)));
+  return max_of_halves<In>(__hmax2(absmax8_x2<In>(a), absmax8_x2<In>(b)));
 }
 
-__device__ __forceinline__ uint32_t max_mag8(const uint4& v) { return max_of_halves(absmax8_x2(v)); }
+template <class In>
+__device__ __forceinline__ uint32_t max_mag8(const uint4& v) {
+  return max_of_halves<In>(absmax8_x2<In>(v));
+}
 
-// As max_mag8, with +-inf counted as the largest finite bf16 (sane_mag).
-__device__ __forceinline__ uint32_t max_sane_mag8(const uint4& v) { return min(max_mag8(v), 0x7F7Fu); }
+// As max_mag8, with +-inf counted as the largest finite value (sane_mag).
+template <class In>
+__device__ __forceinline__ uint32_t max_sane_mag8(const uint4& v) {
+  return min(max_mag8<In>(v), In::kMaxFinite);
+}
 
 __device__ __forceinline__ uint32_t warp_max(uint32_t m) {
 #pragma unroll
@@ -81,27 +129,28 @@ __device__ __forceinline__ uint32_t warp_max(uint32_t m) {
   return m;
 }
 
-// gs = amax > 0 ? fl32(2688 / amax) : 1, from a sanitized |bf16| bit pattern.
+// gs = amax > 0 ? fl32(2688 / amax) : 1, from a sanitized |x| bit pattern.
+template <class In>
 __device__ __forceinline__ float global_scale_from_mag(uint32_t mag) {
-  return mag == 0u ? 1.0f : __fdiv_rn(2688.0f, bf16_bits_to_f32(mag));
+  return mag == 0u ? 1.0f : __fdiv_rn(2688.0f, In::value(mag));
 }
 
 // NVFP4 scale byte and reciprocal of one group with amax bit pattern `mag`.
+template <class In>
 __device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sfb, float& inv) {
-  const float amax = bf16_bits_to_f32(mag);
+  const float amax = In::value(mag);
   const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
   sfb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
   inv = (sfb == 0u) ? 0.0f : __fdiv_rn(gs, e4m3_pos_to_f32(sfb));
 }
 
-// Eight bf16 (one 16-byte chunk) times inv -> eight e2m1 codes in one word.
-// The products are fp32 multiplies, two per packed instruction.
+// Eight elements (one 16-byte chunk) times inv -> eight e2m1 codes in one
+// word.  The products are fp32 multiplies, two per packed instruction.
+template <class In>
 __device__ __forceinline__ uint32_t nvfp4_codes8(const uint4& v, float inv) {
   const float2 i2 = make_float2(inv, inv);
-  const float2 p0 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.x & 0xFFFFu), __uint_as_float(v.x & 0xFFFF0000u)), i2);
-  const float2 p1 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.y & 0xFFFFu), __uint_as_float(v.y & 0xFFFF0000u)), i2);
-  const float2 p2 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.z & 0xFFFFu), __uint_as_float(v.z & 0xFFFF0000u)), i2);
-  const float2 p3 = __fmul2_rn(make_float2(bf16_bits_to_f32(v.w & 0xFFFFu), __uint_as_float(v.w & 0xFFFF0000u)), i2);
+  const float2 p0 = __fmul2_rn(In::values2(v.x), i2), p1 = __fmul2_rn(In::values2(v.y), i2);
+  const float2 p2 = __fmul2_rn(In::values2(v.z), i2), p3 = __fmul2_rn(In::values2(v.w), i2);
   return cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y);
 }
 
@@ -111,6 +160,7 @@ __device__ __forceinline__ int64_t sf_row_base(int64_t r, int64_t tiles_per_band
 }
 
 // Per-row encode scale of row r (warp-cooperative); lane 0 stores gs and 1/gs.
+template <class In>
 __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row, int64_t K, int64_t r,
                                                 float* row_gs, float* row_inv) {
   const uint32_t lane = lane_id();
@@ -118,11 +168,11 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
   int64_t c = lane * 8;
   for (; c + 768 < K; c += 1024) {  // four independent 16-byte loads in flight
     const uint4 a = ldg16(row + c), b = ldg16(row + c + 256), d = ldg16(row + c + 512), e = ldg16(row + c + 768);
-    m = max(max(m, max(max_sane_mag8(a), max_sane_mag8(b))), max(max_sane_mag8(d), max_sane_mag8(e)));
+    m = max(max(m, max(max_sane_mag8<In>(a), max_sane_mag8<In>(b))), max(max_sane_mag8<In>(d), max_sane_mag8<In>(e)));
   }
-  for (; c < K; c += 256) m = max(m, max_sane_mag8(ldg16(row + c)));
+  for (; c < K; c += 256) m = max(m, max_sane_mag8<In>(ldg16(row + c)));
   m = warp_max(m);
-  const float gs = global_scale_from_mag(m);
+  const float gs = global_scale_from_mag<In>(m);
   if (lane == 0) {
     if (row_gs) row_gs[r] = gs;
     if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
@@ -139,7 +189,7 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
 // lane, then the quantization of each.  `lp`, `cp`, `sp` point at this lane's
 // group, its 8 code bytes, and (for lanes with g % 4 == 0) its 4 scale bytes in
 // the first step.
-template <int U>
+template <class In, int U>
 __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uint8_t* sp, bool live, float gs,
                                             bool store_sf) {
   uint4 v[U][2];
@@ -152,10 +202,10 @@ __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uin
   for (int u = 0; u < U; ++u) {
     uint32_t sfb;
     float inv;
-    nvfp4_scale(group_mag16(v[u][0], v[u][1]), gs, sfb, inv);
+    nvfp4_scale<In>(group_mag16<In>(v[u][0], v[u][1]), gs, sfb, inv);
     uint2 w;
-    w.x = nvfp4_codes8(v[u][0], inv);
-    w.y = nvfp4_codes8(v[u][1], inv);
+    w.x = nvfp4_codes8<In>(v[u][0], inv);
+    w.y = nvfp4_codes8<In>(v[u][1], inv);
     const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
     const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
     const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
@@ -167,7 +217,7 @@ __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uin
 // Per-tensor scale, short rows (K = 512 * S, S <= 3): a warp quantizes two rows
 // per iteration with all 4S 16-byte loads of both rows issued up front, so the
 // memory pipeline stays full although each row is only S warp steps long.
-template <int S>
+template <class In, int S>
 __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const float* __restrict__ gs_ptr,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -202,10 +252,10 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
       for (int st = 0; st < S; ++st) {
         uint32_t sfb;
         float inv;
-        nvfp4_scale(group_mag16(v[h][st][0], v[h][st][1]), gs, sfb, inv);
+        nvfp4_scale<In>(group_mag16<In>(v[h][st][0], v[h][st][1]), gs, sfb, inv);
         uint2 w;
-        w.x = nvfp4_codes8(v[h][st][0], inv);
-        w.y = nvfp4_codes8(v[h][st][1], inv);
+        w.x = nvfp4_codes8<In>(v[h][st][0], inv);
+        w.y = nvfp4_codes8<In>(v[h][st][1], inv);
         const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
         const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
         const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
@@ -223,6 +273,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
 // registers, so each row costs one memory round trip.
 constexpr int kRowG = 4;
 
+template <class In>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, float* __restrict__ row_gs,
     float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -244,7 +295,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
       const bool in = live && g < groups;
       v[i][0] = in ? ldg16(row + g * 16) : make_uint4(0u, 0u, 0u, 0u);
       v[i][1] = in ? ldg16(row + g * 16 + 8) : make_uint4(0u, 0u, 0u, 0u);
-      mag = max(mag, max(max_sane_mag8(v[i][0]), max_sane_mag8(v[i][1])));
+      mag = max(mag, max(max_sane_mag8<In>(v[i][0]), max_sane_mag8<In>(v[i][1])));
     }
     mag = warp_max(mag);
     if (lane == 0) red[threadIdx.x >> 5] = mag;
@@ -253,7 +304,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
       uint32_t m = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0u;
       m = warp_max(m);
       if (threadIdx.x == 0) {
-        const float gs = global_scale_from_mag(m);
+        const float gs = global_scale_from_mag<In>(m);
         gs_sh = gs;
         if (live) {
           if (row_gs) row_gs[r] = gs;
@@ -272,10 +323,10 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
       if (i * kQuantThreads + (t & ~31) >= groups) break;  // warp-uniform
       uint32_t sfb;
       float inv;
-      nvfp4_scale(group_mag16(v[i][0], v[i][1]), gs, sfb, inv);
+      nvfp4_scale<In>(group_mag16<In>(v[i][0], v[i][1]), gs, sfb, inv);
       uint2 w;
-      w.x = nvfp4_codes8(v[i][0], inv);
-      w.y = nvfp4_codes8(v[i][1], inv);
+      w.x = nvfp4_codes8<In>(v[i][0], inv);
+      w.y = nvfp4_codes8<In>(v[i][1], inv);
       const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
       const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
       const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
@@ -289,7 +340,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
   }
 }
 
-template <bool kPerRow>
+template <class In, bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -307,18 +358,18 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const bool live = r < M;
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
-    if (kPerRow && live) gs = row_scale_pass(row, K, r, row_gs, row_inv);
+    if (kPerRow && live) gs = row_scale_pass<In>(row, K, r, row_gs, row_inv);
     // group g = 32 * step + lane: elements 16 g, code bytes 8 g, scale tile g / 4
     const uint16_t* lp = row + lane * 16;
     uint8_t* cp = codes + r * (K >> 1) + lane * 8;
     uint8_t* sp = sf + sf_row_base(r, groups >> 2) + (lane >> 2) * 512;
     int64_t st = 0;
     for (; st + kUnroll <= steps; st += kUnroll)
-      nvfp4_steps<kUnroll>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
-    for (; st < steps; ++st) nvfp4_steps<1>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
+      nvfp4_steps<In, kUnroll>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
+    for (; st < steps; ++st) nvfp4_steps<In, 1>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
     if (rem) {
       const bool in = lane < rem;  // groups beyond the row end are predicated off
-      nvfp4_steps<1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * 4096 : sp, live && in, gs,
+      nvfp4_steps<In, 1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * 4096 : sp, live && in, gs,
                      in && quad_lead);
     }
   }
@@ -327,7 +378,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
 // ---------------------------------------------------------------------------
 // NVFP4, any K % 16 == 0: one warp per row, one lane per group of 16.
 // ---------------------------------------------------------------------------
-template <bool kPerRow>
+template <class In, bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -342,17 +393,17 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
     const bool live = r < M;
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
-    if (kPerRow && live) gs = row_scale_pass(row, K, r, row_gs, row_inv);
+    if (kPerRow && live) gs = row_scale_pass<In>(row, K, r, row_gs, row_inv);
     const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
     for (int64_t c = lane; c < cols4; c += 32) {
       uint32_t sfb = 0;
       if (live && c < groups) {
         const uint4 a = ldg16(row + c * 16), b = ldg16(row + c * 16 + 8);
         float inv;
-        nvfp4_scale(group_mag16(a, b), gs, sfb, inv);
+        nvfp4_scale<In>(group_mag16<In>(a, b), gs, sfb, inv);
         uint2 w;
-        w.x = nvfp4_codes8(a, inv);
-        w.y = nvfp4_codes8(b, inv);
+        w.x = nvfp4_codes8<In>(a, inv);
+        w.y = nvfp4_codes8<In>(b, inv);
         *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
       }
       sf[sfb_row + (c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfb);
@@ -400,8 +451,8 @@ __device__ __forceinline__ void mxfp8_steps(const uint16_t* lp, uint8_t* qp, uin
     for (int i = 0; i < 4; ++i) v[u][i] = live ? ldg16(lp + u * 1024 + i * 8) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    const uint32_t mag = max_of_halves(__hmax2(__hmax2(absmax8_x2(v[u][0]), absmax8_x2(v[u][1])),
-                                               __hmax2(absmax8_x2(v[u][2]), absmax8_x2(v[u][3]))));
+    const uint32_t mag = max_of_halves<InBf16>(__hmax2(__hmax2(absmax8_x2<InBf16>(v[u][0]), absmax8_x2<InBf16>(v[u][1])),
+                                                       __hmax2(absmax8_x2<InBf16>(v[u][2]), absmax8_x2<InBf16>(v[u][3]))));
     uint32_t sfb;
     float mul;
     mx_scale(mag, sfb, mul);
@@ -470,7 +521,7 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_generic_kernel(cons
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           v[i] = ldg16(row + c * 32 + i * 8);
-          mag = max(mag, max_mag8(v[i]));
+          mag = max(mag, max_mag8<InBf16>(v[i]));
         }
         float mul;
         mx_scale(mag, sfb, mul);
@@ -485,14 +536,15 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_generic_kernel(cons
 // ---------------------------------------------------------------------------
 // Global scales.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kQuantThreads) amax_bf16_kernel(const uint16_t* __restrict__ x, int64_t n,
-                                                                   uint32_t* __restrict__ amax_bits) {
+template <class In>
+__global__ void __launch_bounds__(kQuantThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t n,
+                                                              uint32_t* __restrict__ amax_bits) {
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t nvec = n >> 3;
   uint32_t m = 0;
-  for (int64_t i = tid; i < nvec; i += nthreads) m = max(m, max_sane_mag8(ldg16(x + i * 8)));
-  for (int64_t i = (nvec << 3) + tid; i < n; i += nthreads) m = max(m, sane_mag(x[i]));
+  for (int64_t i = tid; i < nvec; i += nthreads) m = max(m, max_sane_mag8<In>(ldg16(x + i * 8)));
+  for (int64_t i = (nvec << 3) + tid; i < n; i += nthreads) m = max(m, sane_mag<In>(x[i]));
   m = warp_max(m);
   __shared__ uint32_t red[kQuantThreads / 32];
   if (lane_id() == 0) red[threadIdx.x >> 5] = m;
@@ -500,8 +552,8 @@ __global__ void __launch_bounds__(kQuantThreads) amax_bf16_kernel(const uint16_t
   if (threadIdx.x < 32) {
     m = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0u;
     m = warp_max(m);
-    // |bf16| << 16 is a non-negative fp32 bit pattern: integer order == value order.
-    if (threadIdx.x == 0 && m != 0u) atomicMax(amax_bits, m << 16);
+    // a non-negative fp32 bit pattern: integer order == value order
+    if (threadIdx.x == 0 && m != 0u) atomicMax(amax_bits, __float_as_uint(In::value(m)));
   }
 }
 
@@ -556,6 +608,7 @@ int grid_for_rows(const DeviceInfo& dev, Kernel kernel, int64_t rows) {
 }
 
 // max|x| folded into *amax (zeroed first when `reset`).
+template <class In>
 int amax_launch(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream, bool reset) {
   if (n < 0 || !amax || (n > 0 && !x)) return BSP_ERR_INVALID_ARG;
   if ((x && !aligned16(x)) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return BSP_ERR_ALIGNMENT;
@@ -567,19 +620,13 @@ int amax_launch(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream, 
   int64_t blocks = ceil_div(ceil_div(n, 8), kQuantThreads);
   const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
   if (blocks > cap) blocks = cap;
-  amax_bf16_kernel<<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(x, n, reinterpret_cast<uint32_t*>(amax));
+  amax_kernel<In><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(x, n, reinterpret_cast<uint32_t*>(amax));
   return launch_status();
 }
 
-}  // namespace
-}  // namespace bsp
-
-using namespace bsp;
-
-extern "C" {
-
-int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
-                   float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
+template <class In>
+int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
+                       float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
   if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K) return BSP_ERR_INVALID_ARG;
   if (sf_mode != BSP_SF_PER_TENSOR && sf_mode != BSP_SF_PER_ROW) return BSP_ERR_INVALID_ARG;
   if (M == 0) return BSP_OK;
@@ -594,8 +641,8 @@ int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const 
     int rowblock_cap = 0;  // rows the block-per-row kernel keeps resident at once
     if (per_row && K <= 16 * kQuantThreads * kRowG) {
       int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_quant_rowblock_kernel, kQuantThreads, 0) !=
-              cudaSuccess ||
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_quant_rowblock_kernel<In>, kQuantThreads,
+                                                        0) != cudaSuccess ||
           per_sm < 1) {
         cudaGetLastError();
         per_sm = 1;
@@ -604,38 +651,55 @@ int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const 
     }
     if (per_row && Mp <= rowblock_cap) {
       // few rows: one block per row, all rows in one wave, one memory round trip
-      nvfp4_quant_rowblock_kernel<<<static_cast<int>(Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, row_gs,
+      nvfp4_quant_rowblock_kernel<In><<<static_cast<int>(Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, row_gs,
                                                                                       row_inv_gs, codes, sf);
     } else if (per_row) {
-      auto k = nvfp4_quant_k64_kernel<true>;
+      auto k = nvfp4_quant_k64_kernel<In, true>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
                                                                  codes, sf);
     } else if (K == 1024 || K == 1536) {
       const int64_t pairs = ceil_div(Mp, 2);
       if (K == 1024) {
-        auto k = nvfp4_quant_short_kernel<2>;
+        auto k = nvfp4_quant_short_kernel<In, 2>;
         k<<<grid_for_rows(dev, k, pairs), kQuantThreads, 0, stream>>>(x, M, Mp, ld_x, global_sf, codes, sf);
       } else {
-        auto k = nvfp4_quant_short_kernel<3>;
+        auto k = nvfp4_quant_short_kernel<In, 3>;
         k<<<grid_for_rows(dev, k, pairs), kQuantThreads, 0, stream>>>(x, M, Mp, ld_x, global_sf, codes, sf);
       }
     } else {
-      auto k = nvfp4_quant_k64_kernel<false>;
+      auto k = nvfp4_quant_k64_kernel<In, false>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
                                                                  codes, sf);
     }
   } else {
     if (per_row) {
-      auto k = nvfp4_quant_generic_kernel<true>;
+      auto k = nvfp4_quant_generic_kernel<In, true>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
                                                                  codes, sf);
     } else {
-      auto k = nvfp4_quant_generic_kernel<false>;
+      auto k = nvfp4_quant_generic_kernel<In, false>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
                                                                  codes, sf);
     }
   }
   return launch_status();
+}
+
+}  // namespace
+}  // namespace bsp
+
+using namespace bsp;
+
+extern "C" {
+
+int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
+                   float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
+  return run_nvfp4_quantize<InBf16>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
+}
+
+int nvfp4_quantize_f16(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
+                       float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
+  return run_nvfp4_quantize<InF16>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
 }
 
 int mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, uint8_t* q, uint8_t* sf,
@@ -658,11 +722,19 @@ int mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, uint8_
 }
 
 int bsp_amax_bf16(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
-  return amax_launch(x, n, amax, stream, true);
+  return amax_launch<InBf16>(x, n, amax, stream, true);
 }
 
 int bsp_amax_bf16_into(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
-  return amax_launch(x, n, amax, stream, false);
+  return amax_launch<InBf16>(x, n, amax, stream, false);
+}
+
+int bsp_amax_f16(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
+  return amax_launch<InF16>(x, n, amax, stream, true);
+}
+
+int bsp_amax_f16_into(const uint16_t* x, int64_t n, float* amax, bsp_stream_t stream) {
+  return amax_launch<InF16>(x, n, amax, stream, false);
 }
 
 int bsp_nvfp4_global_scale_max(const float* amax, float fp8_fp4_max, float* gs, float* inv_gs,

@@ -112,6 +112,12 @@ int bsp_amax_bf16(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream
  * Errors as bsp_amax_bf16. */
 int bsp_amax_bf16_into(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream);
 
+/* bsp_amax_bf16 / bsp_amax_bf16_into for fp16 data (the weight of an fp16
+ * model, convert_model_to_fp4): NaN counts as 0, +-inf as 65504.
+ *   x : fp16 [n] bit patterns, 16-byte aligned; the rest as bsp_amax_bf16. */
+int bsp_amax_f16(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream);
+int bsp_amax_f16_into(const uint16_t *x, int64_t n, float *amax, bsp_stream_t stream);
+
 /* NVFP4 encode scale from an amax, on the device (no host sync):
  *   gs = amax > 0 ? fl32(448*6 / amax) : 1.0     (convert_model_to_fp4; the
  *        all-zero guard is nvfp4_online.py _quantize_weight_nvfp4)
@@ -168,6 +174,16 @@ int bsp_nvfp4_alpha(const float *gs_x, const float *gs_w, float *alpha, bsp_stre
 int nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
                    const float *global_sf, int sf_mode, float *row_gs, float *row_inv_gs,
                    uint8_t *codes, uint8_t *sf, bsp_stream_t stream);
+
+/* The same for fp16 input.  nvfp4_config.py (_coerce_fp4_input_dtype and
+ * NVFP4QuantizeMethod.apply) feeds bf16 and fp16 activations to the quantizer
+ * as they are; x_i are the exact fp16 values, and the per-row amax treats NaN
+ * as 0 and +-inf as the largest finite fp16 (65504).
+ *   x : fp16 [M, K] bit patterns, row stride ld_x; other arguments, layouts
+ *       and errors as nvfp4_quantize. */
+int nvfp4_quantize_f16(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                       const float *global_sf, int sf_mode, float *row_gs, float *row_inv_gs,
+                       uint8_t *codes, uint8_t *sf, bsp_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * NVFP4 GEMM (nvfp4_qat_config.py, NVFP4QATQuantizeMethod.apply:

@@ -84,6 +84,14 @@ def lib() -> ctypes.CDLL:
         L.bspo_nvfp4_quantize_group.argtypes = [vp, f32, vp, vp]
         L.bspo_nvfp4_quantize.restype = i32
         L.bspo_nvfp4_quantize.argtypes = [vp, i64, i64, i64, vp, i32, vp, vp]
+        L.bspo_nvfp4_quantize_fmt.restype = i32
+        L.bspo_nvfp4_quantize_fmt.argtypes = [vp, i64, i64, i64, i32, vp, i32, vp, vp]
+        L.bspo_f16_value.restype = ctypes.c_double
+        L.bspo_f16_value.argtypes = [ctypes.c_uint16]
+        L.bspo_amax_fmt.restype = f32
+        L.bspo_amax_fmt.argtypes = [vp, i64, i32]
+        L.bspo_row_global_scales_fmt.restype = None
+        L.bspo_row_global_scales_fmt.argtypes = [vp, i64, i64, i64, i32, vp, vp]
         L.bspo_mxfp8_quantize_group.restype = None
         L.bspo_mxfp8_quantize_group.argtypes = [vp, vp, vp]
         L.bspo_mxfp8_quantize.restype = i32
@@ -167,9 +175,23 @@ def sf_bytes(rows: int, cols: int) -> int:
 
 
 # --------------------------------------------------------------------------- global scales
+FORMATS = {"bf16": 0, "f16": 1}
+
+
 def amax_bf16(x: np.ndarray) -> float:
     a = np.ascontiguousarray(x, dtype=np.uint16).reshape(-1)
     return float(np.float32(lib().bspo_amax_bf16(_ptr(a), a.size)))
+
+
+def amax_f16(x: np.ndarray) -> float:
+    """amax of fp16 bit patterns (NaN as 0, +-inf as 65504)."""
+    a = np.ascontiguousarray(x, dtype=np.uint16).reshape(-1)
+    return float(np.float32(lib().bspo_amax_fmt(_ptr(a), a.size, 1)))
+
+
+def f16_value(bits: int) -> float:
+    """Exact value of one fp16 bit pattern."""
+    return float(lib().bspo_f16_value(int(bits)))
 
 
 def nvfp4_global_scale(amax: float, fp8_fp4_max: float | None = None) -> np.float32:
@@ -179,13 +201,13 @@ def nvfp4_global_scale(amax: float, fp8_fp4_max: float | None = None) -> np.floa
     return np.float32(lib().bspo_nvfp4_global_scale_max(float(np.float32(amax)), float(np.float32(fp8_fp4_max))))
 
 
-def row_global_scales(x: np.ndarray):
+def row_global_scales(x: np.ndarray, fmt: str = "bf16"):
     """Per-row (per-token) encode scales gs[m] and decode factors 1/gs[m] (fp32)."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     M, K = x.shape
     gs = np.empty(M, np.float32)
     inv = np.empty(M, np.float32)
-    lib().bspo_row_global_scales(_ptr(x), M, K, K, _ptr(gs), _ptr(inv))
+    lib().bspo_row_global_scales_fmt(_ptr(x), M, K, K, FORMATS[fmt], _ptr(gs), _ptr(inv))
     return gs, inv
 
 
@@ -197,8 +219,8 @@ def _row_chunks(M: int, threads: int):
     return [(m0, min(M, m0 + per)) for m0 in range(0, M, per)]
 
 
-def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None = None):
-    """NVFP4 quantization of bf16 bit patterns ``x`` [M, K] along K.
+def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None = None, fmt: str = "bf16"):
+    """NVFP4 quantization of bf16 (or, fmt="f16", fp16) bit patterns ``x`` [M, K] along K.
 
     Returns (codes uint8 [M, K/2], sf uint8 [sf_bytes(M, K/16)] in the 128x4 map).
     ``gs`` is one fp32 encode scale, or one per row if ``per_row``.
@@ -221,8 +243,8 @@ def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None
     def run(rng):
         m0, m1 = rng
         gp = _ptr(g) + (4 * m0 if per_row else 0)
-        rc = L.bspo_nvfp4_quantize(_ptr(x) + 2 * m0 * K, m1 - m0, K, K, gp, int(per_row),
-                                   _ptr(codes) + m0 * (K // 2), _ptr(sf) + m0 * cols_p)
+        rc = L.bspo_nvfp4_quantize_fmt(_ptr(x) + 2 * m0 * K, m1 - m0, K, K, FORMATS[fmt], gp, int(per_row),
+                                       _ptr(codes) + m0 * (K // 2), _ptr(sf) + m0 * cols_p)
         assert rc == 0
 
     chunks = _row_chunks(M, _threads(threads))

@@ -63,6 +63,29 @@ double bspo_bf16_value(uint16_t bits)
     return sign ? -v : v;
 }
 
+/* fp16 (IEEE binary16): sign, 5-bit exponent (bias 15), 10-bit mantissa.
+ * Exact in double. */
+double bspo_f16_value(uint16_t bits)
+{
+    int sign = (bits >> 15) & 1;
+    int e = (bits >> 10) & 0x1F;
+    int m = bits & 0x3FF;
+    double v;
+    if (e == 0x1F)
+        v = (m == 0) ? INFINITY : NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -14 - 10);
+    else
+        v = ldexp(1.0 + m / 1024.0, e - 15);
+    return sign ? -v : v;
+}
+
+/* Input element formats of the quantizers: 0 = bf16, 1 = fp16. */
+static double elem_value(uint16_t bits, int fmt)
+{
+    return fmt ? bspo_f16_value(bits) : bspo_bf16_value(bits);
+}
+
 /* e2m1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0.  No inf/NaN. */
 double bspo_e2m1_value(int code)
 {
@@ -200,19 +223,25 @@ int64_t bspo_sf_bytes(int64_t rows, int64_t cols)
 
 /* amax of |x| as the pages compute it: abs().nan_to_num().amax() on the bf16
  * tensor -- NaN counts as 0 and +-inf as the largest finite bf16 value. */
-float bspo_amax_bf16(const uint16_t *x, int64_t n)
+float bspo_amax_fmt(const uint16_t *x, int64_t n, int fmt)
 {
+    double top = fmt ? bspo_f16_value(0x7BFF) : bspo_bf16_value(0x7F7F); /* largest finite */
     double amax = 0.0;
     for (int64_t i = 0; i < n; ++i) {
-        double a = fabs(bspo_bf16_value(x[i]));
+        double a = fabs(elem_value(x[i], fmt));
         if (isnan(a))
             a = 0.0;
         else if (isinf(a))
-            a = bspo_bf16_value(0x7F7F);
+            a = top;
         if (a > amax)
             amax = a;
     }
-    return (float)amax; /* exact: a bf16 value */
+    return (float)amax; /* exact: a bf16 or fp16 value */
+}
+
+float bspo_amax_bf16(const uint16_t *x, int64_t n)
+{
+    return bspo_amax_fmt(x, n, 0);
 }
 
 /* Encode global scale fp8_fp4_max/amax in fp32, fp8_fp4_max = e4m3_max * 6;
@@ -234,16 +263,22 @@ float bspo_nvfp4_global_scale(float amax)
 
 /* Per-row (per-token) scales: gs[m] from the row amax; inv[m] = fl32(1/gs[m]),
  * the decode factor the GEMM applies to row m. */
-void bspo_row_global_scales(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
-                            float *gs, float *inv_gs)
+void bspo_row_global_scales_fmt(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int fmt,
+                                float *gs, float *inv_gs)
 {
     for (int64_t m = 0; m < M; ++m) {
-        float g = bspo_nvfp4_global_scale(bspo_amax_bf16(x + m * ld_x, K));
+        float g = bspo_nvfp4_global_scale(bspo_amax_fmt(x + m * ld_x, K, fmt));
         if (gs)
             gs[m] = g;
         if (inv_gs)
             inv_gs[m] = 1.0f / g;
     }
+}
+
+void bspo_row_global_scales(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                            float *gs, float *inv_gs)
+{
+    bspo_row_global_scales_fmt(x, M, K, ld_x, 0, gs, inv_gs);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -271,13 +306,13 @@ void bspo_nvfp4_quantize_group(const float *x, float gs, uint8_t *sfb_out, uint8
     *sfb_out = (uint8_t)sfb;
 }
 
-/* x: bf16 [M, K] with row stride ld_x (elements).  gs: one value, or one per
- * row when per_row != 0.  codes: [M, K/2] bytes, element 2j in the low nibble
- * of byte j and element 2j+1 in the high nibble.  sf: bspo_sf_bytes(M, K/16)
- * bytes in the 128x4 tile map; padding rows and columns are 0.
- * Returns 0, or -1 when K is not a multiple of 16. */
-int bspo_nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
-                        const float *gs, int per_row, uint8_t *codes, uint8_t *sf)
+/* x: bf16 (fmt 0) or fp16 (fmt 1) [M, K] with row stride ld_x (elements).
+ * gs: one value, or one per row when per_row != 0.  codes: [M, K/2] bytes,
+ * element 2j in the low nibble of byte j and element 2j+1 in the high nibble.
+ * sf: bspo_sf_bytes(M, K/16) bytes in the 128x4 tile map; padding rows and
+ * columns are 0.  Returns 0, or -1 when K is not a multiple of 16. */
+int bspo_nvfp4_quantize_fmt(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int fmt,
+                            const float *gs, int per_row, uint8_t *codes, uint8_t *sf)
 {
     if (K % 16 != 0 || M < 0)
         return -1;
@@ -289,7 +324,7 @@ int bspo_nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
         float g = per_row ? gs[m] : gs[0];
         for (int64_t c = 0; c < cols; ++c) {
             for (int i = 0; i < 16; ++i)
-                xs[i] = (float)bspo_bf16_value(x[m * ld_x + c * 16 + i]);
+                xs[i] = (float)elem_value(x[m * ld_x + c * 16 + i], fmt); /* exact */
             uint8_t sfb;
             bspo_nvfp4_quantize_group(xs, g, &sfb, q);
             sf[bspo_sf_offset(m, c, cols_p)] = sfb;
@@ -298,6 +333,12 @@ int bspo_nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
         }
     }
     return 0;
+}
+
+int bspo_nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                        const float *gs, int per_row, uint8_t *codes, uint8_t *sf)
+{
+    return bspo_nvfp4_quantize_fmt(x, M, K, ld_x, 0, gs, per_row, codes, sf);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -1,8 +1,9 @@
-"""Global-scale variants on the GPU vs the oracle: the 4over6 numerator
-(sgl-project sglang nvfp4_online.py, _quantize_weight_nvfp4: e4m3_max = 256)
-and one scale shared by a gated w1/w3 pair (the same file,
-process_loaded_weight).  Scales, codes and scale bytes bit-exact; GEMMs within
-the tolerance of tests/_gpu.py."""
+"""Variants of the NVFP4 path on the GPU vs the oracle: the 4over6 global
+scale numerator (sgl-project sglang nvfp4_online.py, _quantize_weight_nvfp4:
+e4m3_max = 256), one scale shared by a gated w1/w3 pair (the same file,
+process_loaded_weight), and fp16 input (hao-ai-lab-FastVideo nvfp4_config.py,
+_coerce_fp4_input_dtype).  Scales, codes and scale bytes bit-exact; GEMMs
+within the tolerance of tests/_gpu.py."""
 import numpy as np
 import pytest
 import torch
@@ -105,3 +106,78 @@ def test_shared_scale_group_layers(per_token):
                                              bias=None)
         assert_gemm_close(D, ref, bound, f"shared-scale layer per_token={per_token}")
     assert api.device_status() == 0
+
+
+# --------------------------------------------------------------------------- fp16 input
+def _f16(rows, K, seed, std=1.0, special=False):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((rows, K)) * std).astype(np.float16).view(np.uint16)
+    if special and rows * K >= 64:
+        flat = x.reshape(-1)
+        n = flat.size
+        flat[rng.integers(0, n, n // 20)] = 0x8000   # -0
+        flat[rng.integers(0, n, n // 50)] = 0x0001   # smallest subnormal
+        flat[rng.integers(0, n, n // 50)] = 0x8203   # negative subnormal
+        flat[rng.integers(0, n, n // 100)] = 0x7BFF  # largest finite, 65504
+        if K >= 32:
+            x[0, :32] = 0
+    return x
+
+
+def _up_f16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.float16).to(DEV)
+
+
+F16_SHAPES = [(1, 16), (7, 48), (129, 64), (300, 1536), (257, 5120), (64, 13824), (130, 80)]
+
+
+@pytest.mark.parametrize("M,K", F16_SHAPES)
+@pytest.mark.parametrize("per_row", [False, True])
+def test_f16_quantize_bit_exact(M, K, per_row):
+    x = _f16(M, K, seed=M * 3 + K, special=True)
+    if per_row:
+        q = api.nvfp4_quantize(_up_f16(x), per_row=True)
+        gs, inv = oracle.row_global_scales(x, fmt="f16")
+        assert np.array_equal(down(q.row_gs), gs) and np.array_equal(down(q.row_inv_gs), inv)
+        codes, sf = oracle.nvfp4_quantize(x, gs, per_row=True, fmt="f16")
+    else:
+        g = np.float32(0.37109375)
+        q = api.nvfp4_quantize(_up_f16(x), torch.tensor([g], device=DEV))
+        codes, sf = oracle.nvfp4_quantize(x, g, fmt="f16")
+    assert np.array_equal(down(q.codes), codes)
+    assert np.array_equal(down(q.sf), sf)
+
+
+def test_f16_amax():
+    x = _f16(333, 520, seed=42, std=30.0, special=True)
+    x[5, 7] = 0xFC00  # -inf -> 65504
+    a = api.amax(_up_f16(x))
+    assert down(a)[0] == np.float32(oracle.amax_f16(x))
+    y = _f16(10, 64, seed=43)
+    y[0, 0] = 0x7E00  # NaN counts as 0
+    b = api.amax(_up_f16(y))
+    assert down(b)[0] == np.float32(oracle.amax_f16(y))
+
+
+@pytest.mark.parametrize("per_token", [False, True])
+def test_f16_linear(per_token):
+    M, N, K = 200, 512, 1536
+    A, W = _f16(M, K, seed=44), _f16(N, K, seed=45, std=0.02)
+    layer = api.NVFP4Linear(_up_f16(W), per_token=per_token)
+    g_ref = oracle.nvfp4_global_scale(oracle.amax_f16(W))
+    assert down(layer.gs_w)[0] == g_ref
+    cb, sb = oracle.nvfp4_quantize(W, g_ref, fmt="f16")
+    assert np.array_equal(down(layer.weight.codes), cb)
+    D = layer(_up_f16(A))
+    assert D.dtype == torch.bfloat16
+    assert api.device_status() == 0
+    if per_token:
+        gs_rows, inv_rows = oracle.row_global_scales(A, fmt="f16")
+        ca, sa = oracle.nvfp4_quantize(A, gs_rows, per_row=True, fmt="f16")
+        alpha, rs = np.float32(1) / g_ref, inv_rows
+    else:
+        ca, sa = oracle.nvfp4_quantize(A, np.float32(1.0), fmt="f16")
+        alpha, rs = np.float32(1) / (np.float32(1) * g_ref), None
+    ref, bound = oracle.linear_reference(oracle.nvfp4_dequantize(ca, sa, K), oracle.nvfp4_dequantize(cb, sb, K),
+                                         alpha=alpha, row_scale=rs, bias=None)
+    assert_gemm_close(D, ref, bound, f"fp16 linear per_token={per_token}")

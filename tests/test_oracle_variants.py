@@ -53,3 +53,56 @@ def test_shared_scale_pair_equals_split_of_concatenation():
     c3, s3 = oracle.nvfp4_quantize(w3, gs)
     assert np.array_equal(c_cat, np.concatenate([c1, c3]))
     assert np.array_equal(s_cat, np.concatenate([s1, s3]))
+
+
+# --------------------------------------------------------------------------- fp16 input
+# nvfp4_config.py (_coerce_fp4_input_dtype, NVFP4QuantizeMethod.apply) feeds
+# fp16 activations to the quantizer as they are.
+
+def test_f16_decoder_matches_numpy_on_every_pattern():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16_value(int(b)) for b in bits])
+    r = ref
+    same = (got == r) | (np.isnan(got) & np.isnan(r))
+    assert same.all()
+
+
+def test_f16_amax_nan_and_inf():
+    x = np.array([0x3C00, 0xBC00, 0x7E00, 0x4000], np.uint16)  # 1, -1, NaN, 2
+    assert oracle.amax_f16(x) == 2.0
+    assert oracle.amax_f16(np.array([0x3C00, 0xFC00], np.uint16)) == 65504.0  # -inf -> largest finite
+    assert oracle.amax_f16(np.array([0x7E00, 0x8000], np.uint16)) == 0.0
+
+
+def test_f16_and_bf16_agree_on_shared_values():
+    """Values representable in both formats quantize identically."""
+    rng = np.random.default_rng(41)
+    vals = (rng.integers(-64, 65, size=(130, 96)) / 8.0).astype(np.float32)  # k/8: exact in both
+    b16 = wl.f32_to_bf16_bits(vals)
+    f16 = vals.astype(np.float16).view(np.uint16)
+    for per_row in (False, True):
+        if per_row:
+            gs_b, _ = oracle.row_global_scales(b16)
+            gs_f, _ = oracle.row_global_scales(f16, fmt="f16")
+            assert np.array_equal(gs_b, gs_f)
+        else:
+            gs_b = gs_f = oracle.nvfp4_global_scale(oracle.amax_bf16(b16))
+        cb, sb = oracle.nvfp4_quantize(b16, gs_b, per_row=per_row)
+        cf, sf = oracle.nvfp4_quantize(f16, gs_f, per_row=per_row, fmt="f16")
+        assert np.array_equal(cb, cf) and np.array_equal(sb, sf)
+
+
+def test_f16_precision_is_used():
+    """1.25 + 2^-10 is just above the e2m1 tie between 1 and 1.5: in fp16 it
+    rounds up to 1.5 (code 3); rounded to bf16 first it is the tie itself,
+    which goes to the even code 2 (1.0).  Group scale 1: the 6.0 sets amax."""
+    f16 = np.zeros((1, 16), np.uint16)
+    f16[0, 0] = np.float16(6.0).view(np.uint16)
+    f16[0, 1] = np.float16(1.2509765625).view(np.uint16)
+    codes, sf = oracle.nvfp4_quantize(f16, np.float32(1.0), fmt="f16")
+    assert sf[0] == 0x38  # e4m3 1.0
+    assert codes[0, 0] == (0x7 | (0x3 << 4))
+    b16 = wl.f32_to_bf16_bits(np.array([[6.0, 1.2509765625] + [0.0] * 14], np.float32))
+    codes_b, _ = oracle.nvfp4_quantize(b16, np.float32(1.0))
+    assert codes_b[0, 0] == (0x7 | (0x2 << 4))
