@@ -38,6 +38,8 @@ SIGNATURES = {
     "bsp_nvfp4_alpha": (_i32, [_vp, _vp, _vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_f16": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nvfp4_rmsnorm_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, ctypes.c_float, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
+                                      _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "mxfp8_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "mxfp8_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _i64, _vp]),

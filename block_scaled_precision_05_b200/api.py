@@ -192,6 +192,38 @@ def nvfp4_quantize(x: torch.Tensor, global_sf: torch.Tensor | None = None, per_r
     return out
 
 
+def nvfp4_rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                           global_sf: torch.Tensor | None = None, per_row: bool = False,
+                           out: NVFP4Tensor | None = None, rstd_out: torch.Tensor | None = None) -> NVFP4Tensor:
+    """RMSNorm(x) * gamma, rounded to bf16 and quantized to NVFP4 in one kernel
+    (the normalised activation is never written).  bf16 x [..., K], gamma [K]."""
+    _require_cuda(x, gamma, global_sf, rstd_out)
+    if x.dtype != torch.bfloat16 or gamma.dtype != torch.bfloat16:
+        raise TypeError("nvfp4_rmsnorm_quantize expects bf16 x and gamma")
+    x2 = _as_2d(x)
+    M, K = x2.shape
+    if gamma.numel() != K or not gamma.is_contiguous():
+        raise ValueError(f"gamma must be a contiguous [{K}] tensor")
+    if rstd_out is not None and (rstd_out.dtype != torch.float32 or rstd_out.numel() != M):
+        raise ValueError(f"rstd_out must be an fp32 [{M}] tensor")
+    dev = x2.device
+    if out is None:
+        out = NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+        if per_row:
+            out.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
+            out.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
+    if not per_row and global_sf is None:
+        raise ValueError("per-tensor quantization needs global_sf (fp32 device tensor)")
+    st = nat.lib().nvfp4_rmsnorm_quantize(
+        _ptr(x2), M, K, x2.stride(0), _ptr(gamma), float(eps), None if per_row else _ptr(global_sf),
+        nat.BSP_SF_PER_ROW if per_row else nat.BSP_SF_PER_TENSOR,
+        _ptr(out.row_gs) if per_row else None, _ptr(out.row_inv_gs) if per_row else None, _ptr(rstd_out),
+        _ptr(out.codes), _ptr(out.sf), _stream())
+    nat.check(st, "nvfp4_rmsnorm_quantize")
+    return out
+
+
 def mxfp8_quantize(x: torch.Tensor, out: MXFP8Tensor | None = None) -> MXFP8Tensor:
     """Quantize bf16 [..., K] to MXFP8 along K (leading dims flattened)."""
     _require_cuda(x)
@@ -302,6 +334,12 @@ class NVFP4Linear:
     def quantize_input(self, x: torch.Tensor) -> NVFP4Tensor:
         x = coerce_input(x)
         return nvfp4_quantize(x, None if self.per_token else self.gs_x, per_row=self.per_token)
+
+    def rmsnorm_quantize_input(self, x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6) -> NVFP4Tensor:
+        """RMSNorm(x) * gamma quantized for this layer in one kernel: pass the
+        result as `pre_quantized` (the fused norm+quant producer)."""
+        return nvfp4_rmsnorm_quantize(coerce_bf16(x), coerce_bf16(gamma).contiguous(), eps,
+                                      None if self.per_token else self.gs_x, per_row=self.per_token)
 
     def __call__(self, x: torch.Tensor, pre_quantized: NVFP4Tensor | None = None,
                  out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:

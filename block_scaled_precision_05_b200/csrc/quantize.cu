@@ -412,6 +412,110 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// RMSNorm fused into the NVFP4 quantizer (the producer of a pre-quantized
+// activation: hao-ai-lab-FastVideo nvfp4_config.py, NVFP4QuantizeMethod.apply
+// with `pre_quantized` from a fused norm+quant call).  Per row:
+//   ms   = mean(x^2)  (products exact; sum in fp64, any order; one rounding
+//          to fp32 at the end)
+//   rstd = fl32(1 / sqrt(fl32(ms + eps)))     (correctly rounded)
+//   y_k  = bf16(fl32(fl32(x_k * rstd) * gamma_k))
+// and y is quantized exactly as nvfp4_quantize quantizes a bf16 input, so the
+// result equals RMSNorm to bf16 followed by nvfp4_quantize, without writing y.
+// One warp per row: pass 1 the sum of squares, pass 2 (per-token scales) the
+// row amax of y, pass 3 the groups; passes 2 and 3 re-read the row from cache.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+__device__ __forceinline__ double sumsq8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  double s = 0.0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = InBf16::values2(w[i]);
+    s = fma(static_cast<double>(f.x), static_cast<double>(f.x), s);
+    s = fma(static_cast<double>(f.y), static_cast<double>(f.y), s);
+  }
+  return s;
+}
+
+// Eight normalised outputs as bf16 pairs: bf16(fl32(fl32(x * rstd) * gamma)).
+__device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, float rstd) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 xf = InBf16::values2(xw[i]), gf = InBf16::values2(gw[i]);
+    const float lo = __fmul_rn(__fmul_rn(xf.x, rstd), gf.x);
+    const float hi = __fmul_rn(__fmul_rn(xf.y, rstd), gf.y);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    memcpy(&o[i], &h, 4);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <bool kPerRow>
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const uint16_t* __restrict__ gamma,
+    float eps, const float* __restrict__ gs_ptr, float* __restrict__ row_gs, float* __restrict__ row_inv,
+    float* __restrict__ row_rstd, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
+  const uint32_t lane = lane_id();
+  const int64_t groups = K >> 4, cols4 = (groups + 3) & ~int64_t(3);
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+
+  for (int64_t r = warp; r < Mp; r += nwarps) {
+    const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
+    if (r >= M) {  // scale padding rows
+      for (int64_t c = lane; c < cols4; c += 32) sf[sfb_row + (c >> 2) * 512 + (c & 3)] = 0;
+      continue;
+    }
+    const uint16_t* row = x + r * ld_x;
+    double acc = 0.0;
+    for (int64_t g = lane; g < groups; g += 32) acc += sumsq8(ldg16(row + g * 16)) + sumsq8(ldg16(row + g * 16 + 8));
+    acc = warp_sum_f64(acc);
+    const float ms = __double2float_rn(acc / static_cast<double>(K));
+    const float rstd = __frsqrt_rn(__fadd_rn(ms, eps));
+    if (row_rstd != nullptr && lane == 0) row_rstd[r] = rstd;
+
+    float gs = gs_tensor;
+    if (kPerRow) {
+      uint32_t mag = 0;
+      for (int64_t g = lane; g < groups; g += 32) {
+        const uint4 y0 = rmsnorm8(ldg16(row + g * 16), ldg16(gamma + g * 16), rstd);
+        const uint4 y1 = rmsnorm8(ldg16(row + g * 16 + 8), ldg16(gamma + g * 16 + 8), rstd);
+        mag = max(mag, max(max_sane_mag8<InBf16>(y0), max_sane_mag8<InBf16>(y1)));
+      }
+      mag = warp_max(mag);
+      gs = global_scale_from_mag<InBf16>(mag);
+      if (lane == 0) {
+        if (row_gs) row_gs[r] = gs;
+        if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
+      }
+    }
+    for (int64_t c = lane; c < cols4; c += 32) {
+      uint32_t sfb = 0;
+      if (c < groups) {
+        const uint4 y0 = rmsnorm8(ldg16(row + c * 16), ldg16(gamma + c * 16), rstd);
+        const uint4 y1 = rmsnorm8(ldg16(row + c * 16 + 8), ldg16(gamma + c * 16 + 8), rstd);
+        float inv;
+        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv);
+        uint2 w;
+        w.x = nvfp4_codes8<InBf16>(y0, inv);
+        w.y = nvfp4_codes8<InBf16>(y1, inv);
+        *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
+      }
+      sf[sfb_row + (c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfb);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // MXFP8.
 // ---------------------------------------------------------------------------
 // Scale exponent e (and the multiplier 2^-e) of a group with |amax| bits `mag`.
@@ -700,6 +804,32 @@ int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const 
 int nvfp4_quantize_f16(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
                        float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
   return run_nvfp4_quantize<InF16>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
+}
+
+int nvfp4_rmsnorm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const uint16_t* gamma, float eps,
+                           const float* global_sf, int sf_mode, float* row_gs, float* row_inv_gs, float* row_rstd,
+                           uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K) return BSP_ERR_INVALID_ARG;
+  if (sf_mode != BSP_SF_PER_TENSOR && sf_mode != BSP_SF_PER_ROW) return BSP_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !(eps <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
+  if (M == 0) return BSP_OK;
+  if (!x || !gamma || !codes || !sf || (sf_mode == BSP_SF_PER_TENSOR && !global_sf)) return BSP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(codes) || !aligned16(sf) || ld_x % 8 != 0)
+    return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  const int64_t Mp = round_up(M, 128);
+  if (sf_mode == BSP_SF_PER_ROW) {
+    auto k = nvfp4_rmsnorm_quant_kernel<true>;
+    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, row_gs,
+                                                               row_inv_gs, row_rstd, codes, sf);
+  } else {
+    auto k = nvfp4_rmsnorm_quant_kernel<false>;
+    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, nullptr,
+                                                               nullptr, row_rstd, codes, sf);
+  }
+  return launch_status();
 }
 
 int mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, uint8_t* q, uint8_t* sf,

@@ -185,6 +185,28 @@ int nvfp4_quantize_f16(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
                        const float *global_sf, int sf_mode, float *row_gs, float *row_inv_gs,
                        uint8_t *codes, uint8_t *sf, bsp_stream_t stream);
 
+/* RMSNorm fused into the NVFP4 quantizer: the producer of the pre-quantized
+ * activation that NVFP4QuantizeMethod.apply (nvfp4_config.py) accepts from a
+ * fused norm+quant call.  The pages name the fused call but not its norm; this
+ * is RMSNorm with a weight, whose normalised output is quantized as if it had
+ * been written as bf16 and passed to nvfp4_quantize.  Per row m:
+ *   ms   = mean_k x_k^2  (exact products, summed in fp64 in any order, one
+ *          rounding to fp32)
+ *   rstd = fl32(1 / sqrt(fl32(ms + eps)))   (correctly rounded)
+ *   y_k  = bf16(fl32(fl32(x_k * rstd) * gamma_k))
+ *   then y is quantized as nvfp4_quantize does (per-tensor global_sf, or per
+ *   row gs[m] from the row amax of y), without y being stored.
+ *   x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf:
+ *              as nvfp4_quantize (bf16 x)
+ *   gamma    : bf16 [K], 16-byte aligned
+ *   eps      : host fp32, finite and >= 0
+ *   row_rstd : fp32 [M] receives rstd of each row (may be NULL)
+ * Errors as nvfp4_quantize; eps negative or not finite -> INVALID_ARG. */
+int nvfp4_rmsnorm_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                           const uint16_t *gamma, float eps, const float *global_sf, int sf_mode,
+                           float *row_gs, float *row_inv_gs, float *row_rstd, uint8_t *codes,
+                           uint8_t *sf, bsp_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * NVFP4 GEMM (nvfp4_qat_config.py, NVFP4QATQuantizeMethod.apply:
  * mm_fp4(x_fp4, w_fp4.T, x_scale, w_scale.T, 1/(gs_x*gs_w), bf16) then

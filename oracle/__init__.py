@@ -23,9 +23,11 @@ Parity pins for every function live in ``tests/test_oracle_*.py``.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 from concurrent.futures import ThreadPoolExecutor
+from fractions import Fraction
 
 import numpy as np
 
@@ -329,3 +331,104 @@ def linear_reference(decA: np.ndarray, decB: np.ndarray, alpha: float = 1.0,
     if bias is not None:
         y = y + bf16_bits_to_f64(bias)[None, :]
     return y, np.abs(f) * mag
+
+
+# --------------------------------------------------------------------------- RMSNorm before the quantizer
+# The producer of a pre-quantized activation (hao-ai-lab-FastVideo
+# nvfp4_config.py, NVFP4QuantizeMethod.apply: `pre_quantized` from "fused
+# norm+quant" calls).  The pages do not print the norm; the reading is RMSNorm
+# with a weight, its output rounded to bf16 and then quantized as any bf16
+# activation:
+#   ms   = (1/K) sum_k x_k^2            (exact, then rounded once to fp32)
+#   rstd = RN32(1 / sqrt(RN32(ms + eps)))
+#   y_k  = bf16(RN32(RN32(x_k * rstd) * gamma_k))
+def _rn_f32_ratio(p: int, q: int) -> np.float32:
+    """The fp32 nearest to p/q (p >= 0, q > 0 integers), ties to even."""
+    if p == 0:
+        return np.float32(0.0)
+    # e = floor(log2(p/q))
+    e = p.bit_length() - q.bit_length()
+    if (p << max(0, -e)) < (q << max(0, e)):
+        e -= 1
+    if e > 127:
+        return np.float32(np.inf)
+    shift = 23 - max(e, -126)  # fraction bits kept: 24 for normals, fewer below 2^-126
+    num, den = (p << shift, q) if shift >= 0 else (p, q << -shift)
+    n, rem = divmod(num, den)
+    if 2 * rem > den or (2 * rem == den and (n & 1)):
+        n += 1
+    return np.float32(math.ldexp(float(n), -shift))  # n < 2^25: exact in fp64 and fp32
+
+
+def _rsqrt_rn32(t: np.float32) -> np.float32:
+    """RN32(1/sqrt(t)) for a positive fp32 t, decided exactly."""
+    tf = Fraction(float(t))
+    c = np.float32(1.0 / math.sqrt(float(t)))
+    for _ in range(4):  # the fp64 estimate is within an fp32 ulp: at most one step either way
+        up = np.nextafter(c, np.float32(np.inf), dtype=np.float32)
+        dn = np.nextafter(c, np.float32(0), dtype=np.float32)
+        mid_up = (Fraction(float(c)) + Fraction(float(up))) / 2
+        mid_dn = (Fraction(float(c)) + Fraction(float(dn))) / 2
+        # z = t^(-1/2) > m  <=>  m^2 t < 1
+        if mid_up * mid_up * tf < 1 or (mid_up * mid_up * tf == 1 and (np.float32(up).view(np.uint32) & 1) == 0):
+            c = up
+        elif mid_dn * mid_dn * tf > 1 or (mid_dn * mid_dn * tf == 1 and (np.float32(dn).view(np.uint32) & 1) == 0):
+            c = dn
+        else:
+            return c
+    raise AssertionError("rsqrt rounding did not settle")
+
+
+def _bf16_exact_parts(bits: np.ndarray):
+    """(m, e) integers with value = m * 2^e for each bf16 pattern (finite)."""
+    b = np.asarray(bits, dtype=np.int64)
+    sign = np.where(b & 0x8000, -1, 1)
+    ex = (b >> 7) & 0xFF
+    man = b & 0x7F
+    m = np.where(ex == 0, man, man | 0x80) * sign
+    e = np.where(ex == 0, -133, ex - 134)
+    return m, e
+
+
+def rmsnorm_rstd(x: np.ndarray, eps: float) -> np.ndarray:
+    """Exact-reading rstd per row of bf16 bit patterns x [M, K] (fp32 [M])."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    out = np.empty(M, np.float32)
+    e32 = np.float32(eps)
+    for r in range(M):
+        m, e = _bf16_exact_parts(x[r])
+        emin = int(e.min())
+        s = 0
+        for mi, ei in zip(m.tolist(), e.tolist()):
+            s += (mi * mi) << (2 * (ei - emin))
+        # ms = s * 2^(2 emin) / K
+        if 2 * emin >= 0:
+            ms = _rn_f32_ratio(s << (2 * emin), K)
+        else:
+            ms = _rn_f32_ratio(s, K << (-2 * emin))
+        t = np.float32(ms + e32)  # fp32 add, round to nearest even
+        out[r] = _rsqrt_rn32(t)
+    return out
+
+
+def rmsnorm_bf16(x: np.ndarray, gamma: np.ndarray, rstd: np.ndarray) -> np.ndarray:
+    """y = bf16(RN32(RN32(x * rstd) * gamma)) as bf16 bit patterns [M, K]."""
+    xv = bf16_bits_to_f64(x).astype(np.float32)  # exact
+    gv = bf16_bits_to_f64(gamma).astype(np.float32)
+    y = (xv * np.asarray(rstd, np.float32)[:, None]) * gv[None, :]  # two fp32 multiplies, each rounded
+    return bf16_round(y.astype(np.float64))
+
+
+def rmsnorm_quantize(x: np.ndarray, gamma: np.ndarray, eps: float, gs=None, per_row: bool = False, rstd=None):
+    """RMSNorm to bf16, then NVFP4 quantization.  `rstd` may be given (e.g. the
+    values a kernel reports) to check everything downstream of the reduction.
+    Returns (codes, sf, rstd, row_gs or None, row_inv or None)."""
+    rstd = rmsnorm_rstd(x, eps) if rstd is None else np.asarray(rstd, np.float32)
+    y = rmsnorm_bf16(x, gamma, rstd)
+    if per_row:
+        g, inv = row_global_scales(y)
+        codes, sf = nvfp4_quantize(y, g, per_row=True)
+        return codes, sf, rstd, g, inv
+    codes, sf = nvfp4_quantize(y, gs)
+    return codes, sf, rstd, None, None

@@ -65,6 +65,11 @@ def test_host_validation_rejects_bad_arguments():
     assert L.mxfp8_gemm(p, p, p, p, 4, 8, 48, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_amax_bf16(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_amax_bf16_into(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
+    for bad in (-1.0, float("inf"), float("nan")):  # eps
+        assert L.nvfp4_rmsnorm_quantize(p, 4, 32, 32, p, bad, p, 0, None, None, None, p, p, None) == \
+            nat.BSP_ERR_INVALID_ARG
+    assert L.nvfp4_rmsnorm_quantize(p, 4, 24, 24, p, 0.0, p, 0, None, None, None, p, p, None) == \
+        nat.BSP_ERR_INVALID_ARG  # K % 16
     for bad in (0.0, -2688.0, float("inf"), float("nan")):
         assert L.bsp_nvfp4_global_scale_max(p, bad, p, p, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_nvfp4_global_scale_max(p, 1536.0, None, None, None) == nat.BSP_ERR_INVALID_ARG
