@@ -160,6 +160,29 @@ def make_workload(name: str):
     raise SystemExit(f"unknown --config {name}")
 
 
+NORM_EPS = 1e-6
+
+
+def norm_gamma(lin):
+    """Seeded RMSNorm weight for --norm rmsnorm: 1 + 0.2 N(0, 1), bf16 bits."""
+    from block_scaled_precision_05_b200 import workloads as wl
+    rng = np.random.default_rng(77)
+    return wl.f32_to_bf16_bits((1.0 + 0.2 * rng.standard_normal(lin.K)).astype(np.float32))
+
+
+def apply_input_format(lin, kind, fmt):
+    """fp16 activations (--input f16, NVFP4 only): the workload's bf16 values
+    rounded to fp16 on the host; the oracle quantizes the same fp16 bits."""
+    lin.fmt = "bf16"
+    if fmt == "f16":
+        if kind != "nvfp4":
+            raise SystemExit("--input f16 applies to the NVFP4 workloads")
+        f32 = (np.ascontiguousarray(lin.A).astype(np.uint32) << 16).view(np.float32)
+        lin.A = f32.astype(np.float16).view(np.uint16)
+        lin.fmt = "f16"
+    return lin
+
+
 def describe(lin, kind):
     d = {"workload": f"{lin.name}: {kind.upper()} linear A[{lin.M},{lin.K}] x W[{lin.N},{lin.K}]^T"
                      + (" + bias" if lin.bias is not None else "")
@@ -188,11 +211,17 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     lin, kind = make_workload(args.config)
+    lin = apply_input_format(lin, kind, args.input)
+    a_dtype = torch.float16 if lin.fmt == "f16" else torch.bfloat16
 
-    def up(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    def up(a, dtype=torch.bfloat16):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dtype).to(dev)
 
-    A = up(lin.A)
+    A = up(lin.A, a_dtype)
+    if args.norm == "rmsnorm":
+        if kind != "nvfp4" or lin.fmt != "bf16":
+            raise SystemExit("--norm rmsnorm applies to the bf16 NVFP4 workloads")
+        gamma = up(norm_gamma(lin))
     W = up(lin.W)
     bias = None if lin.bias is None else up(lin.bias)
     if kind == "nvfp4":
@@ -218,7 +247,10 @@ def run_ours(args, rank, world, local_rank):
     D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
 
     def quantize():
-        if kind == "nvfp4":
+        if args.norm == "rmsnorm":
+            api.nvfp4_rmsnorm_quantize(A, gamma, NORM_EPS, None if lin.per_token else layer.gs_x,
+                                       per_row=lin.per_token, out=xq)
+        elif kind == "nvfp4":
             api.nvfp4_quantize(A, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=xq)
         else:
             api.mxfp8_quantize(A, out=xq)
@@ -294,14 +326,17 @@ def run_ours(args, rank, world, local_rank):
     del g_warm, g_timed, g_split, ev_warm
 
     # ---- end to end through the public API: pinned host A in, D back to pinned host
-    A_host = torch.from_numpy(np.ascontiguousarray(lin.A).view(np.int16)).view(torch.bfloat16).pin_memory()
+    A_host = torch.from_numpy(np.ascontiguousarray(lin.A).view(np.int16)).view(a_dtype).pin_memory()
     D_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     A_dev = torch.empty_like(A)
     e2e_steps = max(1, min(args.steps, 20))
 
     def e2e_step():
         A_dev.copy_(A_host, non_blocking=True)
-        y = layer(A_dev)
+        if args.norm == "rmsnorm":
+            y = layer(A_dev, pre_quantized=layer.rmsnorm_quantize_input(A_dev, gamma, NORM_EPS))
+        else:
+            y = layer(A_dev)
         D_host.copy_(y, non_blocking=True)
 
     for _ in range(2):
@@ -331,7 +366,8 @@ def run_ours(args, rank, world, local_rank):
     ratio = FP4_PER_BF16 if kind == "nvfp4" else FP8_PER_BF16
     tensor_peak = peaks["bf16_tflops"] * ratio
     hbm_peak = peaks["hbm_gbs"]
-    wname = args.config
+    wname = args.config + ("_rmsnorm" if args.norm == "rmsnorm" else "")
+    qname = "nvfp4_rmsnorm_quantize" if args.norm == "rmsnorm" else f"{kind}_quantize"
     if M <= 128:
         # skinny M: the GEMM streams the weight once; bound by HBM
         gb = (M * K + N * K) * (0.5 if kind == "nvfp4" else 1.0) + (M + N) * (K // 16 if kind == "nvfp4" else K // 32) \
@@ -348,12 +384,15 @@ def run_ours(args, rank, world, local_rank):
                 "peak_source": f"{peak_src}: bf16_tflops (burst) x {ratio:g} nominal {kind} ratio",
                 "algorithmic": f"2*M*N*K = {flops:.4g} flop per launch"}
     else:
-        roof = {"kernel": f"{kind}_quantize", "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4), "traffic": traffic_for(f"{kind}_quantize", wname),
+        roof = {"kernel": qname, "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4), "traffic": traffic_for(qname, wname),
                 "peak_source": f"{peak_src}: hbm_gbs", "algorithmic": f"{qb} bytes per launch"}
 
     cfg = describe(lin, kind)
     cfg["parallelism"] = f"replicas x{world}"
+    cfg["activation_dtype"] = "fp16" if lin.fmt == "f16" else "bf16"
+    if args.norm == "rmsnorm":
+        cfg["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
     if kind == "nvfp4":
         cfg["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
     out = {
@@ -362,7 +401,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "nvfp4" if kind == "nvfp4" else "mxfp8", "data": "synthetic (seeded numpy)",
         "config": cfg, "roofline": roof,
         "kernels": {
-            f"{kind}_quantize": {"ms": round(q_ms, 5), "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / hbm_peak, 4)},
+            qname: {"ms": round(q_ms, 5), "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / hbm_peak, 4)},
             f"{kind}_gemm": {"ms": round(g_ms, 5), "TFLOP/s": round(g_tflops, 1),
                              "frac_tensor_peak": round(g_tflops / tensor_peak, 4)},
         },
@@ -373,7 +412,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = oracle_baseline(lin, kind, budget_s=args.cpu_budget, four_over_six=args.four_over_six)
+        out["cpu_baseline"] = oracle_baseline(lin, kind, budget_s=args.cpu_budget, four_over_six=args.four_over_six,
+                                              norm=args.norm)
     return out
 
 
@@ -462,19 +502,22 @@ def run_loadtime(args, rank, world, local_rank):
 
 
 # --------------------------------------------------------------------------- oracle arm
-def oracle_step(lin, kind, rows, wq):
+def oracle_step(lin, kind, rows, wq, norm=None):
     """The oracle's linear layer on `rows` of A: quantize, decode, float64 GEMM, epilogue."""
     import oracle
     K = lin.K
     A = lin.A[rows]
     if kind == "nvfp4":
         gs_w, codes_b, sf_b, decB = wq
+        fmt = getattr(lin, "fmt", "bf16")
+        if norm == "rmsnorm":
+            A = oracle.rmsnorm_bf16(A, norm_gamma(lin), oracle.rmsnorm_rstd(A, NORM_EPS))
         if lin.per_token:
-            gs, inv = oracle.row_global_scales(A)
-            ca, sa = oracle.nvfp4_quantize(A, gs, per_row=True)
+            gs, inv = oracle.row_global_scales(A, fmt=fmt)
+            ca, sa = oracle.nvfp4_quantize(A, gs, per_row=True, fmt=fmt)
             alpha, rs = np.float32(1) / gs_w, inv
         else:
-            ca, sa = oracle.nvfp4_quantize(A, 1.0)
+            ca, sa = oracle.nvfp4_quantize(A, 1.0, fmt=fmt)
             alpha, rs = np.float32(1) / (np.float32(1) * gs_w), None
         decA = oracle.nvfp4_dequantize(ca, sa, K)
     else:
@@ -504,18 +547,18 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_baseline(lin, kind, budget_s=10.0, four_over_six=False):
+def oracle_baseline(lin, kind, budget_s=10.0, four_over_six=False, norm=None):
     """Times the oracle on a bounded row sample, scaled to TFLOP/s."""
     wq = oracle_weights(lin, kind, four_over_six)
     rng = np.random.default_rng(123)
     rows = np.sort(rng.choice(lin.M, size=min(lin.M, 128), replace=False))
     t0 = time.perf_counter()
-    oracle_step(lin, kind, rows, wq)
+    oracle_step(lin, kind, rows, wq, norm)
     dt = time.perf_counter() - t0
     n = int(min(lin.M, max(128, 128 * budget_s / max(dt, 1e-3))))
     rows = np.sort(rng.choice(lin.M, size=n, replace=False))
     t0 = time.perf_counter()
-    oracle_step(lin, kind, rows, wq)
+    oracle_step(lin, kind, rows, wq, norm)
     dt = time.perf_counter() - t0
     flops = 2.0 * n * lin.N * lin.K
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": max(os.cpu_count() or 1, blas_threads()),
@@ -561,14 +604,15 @@ def run_reference(args):
     if args.config == "loadtime":
         return run_reference_loadtime(args)
     lin, kind = make_workload(args.config)
+    lin = apply_input_format(lin, kind, args.input)
     wq = oracle_weights(lin, kind, args.four_over_six)
     rng = np.random.default_rng(7)
     n = min(lin.M, args.ref_rows)
     for _ in range(args.warmup):
-        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq)
+        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq, args.norm)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq)
+        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq, args.norm)
     dt = time.perf_counter() - t0
     flops = 2.0 * n * lin.N * lin.K * args.steps
     value = flops / dt / 1e12
@@ -577,6 +621,9 @@ def run_reference(args):
               f"rounding; weight quantized beforehand (load time)")
     cfg = describe(lin, kind)
     cfg["parallelism"] = "host cores"
+    cfg["activation_dtype"] = "fp16" if lin.fmt == "f16" else "bf16"
+    if args.norm == "rmsnorm":
+        cfg["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
     if kind == "nvfp4":
         cfg["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
@@ -595,6 +642,10 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="wan13")
+    ap.add_argument("--norm", choices=["none", "rmsnorm"], default="none",
+                    help="NVFP4 workloads: fuse an RMSNorm of the activation into the quantizer")
+    ap.add_argument("--input", choices=["bf16", "f16"], default="bf16",
+                    help="activation dtype of the NVFP4 workloads (f16: the bf16 values rounded to fp16)")
     ap.add_argument("--four-over-six", action="store_true",
                     help="NVFP4 weight global scale 256*6/amax (the 4over6 setting) instead of 448*6/amax")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -415,8 +415,8 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
 // RMSNorm fused into the NVFP4 quantizer (the producer of a pre-quantized
 // activation: hao-ai-lab-FastVideo nvfp4_config.py, NVFP4QuantizeMethod.apply
 // with `pre_quantized` from a fused norm+quant call).  Per row:
-//   ms   = mean(x^2)  (products exact; sum in fp64, any order; one rounding
-//          to fp32 at the end)
+//   ms   = mean(x^2)  (relative error <= 2^-24: pairs of exact squares added in
+//          fp32, the pair sums in fp64, one rounding to fp32 at the end)
 //   rstd = fl32(1 / sqrt(fl32(ms + eps)))     (correctly rounded)
 //   y_k  = bf16(fl32(fl32(x_k * rstd) * gamma_k))
 // and y is quantized exactly as nvfp4_quantize quantizes a bf16 input, so the
@@ -430,14 +430,17 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
   return v;
 }
 
+// Sum of squares of 8 bf16 values: the squares of a pair are added with one
+// fp32 rounding (fma of the exact second square onto the exact first), the
+// four pair sums in fp64.  Relative error <= 2^-24 (all terms are
+// non-negative), at half the fp32-to-fp64 conversions of a per-element fp64 sum.
 __device__ __forceinline__ double sumsq8(const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   double s = 0.0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 f = InBf16::values2(w[i]);
-    s = fma(static_cast<double>(f.x), static_cast<double>(f.x), s);
-    s = fma(static_cast<double>(f.y), static_cast<double>(f.y), s);
+    s += static_cast<double>(__fmaf_rn(f.y, f.y, __fmul_rn(f.x, f.x)));
   }
   return s;
 }

@@ -190,9 +190,10 @@ int nvfp4_quantize_f16(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
  * fused norm+quant call.  The pages name the fused call but not its norm; this
  * is RMSNorm with a weight, whose normalised output is quantized as if it had
  * been written as bf16 and passed to nvfp4_quantize.  Per row m:
- *   ms   = mean_k x_k^2  (exact products, summed in fp64 in any order, one
- *          rounding to fp32)
- *   rstd = fl32(1 / sqrt(fl32(ms + eps)))   (correctly rounded)
+ *   ms   = mean_k x_k^2  (relative error <= 2^-24: pairs of exact squares
+ *          added in fp32, pair sums in fp64 in any order, one rounding to fp32)
+ *   rstd = fl32(1 / sqrt(fl32(ms + eps)))   (correctly rounded from that ms, so
+ *          within 2 ulp of rstd from the exact mean)
  *   y_k  = bf16(fl32(fl32(x_k * rstd) * gamma_k))
  *   then y is quantized as nvfp4_quantize does (per-tensor global_sf, or per
  *   row gs[m] from the row amax of y), without y being stored.

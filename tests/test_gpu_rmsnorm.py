@@ -2,10 +2,13 @@
 producer of the pre-quantized activation of hao-ai-lab-FastVideo
 nvfp4_config.py, NVFP4QuantizeMethod.apply).
 
-The row reduction's order is free (fp64 sum of exact squares, one rounding), so
-rstd is checked within one fp32 ulp of the exactly rounded value; everything
-after it -- y in bf16, the group scales and codes, per-token scales -- is
-checked bit for bit by running the oracle from the rstd the kernel reports."""
+The kernel's mean of squares has relative error <= 2^-24 (pairs of exact
+squares added in fp32, pair sums in fp64 in any order, one rounding to fp32):
+with the correctly rounded rsqrt after it, rstd lies within 0.5 ulp + 2^-24
+relative of the true value, so within 2 fp32 ulp of the exactly rounded one,
+which is the tolerance here.  Everything after it -- y in bf16, the group
+scales and codes, per-token scales -- is checked bit for bit by running the
+oracle from the rstd the kernel reports."""
 import numpy as np
 import pytest
 import torch
@@ -44,7 +47,7 @@ def test_rmsnorm_quantize(M, K, per_row):
     assert api.device_status() == 0
     r_gpu = down(rstd)
     r_exact = oracle.rmsnorm_rstd(x, eps)
-    assert _ulps(r_gpu, r_exact).max() <= 1
+    assert _ulps(r_gpu, r_exact).max() <= 2
     codes, sf, _, g_rows, inv_rows = oracle.rmsnorm_quantize(x, g, eps, np.float32(0.75), per_row=per_row,
                                                                rstd=r_gpu)
     assert np.array_equal(down(q.codes), codes)
