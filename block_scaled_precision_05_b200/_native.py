@@ -20,6 +20,10 @@ BSP_SF_PER_TENSOR = 0
 BSP_SF_PER_ROW = 1
 BSP_OUT_BF16 = 0
 BSP_OUT_F32 = 1
+BSP_IN_BF16 = 0
+BSP_IN_F16 = 1
+BSP_SF_LAYOUT_128X4 = 0
+BSP_SF_LAYOUT_8X4 = 1
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 
@@ -29,6 +33,7 @@ SIGNATURES = {
     "bsp_version": (_i32, []),
     "bsp_nvfp4_sf_bytes": (_sz, [_i64, _i64]),
     "bsp_mxfp8_sf_bytes": (_sz, [_i64, _i64]),
+    "bsp_nvfp4_sf_bytes_layout": (_sz, [_i64, _i64, _i32]),
     "bsp_amax_bf16": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_amax_bf16_into": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_amax_f16": (_i32, [_vp, _i64, _vp, _vp]),
@@ -38,9 +43,11 @@ SIGNATURES = {
     "bsp_nvfp4_alpha": (_i32, [_vp, _vp, _vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_f16": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nvfp4_quantize_ex": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_rmsnorm_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, ctypes.c_float, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
                                       _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
+    "nvfp4_gemm_ex": (_i32, [_vp, _vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "mxfp8_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "mxfp8_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _i64, _vp]),
     "bsp_device_status": (_i32, [_vp]),

@@ -59,8 +59,8 @@ def coerce_bf16(x: torch.Tensor) -> torch.Tensor:
 _HALF_TYPES = (torch.bfloat16, torch.float16)
 
 
-def nvfp4_sf_bytes(rows: int, K: int) -> int:
-    return int(nat.lib().bsp_nvfp4_sf_bytes(rows, K))
+def nvfp4_sf_bytes(rows: int, K: int, sf_layout: str = "128x4") -> int:
+    return int(nat.lib().bsp_nvfp4_sf_bytes_layout(rows, K, SF_LAYOUTS[sf_layout]))
 
 
 def mxfp8_sf_bytes(rows: int, K: int) -> int:
@@ -132,14 +132,19 @@ def nvfp4_alpha(gs_x: torch.Tensor, gs_w: torch.Tensor) -> torch.Tensor:
 
 
 # --------------------------------------------------------------------------- quantize
+SF_LAYOUTS = {"128x4": nat.BSP_SF_LAYOUT_128X4, "8x4": nat.BSP_SF_LAYOUT_8X4}
+
+
 @dataclass
 class NVFP4Tensor:
-    """Packed NVFP4 rows: codes uint8 [M, K/2], scales uint8 (128x4 layout)."""
+    """Packed NVFP4 rows: codes uint8 [M, K/2], scales uint8 in the 128x4 (or,
+    for small M, 8x4) tile layout."""
     codes: torch.Tensor
     sf: torch.Tensor
     K: int
     row_gs: torch.Tensor | None = None      # per-row encode scales (PER_ROW)
     row_inv_gs: torch.Tensor | None = None  # per-row decode factors 1/gs (PER_ROW)
+    sf_layout: str = "128x4"
 
     @property
     def rows(self) -> int:
@@ -166,29 +171,35 @@ def _as_2d(x: torch.Tensor) -> torch.Tensor:
 
 
 def nvfp4_quantize(x: torch.Tensor, global_sf: torch.Tensor | None = None, per_row: bool = False,
-                   out: NVFP4Tensor | None = None) -> NVFP4Tensor:
-    """Quantize bf16 or fp16 [..., K] to NVFP4 along K (leading dims flattened)."""
+                   out: NVFP4Tensor | None = None, sf_layout: str = "128x4") -> NVFP4Tensor:
+    """Quantize bf16 or fp16 [..., K] to NVFP4 along K (leading dims flattened).
+    sf_layout "8x4" stores the scales in 8-row tiles (small M; nvfp4_gemm then
+    takes them for M <= 64)."""
     _require_cuda(x, global_sf)
     if x.dtype not in _HALF_TYPES:
         raise TypeError("nvfp4_quantize expects bf16 or fp16 input (use coerce_input first)")
     x2 = _as_2d(x)
     M, K = x2.shape
     dev = x2.device
+    if sf_layout not in SF_LAYOUTS:
+        raise ValueError(f"sf_layout must be one of {sorted(SF_LAYOUTS)}")
     if out is None:
         out = NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
-                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+                          torch.empty(nvfp4_sf_bytes(M, K, sf_layout), dtype=torch.uint8, device=dev), K,
+                          sf_layout=sf_layout)
         if per_row:
             out.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
             out.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
+    elif out.sf_layout != sf_layout:
+        raise ValueError("out was allocated for another scale layout")
     if not per_row and global_sf is None:
         raise ValueError("per-tensor quantization needs global_sf (fp32 device tensor)")
-    fn = nat.lib().nvfp4_quantize if x2.dtype == torch.bfloat16 else nat.lib().nvfp4_quantize_f16
-    st = fn(
-        _ptr(x2), M, K, x2.stride(0), None if per_row else _ptr(global_sf),
-        nat.BSP_SF_PER_ROW if per_row else nat.BSP_SF_PER_TENSOR,
-        _ptr(out.row_gs) if per_row else None, _ptr(out.row_inv_gs) if per_row else None,
+    st = nat.lib().nvfp4_quantize_ex(
+        _ptr(x2), nat.BSP_IN_BF16 if x2.dtype == torch.bfloat16 else nat.BSP_IN_F16, M, K, x2.stride(0),
+        None if per_row else _ptr(global_sf), nat.BSP_SF_PER_ROW if per_row else nat.BSP_SF_PER_TENSOR,
+        SF_LAYOUTS[sf_layout], _ptr(out.row_gs) if per_row else None, _ptr(out.row_inv_gs) if per_row else None,
         _ptr(out.codes), _ptr(out.sf), _stream())
-    nat.check(st, "nvfp4_quantize" if x2.dtype == torch.bfloat16 else "nvfp4_quantize_f16")
+    nat.check(st, "nvfp4_quantize_ex")
     return out
 
 
@@ -269,10 +280,12 @@ def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, alpha: torch.Tensor | None = None
     M, N = a.rows, b.rows
     _check_epilogue_args(alpha, row_scale, bias, N)
     out, d_dtype = _out(M, N, out_dtype, a.codes.device, out)
-    st = nat.lib().nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, a.K,
-                              _ptr(alpha), _ptr(row_scale), _ptr(bias), _ptr(out), d_dtype, out.stride(0),
-                              _stream())
-    nat.check(st, "nvfp4_gemm")
+    if b.sf_layout != "128x4":
+        raise ValueError("the weight's scales must be in the 128x4 layout")
+    st = nat.lib().nvfp4_gemm_ex(_ptr(a.codes), _ptr(a.sf), SF_LAYOUTS[a.sf_layout], _ptr(b.codes), _ptr(b.sf), M, N,
+                                 a.K, _ptr(alpha), _ptr(row_scale), _ptr(bias), _ptr(out), d_dtype, out.stride(0),
+                                 _stream())
+    nat.check(st, "nvfp4_gemm_ex")
     return out
 
 
@@ -331,9 +344,9 @@ class NVFP4Linear:
         self.alpha = self.inv_gs_w if per_token else nvfp4_alpha(self.gs_x, self.gs_w)
         self.bias = None if bias is None else coerce_bf16(bias).contiguous()
 
-    def quantize_input(self, x: torch.Tensor) -> NVFP4Tensor:
+    def quantize_input(self, x: torch.Tensor, sf_layout: str = "128x4") -> NVFP4Tensor:
         x = coerce_input(x)
-        return nvfp4_quantize(x, None if self.per_token else self.gs_x, per_row=self.per_token)
+        return nvfp4_quantize(x, None if self.per_token else self.gs_x, per_row=self.per_token, sf_layout=sf_layout)
 
     def rmsnorm_quantize_input(self, x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6) -> NVFP4Tensor:
         """RMSNorm(x) * gamma quantized for this layer in one kernel: pass the
@@ -342,9 +355,11 @@ class NVFP4Linear:
                                       None if self.per_token else self.gs_x, per_row=self.per_token)
 
     def __call__(self, x: torch.Tensor, pre_quantized: NVFP4Tensor | None = None,
-                 out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+                 out_dtype: torch.dtype = torch.bfloat16, sf_layout: str = "128x4") -> torch.Tensor:
+        """sf_layout "8x4": the activation's scales in 8-row tiles (mm_fp4's
+        use_8x4_sf_layout), for at most 64 rows."""
         lead = x.shape[:-1]
-        xq = pre_quantized if pre_quantized is not None else self.quantize_input(x)
+        xq = pre_quantized if pre_quantized is not None else self.quantize_input(x, sf_layout)
         y = nvfp4_gemm(xq, self.weight, self.alpha, xq.row_inv_gs if self.per_token else None, self.bias,
                        out_dtype=out_dtype)
         return y.view(*lead, self.out_features)

@@ -83,6 +83,12 @@ size_t bsp_nvfp4_sf_bytes(int64_t rows, int64_t K) {
   return static_cast<size_t>(bsp::round_up(rows, 128) * bsp::round_up(K / 16, 4));
 }
 
+size_t bsp_nvfp4_sf_bytes_layout(int64_t rows, int64_t K, int sf_layout) {
+  if (sf_layout == BSP_SF_LAYOUT_128X4) return bsp_nvfp4_sf_bytes(rows, K);
+  if (sf_layout != BSP_SF_LAYOUT_8X4 || rows < 0 || K < 0 || K % 16 != 0) return 0;
+  return static_cast<size_t>(bsp::round_up(rows, 8) * bsp::round_up(K / 16, 4));
+}
+
 size_t bsp_mxfp8_sf_bytes(int64_t rows, int64_t K) {
   if (rows < 0 || K < 0 || K % 32 != 0) return 0;
   return static_cast<size_t>(bsp::round_up(rows, 128) * bsp::round_up(K / 32, 4));

@@ -528,7 +528,10 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
 // TMEM column per activation row m; each warp writes 32 consecutive n of a
 // row of D per instruction).
 // ---------------------------------------------------------------------------
-template <int KIND, int BNA>
+// kSf8: the activation scales are in the 8x4 layout (32-byte tiles of 8 rows x
+// 4 K-groups, row-major); a stage's box is the BNA/8 row tiles x 4 K-group
+// tiles (fp4) of 32 bytes.
+template <int KIND, int BNA, bool kSf8 = false>
 struct SkCfg {
   static constexpr int BM = 128;                         // weight rows per tile (MMA M)
   static constexpr int ROW_BYTES = 128;
@@ -537,7 +540,8 @@ struct SkCfg {
   static constexpr int W_BYTES = BM * ROW_BYTES;
   static constexpr int X_BYTES = BNA * ROW_BYTES;
   static constexpr int SFW_BYTES = ATOMS * 512;
-  static constexpr int SFX_BYTES = ATOMS * 512;         // one 128-row band of activation scales
+  static constexpr int SFX_BYTES = kSf8 ? (BNA / 8) * ATOMS * 32  // BNA/8 row tiles x ATOMS tiles of 32 bytes
+                                        : ATOMS * 512;            // one 128-row band of activation scales
   static constexpr int TX_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
   static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
   static constexpr int SFW_COLS = ATOMS * 4;
@@ -554,12 +558,12 @@ struct SkCfg {
   static_assert(STAGES >= 2 && ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "budget");
 };
 
-template <int KIND, int BNA>
-__global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
+template <int KIND, int BNA, bool kSf8>
+__global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmSFW, const __grid_constant__ CUtensorMap tmSFX,
                        const GemmParams p) {
-  using C = SkCfg<KIND, BNA>;
+  using C = SkCfg<KIND, BNA, kSf8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -621,8 +625,12 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
           tma_load_2d(st, &tmW, &full[stage], kb * C::ROW_BYTES, nb * C::BM);
           tma_load_2d(st + C::W_BYTES, &tmX, &full[stage], kb * C::ROW_BYTES, mb * BNA);
           tma_load_3d(st + C::W_BYTES + C::X_BYTES, &tmSFW, &full[stage], 0, kb * C::ATOMS, nb);
-          tma_load_3d(st + C::W_BYTES + C::X_BYTES + C::SFW_BYTES, &tmSFX, &full[stage], 0, kb * C::ATOMS,
-                      (mb * BNA) >> 7);
+          if constexpr (kSf8)
+            tma_load_2d(st + C::W_BYTES + C::X_BYTES + C::SFW_BYTES, &tmSFX, &full[stage], kb * C::ATOMS * 32,
+                        mb * (BNA / 8));
+          else
+            tma_load_3d(st + C::W_BYTES + C::X_BYTES + C::SFW_BYTES, &tmSFX, &full[stage], 0, kb * C::ATOMS,
+                        (mb * BNA) >> 7);
           ++issued[stage];
           if (++stage == C::STAGES) {
             stage = 0;
@@ -702,7 +710,20 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
 #pragma unroll
         for (int a = 0; a < C::ATOMS; ++a) {
           const uint4 w = *reinterpret_cast<const uint4*>(sfw_s + 512 * a + lane * 16);
-          const uint4 x = *reinterpret_cast<const uint4*>(sfx_s + 512 * a + lane * 16);
+          uint4 x;
+          if constexpr (kSf8) {
+            // the 4 scales of activation row m for K-group tile a; rows past BNA are not in the box
+            uint32_t q[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int m = static_cast<int>(lane) + 32 * j;
+              if (m < BNA) q[j] = *reinterpret_cast<const uint32_t*>(sfx_s + (m >> 3) * (C::ATOMS * 32) + a * 32 +
+                                                                      (m & 7) * 4);
+            }
+            x = make_uint4(q[0], q[1], q[2], q[3]);
+          } else {
+            x = *reinterpret_cast<const uint4*>(sfx_s + 512 * a + lane * 16);
+          }
           v[4 * a + 0] = w.x;
           v[4 * a + 1] = w.y;
           v[4 * a + 2] = w.z;
@@ -798,12 +819,13 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA>::THREADS, 1)
 int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows,
                    int box_bytes = 128);
 int encode_scales(CUtensorMap* m, const void* base, int64_t bands, int64_t tiles_per_band, int atoms, int box_bands);
+int encode_rows_plain(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows, int box_bytes);
 
-template <int KIND, int BNA>
+template <int KIND, int BNA, bool kSf8 = false>
 int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                   int64_t row_bytes, int64_t tiles_per_band, GemmParams p, cudaStream_t stream) {
-  using C = SkCfg<KIND, BNA>;
-  auto kernel = skinny_gemm_kernel<KIND, BNA>;
+  using C = SkCfg<KIND, BNA, kSf8>;
+  auto kernel = skinny_gemm_kernel<KIND, BNA, kSf8>;
   static bool attr_set[64] = {};
   if (!attr_set[dev.id]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
@@ -815,7 +837,14 @@ int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, c
   if ((st = encode_operand(&tmW, B, p.N, row_bytes, C::BM)) != BSP_OK) return st;
   if ((st = encode_operand(&tmX, A, p.M, row_bytes, BNA)) != BSP_OK) return st;
   if ((st = encode_scales(&tmSFW, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
-  if ((st = encode_scales(&tmSFX, sfA, ceil_div(p.M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
+  if constexpr (kSf8) {
+    // [row tiles][tiles_per_band x 32 bytes], boxes of BNA/8 row tiles x ATOMS tiles
+    if ((st = encode_rows_plain(&tmSFX, sfA, ceil_div(p.M, 8), tiles_per_band * 32, BNA / 8, C::ATOMS * 32)) !=
+        BSP_OK)
+      return st;
+  } else {
+    if ((st = encode_scales(&tmSFX, sfA, ceil_div(p.M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
+  }
   p.num_n = static_cast<int>(ceil_div(p.N, C::BM));
   p.num_m = static_cast<int>(ceil_div(p.M, BNA));
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
@@ -844,6 +873,18 @@ int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_b
   CUresult r = encode_tiled_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
                                  CU_TENSOR_MAP_INTERLEAVE_NONE,
                                  box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
+}
+
+// Row-major bytes [rows, row_bytes], boxes of box_rows x box_bytes, no swizzle.
+int encode_rows_plain(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows, int box_bytes) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = encode_tiled_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
@@ -935,10 +976,13 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
 template <int KIND>
 int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, int64_t M, int64_t N,
              int64_t K, const float* alpha, const float* row_scale, const uint16_t* bias, void* D, int d_dtype,
-             int64_t ld_d, cudaStream_t stream) {
+             int64_t ld_d, cudaStream_t stream, int a_sf_layout = BSP_SF_LAYOUT_128X4) {
   const int64_t group = KIND == kNVF4 ? 16 : 32;
   if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return BSP_ERR_INVALID_ARG;
   if (d_dtype != BSP_OUT_BF16 && d_dtype != BSP_OUT_F32) return BSP_ERR_INVALID_ARG;
+  const bool sf8 = a_sf_layout == BSP_SF_LAYOUT_8X4;
+  if (!sf8 && a_sf_layout != BSP_SF_LAYOUT_128X4) return BSP_ERR_INVALID_ARG;
+  if (sf8 && (KIND != kNVF4 || M > BSP_GEMM_SKINNY_MAX_M)) return BSP_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return BSP_OK;
   if (N % 8 != 0 || ld_d < N) return BSP_ERR_INVALID_ARG;
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return BSP_ERR_INVALID_ARG;
@@ -971,6 +1015,13 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   p.ld_d = ld_d;
   p.out_f32 = d_dtype == BSP_OUT_F32;
   p.err = dev.err_word;
+  if constexpr (KIND == kNVF4) {
+    if (sf8) {  // 8x4 activation scales: M <= 64, the transposed kernel
+      if (M <= 16) return launch_skinny<KIND, 16, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+      if (M <= 32) return launch_skinny<KIND, 32, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+      return launch_skinny<KIND, 64, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    }
+  }
   if (skinny) {
     if (M <= 16) return launch_skinny<KIND, 16>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
     if (M <= 32) return launch_skinny<KIND, 32>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
@@ -989,6 +1040,13 @@ int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uin
                int64_t K, const float* alpha, const float* row_scale, const uint16_t* bias, void* D, int d_dtype,
                int64_t ld_d, bsp_stream_t stream) {
   return bsp::run_gemm<bsp::kNVF4>(A, sfA, B, sfB, M, N, K, alpha, row_scale, bias, D, d_dtype, ld_d, stream);
+}
+
+int nvfp4_gemm_ex(const uint8_t* A, const uint8_t* sfA, int a_sf_layout, const uint8_t* B, const uint8_t* sfB,
+                  int64_t M, int64_t N, int64_t K, const float* alpha, const float* row_scale, const uint16_t* bias,
+                  void* D, int d_dtype, int64_t ld_d, bsp_stream_t stream) {
+  return bsp::run_gemm<bsp::kNVF4>(A, sfA, B, sfB, M, N, K, alpha, row_scale, bias, D, d_dtype, ld_d, stream,
+                                   a_sf_layout);
 }
 
 int mxfp8_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, int64_t M, int64_t N,

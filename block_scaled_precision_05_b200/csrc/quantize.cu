@@ -154,10 +154,26 @@ __device__ __forceinline__ uint32_t nvfp4_codes8(const uint4& v, float inv) {
   return cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y);
 }
 
-// Byte offset of the first of the four scale bytes (r, 4*tile_col .. +3).
-__device__ __forceinline__ int64_t sf_row_base(int64_t r, int64_t tiles_per_band) {
-  return (r >> 7) * tiles_per_band * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
-}
+// Scale-factor tile layouts.  row_base(r, tiles) is the byte offset of the
+// first of the four scale bytes (r, 4*tile_col .. +3) of tile column 0; tile
+// column j is kTileBytes further.
+//   128x4 (layout_128x4): 512-byte tiles of 128 rows x 4 columns, 32 lines of
+//     16 bytes, line l holding rows l, l+32, l+64, l+96; what the tensor core
+//     consumes.
+//   8x4 (layout_8x4, the small-M layout of mm_fp4's use_8x4_sf_layout):
+//     32-byte tiles of 8 rows x 4 columns, row-major.
+struct Sf128x4 {
+  static constexpr int kRowTile = 128, kTileBytes = 512;
+  static __device__ __forceinline__ int64_t row_base(int64_t r, int64_t tiles) {
+    return (r >> 7) * tiles * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+  }
+};
+struct Sf8x4 {
+  static constexpr int kRowTile = 8, kTileBytes = 32;
+  static __device__ __forceinline__ int64_t row_base(int64_t r, int64_t tiles) {
+    return (r >> 3) * tiles * 32 + (r & 7) * 4;
+  }
+};
 
 // Per-row encode scale of row r (warp-cooperative); lane 0 stores gs and 1/gs.
 template <class In>
@@ -189,7 +205,7 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
 // lane, then the quantization of each.  `lp`, `cp`, `sp` point at this lane's
 // group, its 8 code bytes, and (for lanes with g % 4 == 0) its 4 scale bytes in
 // the first step.
-template <class In, int U>
+template <class In, class L, int U>
 __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uint8_t* sp, bool live, float gs,
                                             bool store_sf) {
   uint4 v[U][2];
@@ -210,14 +226,14 @@ __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uin
     const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
     const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
     if (live) *reinterpret_cast<uint2*>(cp + u * 256) = w;
-    if (store_sf) *reinterpret_cast<uint32_t*>(sp + u * 4096) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    if (store_sf) *reinterpret_cast<uint32_t*>(sp + u * 8 * L::kTileBytes) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
   }
 }
 
 // Per-tensor scale, short rows (K = 512 * S, S <= 3): a warp quantizes two rows
 // per iteration with all 4S 16-byte loads of both rows issued up front, so the
 // memory pipeline stays full although each row is only S warp steps long.
-template <class In, int S>
+template <class In, class L, int S>
 __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const float* __restrict__ gs_ptr,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -247,7 +263,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
       if (r >= Mp) break;
       const bool live = r < M;
       uint8_t* cp = codes + r * (K >> 1) + lane * 8;
-      uint8_t* sp = sf + sf_row_base(r, K >> 6) + (lane >> 2) * 512;
+      uint8_t* sp = sf + L::row_base(r, K >> 6) + (lane >> 2) * L::kTileBytes;
 #pragma unroll
       for (int st = 0; st < S; ++st) {
         uint32_t sfb;
@@ -260,7 +276,8 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
         const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
         const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
         if (live) *reinterpret_cast<uint2*>(cp + st * 256) = w;
-        if (quad_lead) *reinterpret_cast<uint32_t*>(sp + st * 4096) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        if (quad_lead)
+          *reinterpret_cast<uint32_t*>(sp + st * 8 * L::kTileBytes) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
     }
   }
@@ -273,7 +290,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
 // registers, so each row costs one memory round trip.
 constexpr int kRowG = 4;
 
-template <class In>
+template <class In, class L>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, float* __restrict__ row_gs,
     float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -315,7 +332,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
     __syncthreads();
     const float gs = gs_sh;
     uint8_t* crow = codes + r * (K >> 1);
-    const int64_t sbase = sf_row_base(r, tiles_per_band);
+    const int64_t sbase = L::row_base(r, tiles_per_band);
 #pragma unroll
     for (int i = 0; i < kRowG; ++i) {
       const int g = t + i * kQuantThreads;
@@ -333,14 +350,15 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
       if (g < groups) {
         if (live) *reinterpret_cast<uint2*>(crow + g * 8) = w;
         if ((g & 3) == 0)
-          *reinterpret_cast<uint32_t*>(sf + sbase + (g >> 2) * 512) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          *reinterpret_cast<uint32_t*>(sf + sbase + (g >> 2) * L::kTileBytes) =
+              sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
     }
     __syncthreads();  // red / gs_sh are reused by the next row
   }
 }
 
-template <class In, bool kPerRow>
+template <class In, class L, bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -362,15 +380,17 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     // group g = 32 * step + lane: elements 16 g, code bytes 8 g, scale tile g / 4
     const uint16_t* lp = row + lane * 16;
     uint8_t* cp = codes + r * (K >> 1) + lane * 8;
-    uint8_t* sp = sf + sf_row_base(r, groups >> 2) + (lane >> 2) * 512;
+    uint8_t* sp = sf + L::row_base(r, groups >> 2) + (lane >> 2) * L::kTileBytes;
+    constexpr int kStepSf = 8 * L::kTileBytes;  // a warp step covers 8 scale tiles
     int64_t st = 0;
     for (; st + kUnroll <= steps; st += kUnroll)
-      nvfp4_steps<In, kUnroll>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
-    for (; st < steps; ++st) nvfp4_steps<In, 1>(lp + st * 512, cp + st * 256, sp + st * 4096, live, gs, quad_lead);
+      nvfp4_steps<In, L, kUnroll>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
+    for (; st < steps; ++st)
+      nvfp4_steps<In, L, 1>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
     if (rem) {
       const bool in = lane < rem;  // groups beyond the row end are predicated off
-      nvfp4_steps<In, 1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * 4096 : sp, live && in, gs,
-                     in && quad_lead);
+      nvfp4_steps<In, L, 1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * kStepSf : sp,
+                            live && in, gs, in && quad_lead);
     }
   }
 }
@@ -378,7 +398,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
 // ---------------------------------------------------------------------------
 // NVFP4, any K % 16 == 0: one warp per row, one lane per group of 16.
 // ---------------------------------------------------------------------------
-template <class In, bool kPerRow>
+template <class In, class L, bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
@@ -394,7 +414,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
     if (kPerRow && live) gs = row_scale_pass<In>(row, K, r, row_gs, row_inv);
-    const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
+    const int64_t sfb_row = L::row_base(r, cols4 >> 2);
     for (int64_t c = lane; c < cols4; c += 32) {
       uint32_t sfb = 0;
       if (live && c < groups) {
@@ -406,7 +426,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
         w.y = nvfp4_codes8<In>(b, inv);
         *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
       }
-      sf[sfb_row + (c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfb);
+      sf[sfb_row + (c >> 2) * L::kTileBytes + (c & 3)] = static_cast<uint8_t>(sfb);
     }
   }
 }
@@ -460,7 +480,7 @@ __device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, floa
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <bool kPerRow>
+template <class L, bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const uint16_t* __restrict__ gamma,
     float eps, const float* __restrict__ gs_ptr, float* __restrict__ row_gs, float* __restrict__ row_inv,
@@ -473,9 +493,9 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
-    const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
+    const int64_t sfb_row = L::row_base(r, cols4 >> 2);
     if (r >= M) {  // scale padding rows
-      for (int64_t c = lane; c < cols4; c += 32) sf[sfb_row + (c >> 2) * 512 + (c & 3)] = 0;
+      for (int64_t c = lane; c < cols4; c += 32) sf[sfb_row + (c >> 2) * L::kTileBytes + (c & 3)] = 0;
       continue;
     }
     const uint16_t* row = x + r * ld_x;
@@ -513,7 +533,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
         w.y = nvfp4_codes8<InBf16>(y1, inv);
         *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
       }
-      sf[sfb_row + (c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfb);
+      sf[sfb_row + (c >> 2) * L::kTileBytes + (c & 3)] = static_cast<uint8_t>(sfb);
     }
   }
 }
@@ -594,7 +614,7 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_k128_kernel(const u
     const bool live = r < M;
     const uint16_t* lp = x + r * ld_x + lane * 32;
     uint8_t* qp = q + r * K + lane * 32;
-    uint8_t* sp = sf + sf_row_base(r, groups >> 2) + (lane >> 2) * 512;
+    uint8_t* sp = sf + Sf128x4::row_base(r, groups >> 2) + (lane >> 2) * 512;
     int64_t st = 0;
     for (; st + kU <= steps; st += kU) mxfp8_steps<kU>(lp + st * 1024, qp + st * 1024, sp + st * 4096, live, quad_lead);
     for (; st < steps; ++st) mxfp8_steps<1>(lp + st * 1024, qp + st * 1024, sp + st * 4096, live, quad_lead);
@@ -619,7 +639,7 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_quant_generic_kernel(cons
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const bool live = r < M;
     const uint16_t* row = x + r * ld_x;
-    const int64_t sfb_row = sf_row_base(r, cols4 >> 2);
+    const int64_t sfb_row = Sf128x4::row_base(r, cols4 >> 2);
     for (int64_t c = lane; c < cols4; c += 32) {
       uint32_t sfb = 0;
       if (live && c < groups) {
@@ -731,7 +751,7 @@ int amax_launch(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream, 
   return launch_status();
 }
 
-template <class In>
+template <class In, class L>
 int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
                        float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
   if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K) return BSP_ERR_INVALID_ARG;
@@ -742,13 +762,13 @@ int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, co
   DeviceInfo dev;
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
-  const int64_t Mp = round_up(M, 128);
+  const int64_t Mp = round_up(M, L::kRowTile);
   const bool per_row = sf_mode == BSP_SF_PER_ROW;
   if (K % 64 == 0) {
     int rowblock_cap = 0;  // rows the block-per-row kernel keeps resident at once
     if (per_row && K <= 16 * kQuantThreads * kRowG) {
       int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_quant_rowblock_kernel<In>, kQuantThreads,
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_quant_rowblock_kernel<In, L>, kQuantThreads,
                                                         0) != cudaSuccess ||
           per_sm < 1) {
         cudaGetLastError();
@@ -758,33 +778,33 @@ int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, co
     }
     if (per_row && Mp <= rowblock_cap) {
       // few rows: one block per row, all rows in one wave, one memory round trip
-      nvfp4_quant_rowblock_kernel<In><<<static_cast<int>(Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, row_gs,
+      nvfp4_quant_rowblock_kernel<In, L><<<static_cast<int>(Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, row_gs,
                                                                                       row_inv_gs, codes, sf);
     } else if (per_row) {
-      auto k = nvfp4_quant_k64_kernel<In, true>;
+      auto k = nvfp4_quant_k64_kernel<In, L, true>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
                                                                  codes, sf);
     } else if (K == 1024 || K == 1536) {
       const int64_t pairs = ceil_div(Mp, 2);
       if (K == 1024) {
-        auto k = nvfp4_quant_short_kernel<In, 2>;
+        auto k = nvfp4_quant_short_kernel<In, L, 2>;
         k<<<grid_for_rows(dev, k, pairs), kQuantThreads, 0, stream>>>(x, M, Mp, ld_x, global_sf, codes, sf);
       } else {
-        auto k = nvfp4_quant_short_kernel<In, 3>;
+        auto k = nvfp4_quant_short_kernel<In, L, 3>;
         k<<<grid_for_rows(dev, k, pairs), kQuantThreads, 0, stream>>>(x, M, Mp, ld_x, global_sf, codes, sf);
       }
     } else {
-      auto k = nvfp4_quant_k64_kernel<In, false>;
+      auto k = nvfp4_quant_k64_kernel<In, L, false>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
                                                                  codes, sf);
     }
   } else {
     if (per_row) {
-      auto k = nvfp4_quant_generic_kernel<In, true>;
+      auto k = nvfp4_quant_generic_kernel<In, L, true>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, row_gs, row_inv_gs,
                                                                  codes, sf);
     } else {
-      auto k = nvfp4_quant_generic_kernel<In, false>;
+      auto k = nvfp4_quant_generic_kernel<In, L, false>;
       k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, global_sf, nullptr, nullptr,
                                                                  codes, sf);
     }
@@ -801,12 +821,29 @@ extern "C" {
 
 int nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
                    float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
-  return run_nvfp4_quantize<InBf16>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
+  return run_nvfp4_quantize<InBf16, Sf128x4>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
 }
 
 int nvfp4_quantize_f16(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
                        float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
-  return run_nvfp4_quantize<InF16>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
+  return run_nvfp4_quantize<InF16, Sf128x4>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf, stream);
+}
+
+int nvfp4_quantize_ex(const uint16_t* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x, const float* global_sf,
+                      int sf_mode, int sf_layout, float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf,
+                      bsp_stream_t stream) {
+  if (x_dtype != BSP_IN_BF16 && x_dtype != BSP_IN_F16) return BSP_ERR_INVALID_ARG;
+  if (sf_layout != BSP_SF_LAYOUT_128X4 && sf_layout != BSP_SF_LAYOUT_8X4) return BSP_ERR_INVALID_ARG;
+  const bool f16 = x_dtype == BSP_IN_F16;
+  if (sf_layout == BSP_SF_LAYOUT_8X4)
+    return f16 ? run_nvfp4_quantize<InF16, Sf8x4>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf,
+                                                  stream)
+               : run_nvfp4_quantize<InBf16, Sf8x4>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf,
+                                                   stream);
+  return f16 ? run_nvfp4_quantize<InF16, Sf128x4>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf,
+                                                  stream)
+             : run_nvfp4_quantize<InBf16, Sf128x4>(x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf,
+                                                   stream);
 }
 
 int nvfp4_rmsnorm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const uint16_t* gamma, float eps,
@@ -824,11 +861,11 @@ int nvfp4_rmsnorm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x
   if (st != BSP_OK) return st;
   const int64_t Mp = round_up(M, 128);
   if (sf_mode == BSP_SF_PER_ROW) {
-    auto k = nvfp4_rmsnorm_quant_kernel<true>;
+    auto k = nvfp4_rmsnorm_quant_kernel<Sf128x4, true>;
     k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, row_gs,
                                                                row_inv_gs, row_rstd, codes, sf);
   } else {
-    auto k = nvfp4_rmsnorm_quant_kernel<false>;
+    auto k = nvfp4_rmsnorm_quant_kernel<Sf128x4, false>;
     k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, nullptr,
                                                                nullptr, row_rstd, codes, sf);
   }

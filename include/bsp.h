@@ -69,6 +69,19 @@ enum {
     BSP_OUT_F32 = 1
 };
 
+/* Input element types of nvfp4_quantize_ex. */
+enum {
+    BSP_IN_BF16 = 0,
+    BSP_IN_F16 = 1
+};
+
+/* Scale-factor tile layouts (FastVideo nvfp4_config.py: SfLayout.layout_128x4
+ * and layout_8x4, the latter with rows padded to 8, `row_tile = 8`). */
+enum {
+    BSP_SF_LAYOUT_128X4 = 0,
+    BSP_SF_LAYOUT_8X4 = 1
+};
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *bsp_status_string(int status);
 
@@ -87,6 +100,14 @@ int bsp_version(void);
 
 /* NVFP4: cols = K/16 (one e4m3 scale per 16 elements).  0 if K % 16 != 0. */
 size_t bsp_nvfp4_sf_bytes(int64_t rows, int64_t K);
+/* The same for a scale layout: BSP_SF_LAYOUT_128X4 as above; BSP_SF_LAYOUT_8X4
+ * stores 32-byte tiles of 8 rows x 4 columns, row-major inside a tile, tiles
+ * ordered by row tile then column tile:
+ *   ((r/8) * (cols4/4) + c/4) * 32 + (r%8)*4 + c%4
+ * in round_up(rows,8) * round_up(cols,4) bytes.  (The pages name layout_8x4
+ * and its 8-row padding but not its byte order; this row-major tile is the
+ * reading taken.)  0 for an unknown layout or K % 16 != 0. */
+size_t bsp_nvfp4_sf_bytes_layout(int64_t rows, int64_t K, int sf_layout);
 /* MXFP8: cols = K/32 (one e8m0 scale per 32 elements).  0 if K % 32 != 0. */
 size_t bsp_mxfp8_sf_bytes(int64_t rows, int64_t K);
 
@@ -185,6 +206,19 @@ int nvfp4_quantize_f16(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
                        const float *global_sf, int sf_mode, float *row_gs, float *row_inv_gs,
                        uint8_t *codes, uint8_t *sf, bsp_stream_t stream);
 
+/* nvfp4_quantize with the input type and the scale layout as arguments:
+ *   x_dtype  : BSP_IN_BF16 (as nvfp4_quantize) or BSP_IN_F16 (as
+ *              nvfp4_quantize_f16)
+ *   sf_layout: BSP_SF_LAYOUT_128X4 (as nvfp4_quantize) or BSP_SF_LAYOUT_8X4
+ *              (sf holds bsp_nvfp4_sf_bytes_layout(M, K, BSP_SF_LAYOUT_8X4)
+ *              bytes; padding rows up to a multiple of 8 are 0).  An 8x4
+ *              activation is consumed by nvfp4_gemm_ex for M <= 64.
+ * Other arguments and errors as nvfp4_quantize; an unknown x_dtype or
+ * sf_layout -> INVALID_ARG. */
+int nvfp4_quantize_ex(const uint16_t *x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
+                      const float *global_sf, int sf_mode, int sf_layout, float *row_gs,
+                      float *row_inv_gs, uint8_t *codes, uint8_t *sf, bsp_stream_t stream);
+
 /* RMSNorm fused into the NVFP4 quantizer: the producer of the pre-quantized
  * activation that NVFP4QuantizeMethod.apply (nvfp4_config.py) accepts from a
  * fused norm+quant call.  The pages name the fused call but not its norm; this
@@ -232,6 +266,19 @@ int nvfp4_rmsnorm_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x
 int nvfp4_gemm(const uint8_t *A, const uint8_t *sfA, const uint8_t *B, const uint8_t *sfB,
                int64_t M, int64_t N, int64_t K, const float *alpha, const float *row_scale,
                const uint16_t *bias, void *D, int d_dtype, int64_t ld_d, bsp_stream_t stream);
+
+/* nvfp4_gemm with the activation scales in a given layout (mm_fp4's
+ * use_8x4_sf_layout, nvfp4_config.py _mm_fp4):
+ *   a_sf_layout: BSP_SF_LAYOUT_128X4 (as nvfp4_gemm) or BSP_SF_LAYOUT_8X4, for
+ *                M <= 64: sfA holds bsp_nvfp4_sf_bytes_layout(M, K,
+ *                BSP_SF_LAYOUT_8X4) bytes (nvfp4_quantize_ex with that
+ *                layout).  The weight scales sfB are always 128x4.
+ * Other arguments and errors as nvfp4_gemm; an unknown layout, or 8X4 with
+ * M > 64 -> INVALID_ARG. */
+int nvfp4_gemm_ex(const uint8_t *A, const uint8_t *sfA, int a_sf_layout, const uint8_t *B,
+                  const uint8_t *sfB, int64_t M, int64_t N, int64_t K, const float *alpha,
+                  const float *row_scale, const uint16_t *bias, void *D, int d_dtype, int64_t ld_d,
+                  bsp_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * MXFP8 quantization (mxfp8_config.py, DiffusionMXFP8Config: groups of 32

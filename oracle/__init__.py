@@ -74,6 +74,14 @@ def lib() -> ctypes.CDLL:
         L.bspo_sf_offset.argtypes = [i64, i64, i64]
         L.bspo_sf_bytes.restype = i64
         L.bspo_sf_bytes.argtypes = [i64, i64]
+        L.bspo_sf_offset_8x4.restype = i64
+        L.bspo_sf_offset_8x4.argtypes = [i64, i64, i64]
+        L.bspo_sf_bytes_8x4.restype = i64
+        L.bspo_sf_bytes_8x4.argtypes = [i64, i64]
+        L.bspo_nvfp4_quantize_layout.restype = i32
+        L.bspo_nvfp4_quantize_layout.argtypes = [vp, i64, i64, i64, i32, i32, vp, i32, vp, vp]
+        L.bspo_nvfp4_dequantize_rows_layout.restype = None
+        L.bspo_nvfp4_dequantize_rows_layout.argtypes = [vp, vp, i64, i32, vp, i64, vp]
         L.bspo_amax_bf16.restype = f32
         L.bspo_amax_bf16.argtypes = [vp, i64]
         L.bspo_nvfp4_global_scale.restype = f32
@@ -167,12 +175,19 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
-def sf_offset(r: int, c: int, cols_padded: int) -> int:
+LAYOUTS = {"128x4": 0, "8x4": 1}
+
+
+def sf_offset(r: int, c: int, cols_padded: int, layout: str = "128x4") -> int:
+    if layout == "8x4":
+        return lib().bspo_sf_offset_8x4(int(r), int(c), int(cols_padded))
     return lib().bspo_sf_offset(int(r), int(c), int(cols_padded))
 
 
-def sf_bytes(rows: int, cols: int) -> int:
+def sf_bytes(rows: int, cols: int, layout: str = "128x4") -> int:
     """Bytes of a tile-mapped scale buffer for [rows, cols] scales."""
+    if layout == "8x4":
+        return lib().bspo_sf_bytes_8x4(int(rows), int(cols))
     return lib().bspo_sf_bytes(int(rows), int(cols))
 
 
@@ -221,7 +236,8 @@ def _row_chunks(M: int, threads: int):
     return [(m0, min(M, m0 + per)) for m0 in range(0, M, per)]
 
 
-def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None = None, fmt: str = "bf16"):
+def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None = None, fmt: str = "bf16",
+                   layout: str = "128x4"):
     """NVFP4 quantization of bf16 (or, fmt="f16", fp16) bit patterns ``x`` [M, K] along K.
 
     Returns (codes uint8 [M, K/2], sf uint8 [sf_bytes(M, K/16)] in the 128x4 map).
@@ -237,7 +253,7 @@ def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None
     codes = np.empty((M, K // 2), np.uint8)
     cols = K // 16
     cols_p = -(-cols // 4) * 4
-    sf = np.empty(sf_bytes(M, cols), np.uint8)
+    sf = np.empty(sf_bytes(M, cols, layout), np.uint8)
     if M == 0:
         return codes, sf
     L = lib()
@@ -245,8 +261,9 @@ def nvfp4_quantize(x: np.ndarray, gs, per_row: bool = False, threads: int | None
     def run(rng):
         m0, m1 = rng
         gp = _ptr(g) + (4 * m0 if per_row else 0)
-        rc = L.bspo_nvfp4_quantize_fmt(_ptr(x) + 2 * m0 * K, m1 - m0, K, K, FORMATS[fmt], gp, int(per_row),
-                                       _ptr(codes) + m0 * (K // 2), _ptr(sf) + m0 * cols_p)
+        # chunks start at multiples of 128 rows: whole 128-row bands, or 16 8-row tiles
+        rc = L.bspo_nvfp4_quantize_layout(_ptr(x) + 2 * m0 * K, m1 - m0, K, K, FORMATS[fmt], LAYOUTS[layout], gp,
+                                          int(per_row), _ptr(codes) + m0 * (K // 2), _ptr(sf) + m0 * cols_p)
         assert rc == 0
 
     chunks = _row_chunks(M, _threads(threads))
@@ -304,8 +321,12 @@ def _dequant(fn, codes, sf, K, rows, threads):
     return out
 
 
-def nvfp4_dequantize(codes: np.ndarray, sf: np.ndarray, K: int, rows=None, threads=None) -> np.ndarray:
+def nvfp4_dequantize(codes: np.ndarray, sf: np.ndarray, K: int, rows=None, threads=None,
+                     layout: str = "128x4") -> np.ndarray:
     """Real values e2m1(code) * e4m3(scale) of the chosen rows, float64 [len(rows), K]."""
+    if layout == "8x4":
+        f = lib().bspo_nvfp4_dequantize_rows_layout
+        return _dequant(lambda c, s, k, r, n, o: f(c, s, k, 1, r, n, o), codes, sf, K, rows, threads)
     return _dequant(lib().bspo_nvfp4_dequantize_rows, codes, sf, K, rows, threads)
 
 

@@ -217,6 +217,31 @@ int64_t bspo_sf_bytes(int64_t rows, int64_t cols)
     return round_up(rows, 128) * round_up(cols, 4);
 }
 
+/* layout_8x4 ([FV] nvfp4_config.py: SfLayout.layout_8x4, rows padded to 8;
+ * the pages do not give the byte order inside a tile -- the reading here is a
+ * row-major 8x4 tile of 32 bytes, tiles ordered by row tile, then column
+ * tile, like the 128x4 tiles). */
+int64_t bspo_sf_offset_8x4(int64_t r, int64_t c, int64_t cols_padded)
+{
+    return ((r / 8) * (cols_padded / 4) + c / 4) * 32 + (r % 8) * 4 + c % 4;
+}
+
+int64_t bspo_sf_bytes_8x4(int64_t rows, int64_t cols)
+{
+    return round_up(rows, 8) * round_up(cols, 4);
+}
+
+/* Layouts: 0 = 128x4, 1 = 8x4. */
+static int64_t sf_offset_layout(int64_t r, int64_t c, int64_t cols_padded, int layout)
+{
+    return layout ? bspo_sf_offset_8x4(r, c, cols_padded) : bspo_sf_offset(r, c, cols_padded);
+}
+
+static int64_t sf_bytes_layout(int64_t rows, int64_t cols, int layout)
+{
+    return layout ? bspo_sf_bytes_8x4(rows, cols) : bspo_sf_bytes(rows, cols);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Global scales ([FV-QAT] convert_model_to_fp4; [SGL] weight_scale_2).      */
 /* ------------------------------------------------------------------------ */
@@ -311,13 +336,13 @@ void bspo_nvfp4_quantize_group(const float *x, float gs, uint8_t *sfb_out, uint8
  * element 2j in the low nibble of byte j and element 2j+1 in the high nibble.
  * sf: bspo_sf_bytes(M, K/16) bytes in the 128x4 tile map; padding rows and
  * columns are 0.  Returns 0, or -1 when K is not a multiple of 16. */
-int bspo_nvfp4_quantize_fmt(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int fmt,
-                            const float *gs, int per_row, uint8_t *codes, uint8_t *sf)
+int bspo_nvfp4_quantize_layout(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int fmt, int layout,
+                               const float *gs, int per_row, uint8_t *codes, uint8_t *sf)
 {
     if (K % 16 != 0 || M < 0)
         return -1;
     int64_t cols = K / 16, cols_p = round_up(cols, 4);
-    memset(sf, 0, (size_t)bspo_sf_bytes(M, cols));
+    memset(sf, 0, (size_t)sf_bytes_layout(M, cols, layout));
     float xs[16];
     uint8_t q[16];
     for (int64_t m = 0; m < M; ++m) {
@@ -327,12 +352,18 @@ int bspo_nvfp4_quantize_fmt(const uint16_t *x, int64_t M, int64_t K, int64_t ld_
                 xs[i] = (float)elem_value(x[m * ld_x + c * 16 + i], fmt); /* exact */
             uint8_t sfb;
             bspo_nvfp4_quantize_group(xs, g, &sfb, q);
-            sf[bspo_sf_offset(m, c, cols_p)] = sfb;
+            sf[sf_offset_layout(m, c, cols_p, layout)] = sfb;
             for (int j = 0; j < 8; ++j)
                 codes[m * (K / 2) + c * 8 + j] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
         }
     }
     return 0;
+}
+
+int bspo_nvfp4_quantize_fmt(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int fmt,
+                            const float *gs, int per_row, uint8_t *codes, uint8_t *sf)
+{
+    return bspo_nvfp4_quantize_layout(x, M, K, ld_x, fmt, 0, gs, per_row, codes, sf);
 }
 
 int bspo_nvfp4_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
@@ -397,8 +428,8 @@ int bspo_mxfp8_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
 
 /* Decode rows[i] of an NVFP4 operand ([rows_total, K/2] codes + tile-mapped
  * scales) to out[i*K + k] = e2m1(code) * e4m3(scale).  Exact in double. */
-void bspo_nvfp4_dequantize_rows(const uint8_t *codes, const uint8_t *sf, int64_t K,
-                                const int64_t *rows, int64_t nrows, double *out)
+void bspo_nvfp4_dequantize_rows_layout(const uint8_t *codes, const uint8_t *sf, int64_t K, int layout,
+                                       const int64_t *rows, int64_t nrows, double *out)
 {
     int64_t cols_p = round_up(K / 16, 4);
     for (int64_t i = 0; i < nrows; ++i) {
@@ -406,10 +437,16 @@ void bspo_nvfp4_dequantize_rows(const uint8_t *codes, const uint8_t *sf, int64_t
         for (int64_t k = 0; k < K; ++k) {
             uint8_t byte = codes[r * (K / 2) + k / 2];
             int code = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
-            double s = bspo_e4m3_value(sf[bspo_sf_offset(r, k / 16, cols_p)]);
+            double s = bspo_e4m3_value(sf[sf_offset_layout(r, k / 16, cols_p, layout)]);
             out[i * K + k] = bspo_e2m1_value(code) * s;
         }
     }
+}
+
+void bspo_nvfp4_dequantize_rows(const uint8_t *codes, const uint8_t *sf, int64_t K,
+                                const int64_t *rows, int64_t nrows, double *out)
+{
+    bspo_nvfp4_dequantize_rows_layout(codes, sf, K, 0, rows, nrows, out);
 }
 
 void bspo_mxfp8_dequantize_rows(const uint8_t *q, const uint8_t *sf, int64_t K,

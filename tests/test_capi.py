@@ -35,6 +35,14 @@ def test_status_strings():
     assert nat.lib().bsp_version() >= 100
 
 
+def test_sf_bytes_8x4():
+    L = nat.lib()
+    assert L.bsp_nvfp4_sf_bytes_layout(1, 64, nat.BSP_SF_LAYOUT_8X4) == 8 * 4
+    assert L.bsp_nvfp4_sf_bytes_layout(9, 80, nat.BSP_SF_LAYOUT_8X4) == 16 * 8
+    assert L.bsp_nvfp4_sf_bytes_layout(9, 80, nat.BSP_SF_LAYOUT_128X4) == L.bsp_nvfp4_sf_bytes(9, 80)
+    assert L.bsp_nvfp4_sf_bytes_layout(9, 80, 5) == 0
+
+
 @pytest.mark.parametrize("rows,K,nv,mx", [(1, 16, 512, 0), (128, 256, 128 * 16, 128 * 8), (129, 64, 256 * 4, 256 * 4),
                                           (32760, 5120, 32768 * 320, 32768 * 160), (0, 32, 0, 0), (5, 24, 0, 0)])
 def test_sf_bytes(rows, K, nv, mx):
@@ -65,6 +73,10 @@ def test_host_validation_rejects_bad_arguments():
     assert L.mxfp8_gemm(p, p, p, p, 4, 8, 48, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_amax_bf16(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_amax_bf16_into(p, -1, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.nvfp4_quantize_ex(p, 2, 4, 32, 32, p, 0, 0, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG  # dtype
+    assert L.nvfp4_quantize_ex(p, 0, 4, 32, 32, p, 0, 9, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG  # layout
+    assert L.nvfp4_gemm_ex(p, p, 1, p, p, 65, 8, 64, None, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG  # 8x4 M>64
+    assert L.nvfp4_gemm_ex(p, p, 7, p, p, 4, 8, 64, None, None, None, p, 0, 8, None) == nat.BSP_ERR_INVALID_ARG  # layout
     for bad in (-1.0, float("inf"), float("nan")):  # eps
         assert L.nvfp4_rmsnorm_quantize(p, 4, 32, 32, p, bad, p, 0, None, None, None, p, p, None) == \
             nat.BSP_ERR_INVALID_ARG
