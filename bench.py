@@ -194,10 +194,11 @@ def describe(lin, kind):
     return d
 
 
-def quant_bytes(M, K, kind):
+def quant_bytes(M, K, kind, sf_layout="128x4"):
     """Algorithmic HBM bytes of one activation quantize launch."""
     if kind == "nvfp4":
-        return M * K * 2 + M * K // 2 + (-(-M // 128) * 128) * (-(-(K // 16) // 4) * 4)
+        row_tile = 8 if sf_layout == "8x4" else 128
+        return M * K * 2 + M * K // 2 + (-(-M // row_tile) * row_tile) * (-(-(K // 16) // 4) * 4)
     return M * K * 2 + M * K + (-(-M // 128) * 128) * (-(-(K // 32) // 4) * 4)
 
 
@@ -236,8 +237,11 @@ def run_ours(args, rank, world, local_rank):
 
     # preallocated outputs: the timed step launches exactly our two kernels
     if kind == "nvfp4":
+        if args.sf_layout == "8x4" and (M > 64 or args.norm == "rmsnorm"):
+            raise SystemExit("--sf-layout 8x4 applies to NVFP4 workloads with M <= 64 and no fused norm")
         xq = api.NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
-                             torch.empty(api.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+                             torch.empty(api.nvfp4_sf_bytes(M, K, args.sf_layout), dtype=torch.uint8, device=dev), K,
+                             sf_layout=args.sf_layout)
         if lin.per_token:
             xq.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
             xq.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
@@ -251,7 +255,8 @@ def run_ours(args, rank, world, local_rank):
             api.nvfp4_rmsnorm_quantize(A, gamma, NORM_EPS, None if lin.per_token else layer.gs_x,
                                        per_row=lin.per_token, out=xq)
         elif kind == "nvfp4":
-            api.nvfp4_quantize(A, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=xq)
+            api.nvfp4_quantize(A, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=xq,
+                               sf_layout=args.sf_layout)
         else:
             api.mxfp8_quantize(A, out=xq)
 
@@ -336,7 +341,7 @@ def run_ours(args, rank, world, local_rank):
         if args.norm == "rmsnorm":
             y = layer(A_dev, pre_quantized=layer.rmsnorm_quantize_input(A_dev, gamma, NORM_EPS))
         else:
-            y = layer(A_dev)
+            y = layer(A_dev, sf_layout=args.sf_layout) if kind == "nvfp4" else layer(A_dev)
         D_host.copy_(y, non_blocking=True)
 
     for _ in range(2):
@@ -360,7 +365,7 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     q_ms = statistics.mean(t_q)
     g_ms = statistics.mean(t_g)
-    qb = quant_bytes(M, K, kind)
+    qb = quant_bytes(M, K, kind, args.sf_layout)
     q_gbs = qb / (q_ms * 1e-3) / 1e9
     g_tflops = flops / (g_ms * 1e-3) / 1e12
     ratio = FP4_PER_BF16 if kind == "nvfp4" else FP8_PER_BF16
@@ -391,6 +396,8 @@ def run_ours(args, rank, world, local_rank):
     cfg = describe(lin, kind)
     cfg["parallelism"] = f"replicas x{world}"
     cfg["activation_dtype"] = "fp16" if lin.fmt == "f16" else "bf16"
+    if kind == "nvfp4":
+        cfg["activation_sf_layout"] = args.sf_layout
     if args.norm == "rmsnorm":
         cfg["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
     if kind == "nvfp4":
@@ -622,6 +629,8 @@ def run_reference(args):
     cfg = describe(lin, kind)
     cfg["parallelism"] = "host cores"
     cfg["activation_dtype"] = "fp16" if lin.fmt == "f16" else "bf16"
+    if kind == "nvfp4":
+        cfg["activation_sf_layout"] = args.sf_layout
     if args.norm == "rmsnorm":
         cfg["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
     if kind == "nvfp4":
@@ -642,6 +651,8 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="wan13")
+    ap.add_argument("--sf-layout", choices=["128x4", "8x4"], default="128x4",
+                    help="activation scale layout of the NVFP4 workloads (8x4: M <= 64)")
     ap.add_argument("--norm", choices=["none", "rmsnorm"], default="none",
                     help="NVFP4 workloads: fuse an RMSNorm of the activation into the quantizer")
     ap.add_argument("--input", choices=["bf16", "f16"], default="bf16",
