@@ -67,6 +67,23 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (every rank calls this at the same point)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_rank_step: float, world: int, steps: int, total_ms: float) -> float:
+    """Units per second over all ranks: every rank did `steps` steps of the
+    same work in (at most) the slowest rank's time."""
+    return world * work_per_rank_step * steps / (total_ms * 1e-3)
+
+
 def traffic_for(kernel: str, workload: str):
     """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
     summary, or None when missing or taken on different kernel sources."""
@@ -320,14 +337,11 @@ def run_ours(args, rank, world, local_rank):
     t_q = [ev_split[s][0].elapsed_time(ev_split[s][1]) for s in range(args.steps)]
     t_g = [ev_split[s][1].elapsed_time(ev_split[s][2]) for s in range(args.steps)]
     total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     if api.device_status() != 0:
         raise RuntimeError("device error word set during timing")
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, args.steps, total_ms) / 1e12
     del g_warm, g_timed, g_split, ev_warm
 
     # ---- end to end through the public API: pinned host A in, D back to pinned host
@@ -356,10 +370,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
@@ -412,7 +423,7 @@ def run_ours(args, rank, world, local_rank):
             f"{kind}_gemm": {"ms": round(g_ms, 5), "TFLOP/s": round(g_tflops, 1),
                              "frac_tensor_peak": round(g_tflops / tensor_peak, 4)},
         },
-        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(whole_job_rate(flops, world, 1, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(A_host.numel() * 2), "d2h_bytes_per_step": int(D_host.numel() * 2),
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 2 * args.steps,
@@ -482,13 +493,10 @@ def run_loadtime(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
     total_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     elems = sum(N * K for (_, _, N, K) in shapes)
     nbytes = sum(2 * N * K + 2 * N * K + N * K // 2 + api.nvfp4_sf_bytes(N, K) for (_, _, N, K) in shapes)
-    gbs = world * nbytes * args.steps / (total_ms * 1e-3) / 1e9
+    gbs = whole_job_rate(nbytes, world, args.steps, total_ms) / 1e9
     peaks, src = load_peaks()
     del g
     return {
