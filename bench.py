@@ -344,6 +344,96 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_rate(flops, world, args.steps, total_ms) / 1e12
     del g_warm, g_timed, g_split, ev_warm
 
+    # ---- per-kernel durations for the roofline: R launches of one kernel back to
+    # back in a CUDA graph between two events, rotating through enough distinct
+    # operand buffers (> 3x L2 in total) that every launch reads its streamed
+    # operand from DRAM.  Back to back, consecutive launches hide each other's
+    # launch latency as they do in a model; the per-step split above carries an
+    # event-interval floor of about 6 us per kernel and is reported beside it.
+    # R launches last about 2 ms in all (4 to 24), short enough to stay a burst
+    # like the timed steps rather than a sustained power-capped loop.
+    def launches_for(step_ms):
+        return int(min(24, max(4, 2.0 / max(step_ms, 1e-3))))
+
+    q_step_ms, g_step_ms = statistics.mean(t_q), statistics.mean(t_g)
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def rotations(streamed_bytes):
+        return int(min(8, max(2, -(-3 * l2_bytes // max(1, streamed_bytes)))))
+
+    def back_to_back(launch, n_rot, R):
+        for r in range(n_rot):
+            launch(r)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(R):
+                launch(r % n_rot)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / R
+
+    # the GEMM streams A (large M) or the weight (skinny M) from DRAM
+    w_bytes = layer.weight.codes.numel() + layer.weight.sf.numel() if kind == "nvfp4" else \
+        layer.weight.q.numel() + layer.weight.sf.numel()
+    a_bytes = xq.codes.numel() + xq.sf.numel() if kind == "nvfp4" else xq.q.numel() + xq.sf.numel()
+    rotate_weight = w_bytes > a_bytes
+    nq = rotations(A.numel() * A.element_size())  # bf16 inputs of the quantizer
+    nx = max(nq, 1 if rotate_weight else rotations(a_bytes))  # quantized activations
+    A_rot = [A] + [A.clone() for _ in range(nq - 1)]
+    if kind == "nvfp4":
+        xq_rot = [xq] + [api.NVFP4Tensor(torch.empty_like(xq.codes), torch.empty_like(xq.sf), K,
+                                          sf_layout=xq.sf_layout) for _ in range(nx - 1)]
+        for t in xq_rot[1:]:
+            if lin.per_token:
+                t.row_gs, t.row_inv_gs = torch.empty_like(xq.row_gs), torch.empty_like(xq.row_inv_gs)
+    else:
+        xq_rot = [xq] + [api.MXFP8Tensor(torch.empty_like(xq.q), torch.empty_like(xq.sf), K) for _ in range(nx - 1)]
+
+    def quant_launch(r):
+        x, out = A_rot[r % nq], xq_rot[r]
+        if args.norm == "rmsnorm":
+            api.nvfp4_rmsnorm_quantize(x, gamma, NORM_EPS, None if lin.per_token else layer.gs_x,
+                                       per_row=lin.per_token, out=out)
+        elif kind == "nvfp4":
+            api.nvfp4_quantize(x, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=out,
+                               sf_layout=args.sf_layout)
+        else:
+            api.mxfp8_quantize(x, out=out)
+
+    R_q, R_g = launches_for(q_step_ms), launches_for(g_step_ms)
+    q_b2b_ms = back_to_back(quant_launch, nx, max(R_q, nx))  # also fills every quantized buffer
+    ng = rotations(max(w_bytes, a_bytes))
+    if rotate_weight:
+        w = layer.weight
+        if kind == "nvfp4":
+            w_rot = [w] + [api.NVFP4Tensor(w.codes.clone(), w.sf.clone(), K) for _ in range(ng - 1)]
+        else:
+            w_rot = [w] + [api.MXFP8Tensor(w.q.clone(), w.sf.clone(), K) for _ in range(ng - 1)]
+    D_rot = [D] + [torch.empty_like(D) for _ in range(min(ng, 2) - 1)]
+
+    def gemm_launch(r):
+        a = xq if rotate_weight else xq_rot[r]
+        b = w_rot[r] if rotate_weight else layer.weight
+        out = D_rot[r % len(D_rot)]
+        if kind == "nvfp4":
+            api.nvfp4_gemm(a, b, layer.alpha, a.row_inv_gs if lin.per_token else None, layer.bias, out=out)
+        else:
+            api.mxfp8_gemm(a, b, None, layer.bias, out=out)
+
+    g_b2b_ms = back_to_back(gemm_launch, ng if rotate_weight else nx, R_g)
+    del A_rot, xq_rot, D_rot
+    if rotate_weight:
+        del w_rot
+    q_b2b_ms = max_over_ranks(q_b2b_ms, world, dev)
+    g_b2b_ms = max_over_ranks(g_b2b_ms, world, dev)
+
     # ---- end to end through the public API: every step copies its input from
     # pinned host memory and its result back to pinned host memory.  With large
     # copies the steps are pipelined as a serving loop would run them: the
@@ -409,8 +499,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
-    q_ms = statistics.mean(t_q)
-    g_ms = statistics.mean(t_g)
+    q_ms, g_ms = q_b2b_ms, g_b2b_ms
     qb = quant_bytes(M, K, kind, args.sf_layout)
     q_gbs = qb / (q_ms * 1e-3) / 1e9
     g_tflops = flops / (g_ms * 1e-3) / 1e12
@@ -457,6 +546,11 @@ def run_ours(args, rank, world, local_rank):
             qname: {"ms": round(q_ms, 5), "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / hbm_peak, 4)},
             f"{kind}_gemm": {"ms": round(g_ms, 5), "TFLOP/s": round(g_tflops, 1),
                              "frac_tensor_peak": round(g_tflops / tensor_peak, 4)},
+            "timing": f"{R_q} / {R_g} launches back to back in one CUDA graph between two events (about 2 ms), "
+                      "operands rotated through buffers totalling > 3x L2 so each launch streams from DRAM",
+            "per_step_event_split_ms": {qname: round(q_step_ms, 5), f"{kind}_gemm": round(g_step_ms, 5),
+                                        "note": "events around each kernel inside the timed steps; each "
+                                                "interval carries a ~6 us event/launch floor"},
         },
         "e2e": {"value": round(whole_job_rate(flops, world, 1, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(A_host.numel() * 2), "d2h_bytes_per_step": int(D_host[0].numel() * 2),
