@@ -348,6 +348,9 @@ __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
         } else if constexpr (C::SF_COLS == 32) {
           tmem_st_16cols(taddr, v);
           tmem_st_16cols(taddr + 16, v + 16);
+        } else if constexpr (C::SF_COLS == 24) {
+          tmem_st_16cols(taddr, v);
+          tmem_st_8cols(taddr + 16, v + 16);
         } else if constexpr (C::SF_COLS == 12) {
           tmem_st_4cols(taddr, v);
           tmem_st_8cols(taddr + 4, v + 4);
