@@ -109,6 +109,7 @@ class ClockSampler:
 
     def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons = [], 0
+        self.reason_samples = self.reason_errors = self.clock_errors = 0
         self.max_mhz = None
         self._stop = threading.Event()
         self._ok = False
@@ -138,9 +139,13 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
             except Exception:
-                pass
+                self.clock_errors += 1
+            try:
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.reason_samples += 1
+            except Exception:
+                self.reason_errors += 1
             time.sleep(self._period)
 
     def __enter__(self):
@@ -157,8 +162,13 @@ class ClockSampler:
         if not self._ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+        unknown = self.reasons & ~sum(self.REASONS)
+        if unknown:
+            names.append(f"other_bits_{unknown:#x}")
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_min_mhz": min(self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": names, "reason_mask": f"{self.reasons:#x}",
+                "samples": len(self.samples), "reason_samples": self.reason_samples,
+                "reason_errors": self.reason_errors}
 
 
 # --------------------------------------------------------------------------- workloads
