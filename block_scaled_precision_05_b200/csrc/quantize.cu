@@ -468,13 +468,13 @@ __device__ __forceinline__ double sumsq8(const uint4& v) {
 // Eight normalised outputs as bf16 pairs: bf16(fl32(fl32(x * rstd) * gamma)).
 __device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, float rstd) {
   const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+  const float2 r2 = make_float2(rstd, rstd);
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 xf = InBf16::values2(xw[i]), gf = InBf16::values2(gw[i]);
-    const float lo = __fmul_rn(__fmul_rn(xf.x, rstd), gf.x);
-    const float hi = __fmul_rn(__fmul_rn(xf.y, rstd), gf.y);
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    // two fp32 products per packed instruction, each rounded as a scalar one
+    const float2 y = __fmul2_rn(__fmul2_rn(InBf16::values2(xw[i]), r2), InBf16::values2(gw[i]));
+    const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
     memcpy(&o[i], &h, 4);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
@@ -534,6 +534,96 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
         *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
       }
       sf[sfb_row + (c >> 2) * L::kTileBytes + (c & 3)] = static_cast<uint8_t>(sfb);
+    }
+  }
+}
+
+// K = 512 * S (S = 3, 4: the Wan-1.3B hidden size 1536 among them): the same
+// arithmetic with every row read from DRAM once and kept in registers.  Lane
+// l holds elements [512 s + 16 l, 512 s + 16 l + 16) of the row for s < S (one
+// group of 16 per slab); gamma is re-read per row (it stays in L1).  A warp
+// loads R rows before working on the first, like nvfp4_quant_short_kernel.
+// Rows [M, Mp) are scale padding: y = 0, so their scale bytes are 0.
+#ifndef BSP_RMSNORM_ROWS
+#define BSP_RMSNORM_ROWS 1  // rows in flight per warp at K = 1536
+#endif
+#ifndef BSP_RMSNORM_MIN_BLOCKS
+#define BSP_RMSNORM_MIN_BLOCKS 3  // resident blocks per SM the K = 1536 kernel is compiled for
+#endif
+template <bool kPerRow, int S, int R, int kMinBlocks>
+__global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant_short_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const uint16_t* __restrict__ gamma, float eps,
+    const float* __restrict__ gs_ptr, float* __restrict__ row_gs, float* __restrict__ row_inv,
+    float* __restrict__ row_rstd, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  using L = Sf128x4;
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
+  constexpr int64_t K = 512 * S;
+  const uint32_t lane = lane_id();
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+  const bool quad_lead = (lane & 3u) == 0u;
+  const uint16_t* gp = gamma + lane * 16;  // re-read per row from L1 (registers go to rows in flight)
+  for (int64_t r0 = R * warp; r0 < Mp; r0 += R * nwarps) {
+    uint4 v[R][S][2];
+#pragma unroll
+    for (int h = 0; h < R; ++h) {
+      const int64_t r = r0 + h;
+      const bool live = r < M;
+      const uint16_t* lp = x + r * ld_x + lane * 16;
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        v[h][s][0] = live ? ldg16(lp + s * 512) : make_uint4(0u, 0u, 0u, 0u);
+        v[h][s][1] = live ? ldg16(lp + s * 512 + 8) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < R; ++h) {
+      const int64_t r = r0 + h;
+      if (r >= Mp) break;
+      const bool live = r < M;
+      double acc = 0.0;
+#pragma unroll
+      for (int s = 0; s < S; ++s) acc += sumsq8(v[h][s][0]) + sumsq8(v[h][s][1]);
+      acc = warp_sum_f64(acc);
+      const float ms = __double2float_rn(acc / static_cast<double>(K));
+      const float rstd = __frsqrt_rn(__fadd_rn(ms, eps));
+      if (live && row_rstd != nullptr && lane == 0) row_rstd[r] = rstd;
+      const float rs = live ? rstd : 0.0f;
+      // y is recomputed where it is needed rather than held (register pressure)
+      float gs = gs_tensor;
+      if (kPerRow) {
+        uint32_t mag = 0;
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+          mag = max(mag, max(max_sane_mag8<InBf16>(rmsnorm8(v[h][s][0], ldg16(gp + s * 512), rs)),
+                             max_sane_mag8<InBf16>(rmsnorm8(v[h][s][1], ldg16(gp + s * 512 + 8), rs))));
+        mag = warp_max(mag);
+        gs = global_scale_from_mag<InBf16>(mag);
+        if (live && lane == 0) {
+          if (row_gs) row_gs[r] = gs;
+          if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
+        }
+      }
+      uint8_t* cp = codes + r * (K >> 1) + lane * 8;
+      uint8_t* sp = sf + L::row_base(r, K >> 6) + (lane >> 2) * L::kTileBytes;
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        const uint4 y0 = rmsnorm8(v[h][s][0], ldg16(gp + s * 512), rs);
+        const uint4 y1 = rmsnorm8(v[h][s][1], ldg16(gp + s * 512 + 8), rs);
+        uint32_t sfb;
+        float inv;
+        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv);
+        uint2 w;
+        w.x = nvfp4_codes8<InBf16>(y0, inv);
+        w.y = nvfp4_codes8<InBf16>(y1, inv);
+        const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
+        const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
+        const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
+        if (live) *reinterpret_cast<uint2*>(cp + s * 256) = w;
+        if (quad_lead)
+          *reinterpret_cast<uint32_t*>(sp + s * 8 * L::kTileBytes) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
     }
   }
 }
@@ -860,6 +950,27 @@ int nvfp4_rmsnorm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
   const int64_t Mp = round_up(M, 128);
+  // K = 1536 / 2048: rows in registers (at K = 1024 the three-pass kernel below
+  // measured as fast)
+  if (K == 1536 || K == 2048) {
+    const bool per_row = sf_mode == BSP_SF_PER_ROW;
+    auto launch = [&](auto k, int64_t rows_per_warp) {
+      k<<<grid_for_rows(dev, k, ceil_div(Mp, rows_per_warp)), kQuantThreads, 0, stream>>>(
+          x, M, Mp, ld_x, gamma, eps, global_sf, per_row ? row_gs : nullptr, per_row ? row_inv_gs : nullptr, row_rstd,
+          codes, sf);
+    };
+    switch (K / 512) {
+#define BSP_RMS_CASE(S_, R_, B_)                                                                        \
+  case S_:                                                                                             \
+    per_row ? launch(nvfp4_rmsnorm_quant_short_kernel<true, S_, R_, B_>, R_)                           \
+            : launch(nvfp4_rmsnorm_quant_short_kernel<false, S_, R_, B_>, R_);                         \
+    break;
+      BSP_RMS_CASE(3, BSP_RMSNORM_ROWS, BSP_RMSNORM_MIN_BLOCKS)
+      BSP_RMS_CASE(4, 1, 2)
+#undef BSP_RMS_CASE
+    }
+    return launch_status();
+  }
   if (sf_mode == BSP_SF_PER_ROW) {
     auto k = nvfp4_rmsnorm_quant_kernel<Sf128x4, true>;
     k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, row_gs,

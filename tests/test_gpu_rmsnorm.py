@@ -33,7 +33,10 @@ def _ulps(a, b):
     return np.abs(a.view(np.int32).astype(np.int64) - b.view(np.int32).astype(np.int64))
 
 
-SHAPES = [(1, 16), (7, 48), (130, 1536), (300, 5120), (64, 13824), (129, 80), (257, 1024)]
+# K = 1536 and 2048 take the register-resident kernel (ragged, exact-tile and
+# multi-iteration row counts); the others the three-pass kernel.
+SHAPES = [(1, 16), (7, 48), (130, 1536), (300, 5120), (64, 13824), (129, 80), (257, 1024), (1, 1536), (256, 2048),
+          (4100, 1536), (129, 2048)]
 
 
 @pytest.mark.parametrize("M,K", SHAPES)
@@ -83,3 +86,22 @@ def test_norm_quantized_linear():
     ref, bound = oracle.linear_reference(oracle.nvfp4_dequantize(ca, sa, K), oracle.nvfp4_dequantize(cb, sb, K),
                                          alpha=np.float32(1) / (np.float32(1) * gso), row_scale=None, bias=None)
     assert_gemm_close(D, ref, bound, "rmsnorm-quantized linear")
+
+
+@pytest.mark.parametrize("K", [1536, 2048, 1024])
+def test_rmsnorm_strided_rows(K):
+    """Rows read with a row stride larger than K (a column slice of a wider tensor)."""
+    M = 200
+    x, g = _case(M, K + 64, seed=K + 5)
+    xs = up_bf16(x)[:, :K]
+    assert xs.stride(0) == K + 64
+    rstd = torch.empty(M, dtype=torch.float32, device=DEV)
+    q = api.nvfp4_rmsnorm_quantize(xs, up_bf16(g[:K].copy()), 1e-6, None, per_row=True, rstd_out=rstd)
+    assert api.device_status() == 0
+    xk = np.ascontiguousarray(x[:, :K])
+    r_gpu = down(rstd)
+    assert _ulps(r_gpu, oracle.rmsnorm_rstd(xk, 1e-6)).max() <= 2
+    codes, sf, _, g_rows, _ = oracle.rmsnorm_quantize(xk, g[:K].copy(), 1e-6, np.float32(1.0), per_row=True,
+                                                      rstd=r_gpu)
+    assert np.array_equal(down(q.codes), codes) and np.array_equal(down(q.sf), sf)
+    assert np.array_equal(down(q.row_gs), g_rows)
