@@ -27,6 +27,7 @@ Under torchrun (N > 1) every rank runs the same workload on its own GPU
 from __future__ import annotations
 
 import argparse
+import contextlib
 import datetime
 import hashlib
 import json
@@ -581,9 +582,11 @@ def run_loadtime(args, rank, world, local_rank):
     """Load-time weight conversion of a synthetic 14B-class DiT stack: for each
     of the 240 linears of 40 blocks (q, k, v, out 5120x5120; fc_in 13824x5120;
     fc_out 5120x13824; bf16 ~N(0, 0.02), drawn on the device from seeded
-    generators), amax -> gs_w = 2688/amax -> NVFP4 quantize.  The whole sweep
-    (4 launches per weight) is one CUDA graph; one step = one sweep.  The
-    weights (19.7 GB) are far larger than L2."""
+    generators), amax -> gs_w = 2688/amax -> NVFP4 quantize, one
+    nvfp4_quantize_weight launch per weight.  The whole sweep is one CUDA
+    graph; one step = one sweep.  The weights (19.7 GB) are far larger than L2.
+    The same sweep as three launches per weight (amax, global scale, quantize,
+    plus the amax reset) is timed beside it."""
     import torch
     import torch.distributed as dist
 
@@ -599,60 +602,82 @@ def run_loadtime(args, rank, world, local_rank):
         weights.append(w)
         outs.append(api.NVFP4Tensor(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
                                     torch.empty(api.nvfp4_sf_bytes(N, K), dtype=torch.uint8, device=dev), K))
-        scales.append((torch.empty(1, dtype=torch.float32, device=dev), torch.empty(1, dtype=torch.float32, device=dev),
-                       torch.empty(1, dtype=torch.float32, device=dev)))
+        scales.append(tuple(torch.empty(1, dtype=torch.float32, device=dev) for _ in range(3)))
     from block_scaled_precision_05_b200 import _native as nat
     L = nat.lib()
+    ws = api._weight_workspace(dev, nat.BSP_IN_BF16)
 
     def sweep():
+        st = torch.cuda.current_stream().cuda_stream
+        for w, o, (amax, gs, inv) in zip(weights, outs, scales):
+            N, K = w.shape
+            nat.check(L.nvfp4_quantize_weight(w.data_ptr(), nat.BSP_IN_BF16, N, K, K, api.FP8_FP4_MAX,
+                                              amax.data_ptr(), gs.data_ptr(), inv.data_ptr(), o.codes.data_ptr(),
+                                              o.sf.data_ptr(), ws.data_ptr(), ws.numel(), st), "quantize_weight")
+
+    def sweep_unfused():
         st = torch.cuda.current_stream().cuda_stream
         for w, o, (amax, gs, inv) in zip(weights, outs, scales):
             nat.check(L.bsp_amax_bf16(w.data_ptr(), w.numel(), amax.data_ptr(), st), "amax")
             nat.check(L.bsp_nvfp4_global_scale(amax.data_ptr(), gs.data_ptr(), inv.data_ptr(), st), "gs")
             api.nvfp4_quantize(w, gs, out=o)
 
-    for _ in range(2):
-        sweep()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        sweep()
-    for _ in range(args.warmup):
-        g.replay()
-    torch.cuda.synchronize()
-    if api.device_status() != 0:
-        raise RuntimeError("device error word set")
-    stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier(device_ids=[local_rank])
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
-        e0.record(stream)
-        for _ in range(args.steps):
-            g.replay()
-        e1.record(stream)
+    def timed(fn, steps, clocks=None):
+        for _ in range(2):
+            fn()
         torch.cuda.synchronize()
-    total_ms = e0.elapsed_time(e1)
-    total_ms = max_over_ranks(total_ms, world, dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        if api.device_status() != 0:
+            raise RuntimeError("device error word set")
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize()
+        with (clocks if clocks is not None else contextlib.nullcontext()):
+            e0.record(stream)
+            for _ in range(steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        del g
+        if api.device_status() != 0:
+            raise RuntimeError("device error word set")
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    clocks = ClockSampler(local_rank)
+    total_ms = timed(sweep, args.steps, clocks)
+    unfused_ms = timed(sweep_unfused, max(1, args.steps // 2)) / max(1, args.steps // 2)
     elems = sum(N * K for (_, _, N, K) in shapes)
+    # algorithmic bytes of the two passes the conversion needs (the amax pass and
+    # the quantize pass, 2 + 2.5625 B/elt); the one-kernel form re-reads a weight
+    # from L2 where it fits, which this count does not credit
     nbytes = sum(2 * N * K + 2 * N * K + N * K // 2 + api.nvfp4_sf_bytes(N, K) for (_, _, N, K) in shapes)
     gbs = whole_job_rate(nbytes, world, args.steps, total_ms) / 1e9
     peaks, src = load_peaks()
-    del g
     return {
         "metric": "load-time NVFP4 weight conversion (amax + global scale + quantize) GB/s", "value": round(gbs, 1),
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded torch, on device)",
         "config": {"workload": f"loadtime: {len(shapes)} DiT linears ({args.blocks} blocks), {elems / 1e9:.2f} G "
-                               "bf16 elements", "l2": "inputs (19.7 GB at 40 blocks) far larger than L2"},
-        "roofline": {"kernel": "amax + nvfp4_quantize (whole sweep)", "bound": "hbm", "achieved": round(gbs / world, 1),
+                               "bf16 elements", "l2": "inputs (19.7 GB at 40 blocks) far larger than L2",
+                   "kernel": "nvfp4_quantize_weight: one cooperative launch per weight (amax, grid barrier, "
+                             "global scale, quantize last row first)"},
+        "roofline": {"kernel": "nvfp4_quantize_weight (whole sweep)", "bound": "hbm", "achieved": round(gbs / world, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / world / peaks["hbm_gbs"], 4),
                      "traffic": None, "peak_source": f"{src}: hbm_gbs",
-                     "algorithmic": f"{nbytes} bytes per sweep (amax read 2 B/elt; quantize 2 B read + 0.5 B "
-                                    "codes + scales)"},
-        "gpu_launches": 3 * len(shapes) * args.steps,
+                     "algorithmic": f"{nbytes} bytes per sweep (amax pass 2 B/elt; quantize pass 2 B/elt read + "
+                                    "0.5 B/elt codes + scales)"},
+        "unfused": {"ms_per_step": round(unfused_ms, 4),
+                    "GB/s_same_bytes": round(nbytes / (unfused_ms * 1e-3) / 1e9, 1),
+                    "launches_per_weight": "memset + amax + global scale + quantize"},
+        "gpu_launches": len(shapes) * args.steps,
         "clocks": clocks.summary(),
     }
 
@@ -742,7 +767,7 @@ def run_reference_loadtime(args):
     for _ in range(args.steps):
         step()
     dt = time.perf_counter() - t0
-    nbytes = 4 * N * K + N * K // 2 + oracle.sf_bytes(N, K // 16)
+    nbytes = 4 * N * K + N * K // 2 + oracle.sf_bytes(N, K // 16)  # amax pass + quantize pass, as the GPU arm
     value = nbytes * args.steps / dt / 1e9
     cores = os.cpu_count() or 1
     sample = "one 5120x5120 bf16 weight per step: amax + global scale + NVFP4 quantize (plain C oracle)"

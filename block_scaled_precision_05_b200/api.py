@@ -19,6 +19,7 @@ Sources (page title, then symbol):
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 
 import torch
@@ -203,6 +204,53 @@ def nvfp4_quantize(x: torch.Tensor, global_sf: torch.Tensor | None = None, per_r
     return out
 
 
+# one zero-initialised workspace per (device, input format), created on first use
+_WEIGHT_WS: dict[tuple[int, int], torch.Tensor] = {}
+
+
+def _weight_workspace(device: torch.device, w_dtype: int) -> torch.Tensor:
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _WEIGHT_WS.get((idx, w_dtype))
+    if ws is None:
+        if torch.cuda.is_current_stream_capturing():
+            raise RuntimeError("nvfp4_quantize_weight: the first call on a device sets up its workspace and must "
+                               "not be inside a CUDA graph capture")
+        n = ctypes.c_int64(0)
+        with torch.cuda.device(idx):
+            nat.check(nat.lib().bsp_nvfp4_quantize_weight_workspace_bytes(w_dtype, ctypes.addressof(n)),
+                      "bsp_nvfp4_quantize_weight_workspace_bytes")
+        ws = torch.zeros(n.value, dtype=torch.uint8, device=torch.device("cuda", idx))
+        _WEIGHT_WS[(idx, w_dtype)] = ws
+    return ws
+
+
+def nvfp4_quantize_weight(w: torch.Tensor, fp8_fp4_max: float = FP8_FP4_MAX, out: NVFP4Tensor | None = None):
+    """Load-time weight conversion in one kernel: amax, gs = fp8_fp4_max/amax and
+    the per-tensor NVFP4 quantization with gs, bit-identical to amax ->
+    nvfp4_global_scale -> nvfp4_quantize.  bf16 or fp16 [N, K], K % 64 == 0.
+    Returns (NVFP4Tensor, gs, 1/gs, amax), the scalars fp32 [1] device tensors.
+    The kernel's workspace is kept per device; calls on one device must not
+    overlap in time (one stream, or ordered streams)."""
+    _require_cuda(w)
+    w = coerce_input(w)
+    if w.dim() != 2 or w.shape[1] % 64 != 0:
+        raise ValueError(f"nvfp4_quantize_weight expects [N, K] with K % 64 == 0, got {tuple(w.shape)}")
+    if w.stride(1) != 1:
+        w = w.contiguous()
+    N, K = w.shape
+    dev = w.device
+    if out is None:
+        out = NVFP4Tensor(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                          torch.empty(nvfp4_sf_bytes(N, K), dtype=torch.uint8, device=dev), K)
+    gs, inv, am = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(3))
+    w_dtype = nat.BSP_IN_F16 if w.dtype == torch.float16 else nat.BSP_IN_BF16
+    ws = _weight_workspace(dev, w_dtype)
+    nat.check(nat.lib().nvfp4_quantize_weight(_ptr(w), w_dtype, N, K, w.stride(0), float(fp8_fp4_max), _ptr(am),
+                                              _ptr(gs), _ptr(inv), _ptr(out.codes), _ptr(out.sf), _ptr(ws),
+                                              ws.numel(), _stream()), "nvfp4_quantize_weight")
+    return out, gs, inv, am
+
+
 def nvfp4_rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
                            global_sf: torch.Tensor | None = None, per_row: bool = False,
                            out: NVFP4Tensor | None = None, rstd_out: torch.Tensor | None = None) -> NVFP4Tensor:
@@ -313,7 +361,8 @@ def device_status() -> int:
 # --------------------------------------------------------------------------- linear layers
 class NVFP4Linear:
     """W4A4 NVFP4 linear layer: the weight is quantized once at construction
-    (amax -> gs_w -> quantize; the bf16 weight is not kept), each call quantizes
+    (amax -> gs_w -> quantize, one kernel when K % 64 == 0; the bf16 weight is
+    not kept), each call quantizes
     the activation and runs the block-scaled GEMM with alpha and bias fused.
 
     per_token=False: static activation scale gs_x = 1.0 (no reduction, no host
@@ -334,11 +383,15 @@ class NVFP4Linear:
         w = coerce_input(weight).contiguous()
         self.out_features, self.in_features = w.shape
         self.per_token = per_token
-        if global_scale is None:
-            self.gs_w, self.inv_gs_w = nvfp4_global_scale(amax(w), FP8_FP4_MAX_4OVER6 if four_over_six else FP8_FP4_MAX)
+        fmax = FP8_FP4_MAX_4OVER6 if four_over_six else FP8_FP4_MAX
+        if global_scale is None and self.in_features % 64 == 0:
+            self.weight, self.gs_w, self.inv_gs_w, _ = nvfp4_quantize_weight(w, fmax)
         else:
-            self.gs_w, self.inv_gs_w = global_scale
-        self.weight = nvfp4_quantize(w, self.gs_w)
+            if global_scale is None:
+                self.gs_w, self.inv_gs_w = nvfp4_global_scale(amax(w), fmax)
+            else:
+                self.gs_w, self.inv_gs_w = global_scale
+            self.weight = nvfp4_quantize(w, self.gs_w)
         self.gs_x = torch.ones(1, dtype=torch.float32, device=w.device)
         # per-token: the GEMM applies 1/gs_w here and 1/gs_x[m] as the row scale
         self.alpha = self.inv_gs_w if per_token else nvfp4_alpha(self.gs_x, self.gs_w)

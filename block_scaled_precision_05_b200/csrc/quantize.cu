@@ -358,40 +358,48 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
   }
 }
 
+// Row r (K % 64 == 0) with scale gs, by one warp: group g = 32 * step + lane
+// covers elements 16 g, code bytes 8 g and scale tile g / 4.  A row past the
+// tensor (live false) only writes its zero scale bytes.
+template <class In, class L, int U = kUnroll>
+__device__ __forceinline__ void nvfp4_row_k64(const uint16_t* row, int64_t K, int64_t r, bool live, float gs,
+                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, uint32_t lane) {
+  const int64_t groups = K >> 4;
+  const int64_t steps = groups >> 5;  // full warp steps (32 groups) per row
+  const int64_t rem = groups & 31;    // groups of a last, partial step (a multiple of 4)
+  const bool quad_lead = (lane & 3u) == 0u;
+  const uint16_t* lp = row + lane * 16;
+  uint8_t* cp = codes + r * (K >> 1) + lane * 8;
+  uint8_t* sp = sf + L::row_base(r, groups >> 2) + (lane >> 2) * L::kTileBytes;
+  constexpr int kStepSf = 8 * L::kTileBytes;  // a warp step covers 8 scale tiles
+  int64_t st = 0;
+  for (; st + U <= steps; st += U)
+    nvfp4_steps<In, L, U>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
+  for (; st < steps; ++st)
+    nvfp4_steps<In, L, 1>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
+  if (rem) {
+    const bool in = lane < rem;  // groups beyond the row end are predicated off
+    nvfp4_steps<In, L, 1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * kStepSf : sp, live && in,
+                          gs, in && quad_lead);
+  }
+}
+
 template <class In, class L, bool kPerRow>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const float* __restrict__ gs_ptr,
     float* __restrict__ row_gs, float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
   allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   const uint32_t lane = lane_id();
-  const int64_t groups = K >> 4;
-  const int64_t steps = groups >> 5;  // full warp steps (32 groups) per row
-  const int64_t rem = groups & 31;    // groups of a last, partial step (a multiple of 4)
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
-  const bool quad_lead = (lane & 3u) == 0u;
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const bool live = r < M;
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
     if (kPerRow && live) gs = row_scale_pass<In>(row, K, r, row_gs, row_inv);
-    // group g = 32 * step + lane: elements 16 g, code bytes 8 g, scale tile g / 4
-    const uint16_t* lp = row + lane * 16;
-    uint8_t* cp = codes + r * (K >> 1) + lane * 8;
-    uint8_t* sp = sf + L::row_base(r, groups >> 2) + (lane >> 2) * L::kTileBytes;
-    constexpr int kStepSf = 8 * L::kTileBytes;  // a warp step covers 8 scale tiles
-    int64_t st = 0;
-    for (; st + kUnroll <= steps; st += kUnroll)
-      nvfp4_steps<In, L, kUnroll>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
-    for (; st < steps; ++st)
-      nvfp4_steps<In, L, 1>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
-    if (rem) {
-      const bool in = lane < rem;  // groups beyond the row end are predicated off
-      nvfp4_steps<In, L, 1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * kStepSf : sp,
-                            live && in, gs, in && quad_lead);
-    }
+    nvfp4_row_k64<In, L>(row, K, r, live, gs, codes, sf, lane);
   }
 }
 
@@ -781,6 +789,142 @@ __global__ void global_scale_kernel(const float* __restrict__ amax, float fp8_fp
   if (inv_gs) *inv_gs = __fdiv_rn(1.0f, g);
 }
 
+// ---------------------------------------------------------------------------
+// Load-time weight conversion in one launch (the weight path of
+// sgl-project sglang nvfp4_online.py, _quantize_weight_nvfp4, and of
+// hao-ai-lab-FastVideo nvfp4_config.py: amax, then gs_w = fp8_fp4_max / amax,
+// then the NVFP4 quantization with gs_w), K % 64 == 0:
+//   1. every block folds its share of max|w| (sanitized as bsp_amax) into one
+//      word of the workspace;
+//   2. grid barrier;
+//   3. every block reduces the words to amax and derives gs and 1/gs exactly as
+//      bsp_nvfp4_global_scale_max; block 0 stores them;
+//   4. the rows are quantized with gs by nvfp4_row_k64, last row first, so the
+//      rows phase 1 read last are re-read from L2 rather than DRAM (a weight
+//      smaller than L2 is read from DRAM once).
+// The grid is one co-resident wave (a cooperative launch where the runtime
+// allows it), so every block reaches the barrier.
+// Workspace: [0] arrivals at the barrier (0 outside it; must be 0 before the
+// first launch), [1] barrier generation, then one word per block from byte
+// kWeightWsHeader.
+// ---------------------------------------------------------------------------
+constexpr int64_t kWeightWsHeader = 256;
+#ifndef BSP_WQ_AMAX_LOADS
+#define BSP_WQ_AMAX_LOADS 8  // 16-byte loads in flight per thread in the amax phase
+#endif
+#ifndef BSP_WQ_ROW_STEPS
+#define BSP_WQ_ROW_STEPS 4  // warp steps in flight per row in the quantize phase
+#endif
+#ifndef BSP_WQ_MIN_BLOCKS
+#define BSP_WQ_MIN_BLOCKS 1
+#endif
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// All blocks of the grid meet here (bounded: false after kWaitLimitNs, with the
+// error word raised).  The last block to arrive resets the arrival count and
+// advances the generation, which releases the others.
+__device__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks, uint32_t* err) {
+  __shared__ int ok_sh;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    __threadfence();  // this block's writes are visible before its arrival
+    const uint32_t g0 = ld_acquire_gpu(gen);
+    if (atomicAdd(count, 1u) == nblocks - 1u) {
+      atomicExch(count, 0u);
+      __threadfence();
+      atomicAdd(gen, 1u);
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(gen) == g0) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          ok = false;
+          raise_error(err, kErrTimeout);
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    ok_sh = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return ok_sh != 0;
+}
+
+// Block-wide max of a per-thread magnitude, returned to every thread.
+__device__ __forceinline__ uint32_t block_max(uint32_t m) {
+  __shared__ uint32_t red[kQuantThreads / 32];
+  m = warp_max(m);
+  __syncthreads();  // red may still be read from a previous call
+  if (lane_id() == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = lane_id() < kQuantThreads / 32 ? red[lane_id()] : 0u;
+  return warp_max(m);
+}
+
+template <class In>
+__global__ void __launch_bounds__(kQuantThreads, BSP_WQ_MIN_BLOCKS) nvfp4_weight_kernel(
+    const uint16_t* __restrict__ w, int64_t N, int64_t Np, int64_t K, int64_t ld_w, float fp8_fp4_max,
+    float* __restrict__ amax_out, float* __restrict__ gs_out, float* __restrict__ inv_out, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ sf, uint8_t* __restrict__ ws, uint32_t* __restrict__ err) {
+  uint32_t* count = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* gen = count + 1;
+  uint32_t* part = reinterpret_cast<uint32_t*>(ws + kWeightWsHeader);
+  const uint32_t lane = lane_id();
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t warp = tid >> 5, nwarps = nthreads >> 5;
+
+  // 1. max|w| (sanitized magnitudes as in amax_kernel)
+  uint32_t m = 0;
+  if (ld_w == K) {
+    constexpr int A = BSP_WQ_AMAX_LOADS;
+    const int64_t nvec = (N * K) >> 3;
+    int64_t i = tid;
+    for (; i + (A - 1) * nthreads < nvec; i += A * nthreads) {
+      uint4 v[A];
+#pragma unroll
+      for (int j = 0; j < A; ++j) v[j] = ldg16(w + (i + j * nthreads) * 8);
+#pragma unroll
+      for (int j = 0; j < A; ++j) m = max(m, max_sane_mag8<In>(v[j]));
+    }
+    for (; i < nvec; i += nthreads) m = max(m, max_sane_mag8<In>(ldg16(w + i * 8)));
+  } else {
+    for (int64_t r = warp; r < N; r += nwarps)
+      for (int64_t c = lane * 8; c < K; c += 256) m = max(m, max_sane_mag8<In>(ldg16(w + r * ld_w + c)));
+  }
+  m = block_max(m);
+  if (threadIdx.x == 0) part[blockIdx.x] = m;
+
+  // 2.
+  if (!grid_barrier(count, gen, gridDim.x, err)) return;
+
+  // 3. (the words are read through L2: other SMs wrote them)
+  m = 0;
+  for (int64_t i = threadIdx.x; i < gridDim.x; i += blockDim.x) m = max(m, __ldcg(part + i));
+  m = block_max(m);
+  const float amax = m == 0u ? 0.0f : In::value(m);
+  const float gs = amax > 0.0f ? __fdiv_rn(fp8_fp4_max, amax) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (amax_out) *amax_out = amax;
+    if (gs_out) *gs_out = gs;
+    if (inv_out) *inv_out = __fdiv_rn(1.0f, gs);
+  }
+
+  // 4.
+  for (int64_t i = warp; i < Np; i += nwarps) {
+    const int64_t r = Np - 1 - i;
+    const bool live = r < N;
+    nvfp4_row_k64<In, Sf128x4, BSP_WQ_ROW_STEPS>(w + (live ? r : 0) * ld_w, K, r, live, gs, codes, sf, lane);
+  }
+}
+
 __global__ void alpha_kernel(const float* __restrict__ gs_x, const float* __restrict__ gs_w, float* alpha) {
   *alpha = __fdiv_rn(1.0f, __fmul_rn(*gs_x, *gs_w));
 }
@@ -900,6 +1044,51 @@ int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, co
     }
   }
   return launch_status();
+}
+
+// Blocks of nvfp4_weight_kernel<In> resident at once on this device: its grid.
+template <class In>
+int weight_grid(const DeviceInfo& dev, int* grid) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_weight_kernel<In>, kQuantThreads, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return (cudaGetLastError(), BSP_ERR_CUDA);
+  *grid = dev.sm_count * per_sm;
+  return BSP_OK;
+}
+
+template <class In>
+int run_nvfp4_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ld_w, float fp8_fp4_max, float* amax,
+                              float* gs, float* inv_gs, uint8_t* codes, uint8_t* sf, void* ws, int64_t ws_bytes,
+                              cudaStream_t stream) {
+  if (N < 0 || K <= 0 || K % 64 != 0 || ld_w < K) return BSP_ERR_INVALID_ARG;
+  if (!(fp8_fp4_max > 0.0f) || !(fp8_fp4_max <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
+  if ((N > 0 && !w) || !codes || !sf || !gs || !inv_gs || !ws) return BSP_ERR_INVALID_ARG;
+  if ((w && !aligned16(w)) || !aligned16(codes) || !aligned16(sf) || !aligned16(ws) || ld_w % 8 != 0 ||
+      (reinterpret_cast<uintptr_t>(gs) & 3u) || (reinterpret_cast<uintptr_t>(inv_gs) & 3u) ||
+      (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  int grid = 0;
+  if ((st = weight_grid<In>(dev, &grid)) != BSP_OK) return st;
+  if (ws_bytes < kWeightWsHeader + 4 * static_cast<int64_t>(grid)) return BSP_ERR_INVALID_ARG;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeCooperative;  // all blocks resident at once, or no launch
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int64_t Np = round_up(N, 128);
+  if (cudaLaunchKernelEx(&cfg, nvfp4_weight_kernel<In>, w, N, Np, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf,
+                         static_cast<uint8_t*>(ws), dev.err_word) != cudaSuccess)
+    return launch_status();
+  return BSP_OK;
 }
 
 }  // namespace
@@ -1027,6 +1216,29 @@ int bsp_nvfp4_global_scale_max(const float* amax, float fp8_fp4_max, float* gs, 
   if (st != BSP_OK) return st;
   global_scale_kernel<<<1, 1, 0, stream>>>(amax, fp8_fp4_max, gs, inv_gs);
   return launch_status();
+}
+
+int bsp_nvfp4_quantize_weight_workspace_bytes(int w_dtype, int64_t* bytes) {
+  if (!bytes || (w_dtype != BSP_IN_BF16 && w_dtype != BSP_IN_F16)) return BSP_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  int grid = 0;
+  st = w_dtype == BSP_IN_F16 ? weight_grid<InF16>(dev, &grid) : weight_grid<InBf16>(dev, &grid);
+  if (st != BSP_OK) return st;
+  *bytes = kWeightWsHeader + 4 * static_cast<int64_t>(grid);
+  return BSP_OK;
+}
+
+int nvfp4_quantize_weight(const uint16_t* w, int w_dtype, int64_t N, int64_t K, int64_t ld_w, float fp8_fp4_max,
+                          float* amax, float* gs, float* inv_gs, uint8_t* codes, uint8_t* sf, void* workspace,
+                          int64_t workspace_bytes, bsp_stream_t stream) {
+  if (w_dtype == BSP_IN_F16)
+    return run_nvfp4_quantize_weight<InF16>(w, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf, workspace,
+                                            workspace_bytes, stream);
+  if (w_dtype != BSP_IN_BF16) return BSP_ERR_INVALID_ARG;
+  return run_nvfp4_quantize_weight<InBf16>(w, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf, workspace,
+                                           workspace_bytes, stream);
 }
 
 int bsp_nvfp4_global_scale(const float* amax, float* gs, float* inv_gs, bsp_stream_t stream) {

@@ -161,6 +161,43 @@ int bsp_nvfp4_global_scale_max(const float *amax, float fp8_fp4_max, float *gs, 
  * NVFP4QATQuantizeMethod.apply.  All fp32 [1]. */
 int bsp_nvfp4_alpha(const float *gs_x, const float *gs_w, float *alpha, bsp_stream_t stream);
 
+/* Load-time weight conversion in one launch: the sequence
+ *   bsp_amax_{bf16,f16}(w) -> bsp_nvfp4_global_scale_max(amax, fp8_fp4_max)
+ *   -> nvfp4_quantize(w, gs) (per-tensor, layout_128x4)
+ * of the weight path of nvfp4_online.py (_quantize_weight_nvfp4: amax, the
+ * e4m3_max * 6 / amax global scale, quantize) and nvfp4_config.py
+ * (process_weights_after_loading), with bit-identical results.  One grid of
+ * co-resident blocks reduces max|w| through the workspace, meets at a grid
+ * barrier, derives gs on every block and quantizes the rows last row first,
+ * so that a weight smaller than L2 is read from DRAM once.
+ *   w            : bf16 / fp16 [N, K] (w_dtype BSP_IN_BF16 / BSP_IN_F16), row
+ *                  stride ld_w elements, 16-byte aligned
+ *   N, K, ld_w   : N >= 0, K > 0 and K % 64 == 0, ld_w >= K and ld_w % 8 == 0
+ *   fp8_fp4_max  : host value, finite and > 0 (2688, or 1536 for 4over6)
+ *   amax         : fp32 [1] max|w| (NaN 0, +-inf the largest finite), or NULL
+ *   gs, inv_gs   : fp32 [1], as bsp_nvfp4_global_scale_max
+ *   codes, sf    : outputs as nvfp4_quantize (N rows; round_up(N, 128) rows of
+ *                  scales, the padding rows zero)
+ *   workspace    : device memory of workspace_bytes >= the size that
+ *                  bsp_nvfp4_quantize_weight_workspace_bytes reports for this
+ *                  device and w_dtype, 16-byte aligned, its first 4 bytes zero
+ *                  before the first call; each call leaves them zero again.
+ *                  Owned by the caller; calls that overlap in time on one
+ *                  workspace race.
+ * Launched cooperatively (every block resident at once).  Errors:
+ * INVALID_ARG (sizes, modes, NULL pointers, workspace too small), ALIGNMENT,
+ * UNSUPPORTED_DEVICE, CUDA (the launch failed, e.g. a cooperative launch the
+ * context does not allow); a barrier wait that runs out (2 s) raises the
+ * device error word (bsp_device_status: TIMEOUT) and leaves the outputs
+ * unspecified. */
+int nvfp4_quantize_weight(const uint16_t *w, int w_dtype, int64_t N, int64_t K, int64_t ld_w, float fp8_fp4_max,
+                          float *amax, float *gs, float *inv_gs, uint8_t *codes, uint8_t *sf, void *workspace,
+                          int64_t workspace_bytes, bsp_stream_t stream);
+
+/* Workspace bytes nvfp4_quantize_weight needs on the current device for
+ * w_dtype (a header and one word per block of its grid).  Host-only. */
+int bsp_nvfp4_quantize_weight_workspace_bytes(int w_dtype, int64_t *bytes);
+
 /* ------------------------------------------------------------------------
  * NVFP4 quantization (nvfp4_config.py: fastvideo_fp4::nvfp4_quantize and
  * _nvfp4_quantize; module docstring: e2m1 elements, group size 16, e4m3

@@ -86,6 +86,18 @@ def test_host_validation_rejects_bad_arguments():
         assert L.bsp_nvfp4_global_scale_max(p, bad, p, p, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_nvfp4_global_scale_max(p, 1536.0, None, None, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_debug_wait_timeout(10, None) == nat.BSP_ERR_INVALID_ARG
+    qw = L.nvfp4_quantize_weight
+    assert qw(p, 0, 4, 48, 48, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # K % 64
+    assert qw(p, 0, 4, 64, 32, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # ld < K
+    assert qw(p, 2, 4, 64, 64, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # dtype
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert qw(p, 0, 4, 64, 64, bad, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG
+    assert qw(p, 0, 4, 64, 64, 2688.0, None, p, p, p, p, None, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # no ws
+    assert qw(p, 0, 4, 64, 64, 2688.0, None, None, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # no gs
+    assert qw(odd, 0, 4, 64, 64, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_ALIGNMENT
+    assert qw(p, 0, 4, 64, 68, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_ALIGNMENT  # ld % 8
+    assert L.bsp_nvfp4_quantize_weight_workspace_bytes(0, None) == nat.BSP_ERR_INVALID_ARG
+    assert L.bsp_nvfp4_quantize_weight_workspace_bytes(5, p) == nat.BSP_ERR_INVALID_ARG
 
 
 def test_no_gpu_means_an_error_not_a_fallback():

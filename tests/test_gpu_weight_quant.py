@@ -1,0 +1,143 @@
+"""Load-time weight conversion in one kernel (nvfp4_quantize_weight) on the GPU.
+
+The entry fuses the weight path of sgl-project sglang nvfp4_online.py
+(_quantize_weight_nvfp4: amax, gs = e4m3_max * 6 / amax, quantize) into one
+cooperative launch with a grid barrier.  Its results must be bit-identical to
+the three-launch sequence amax -> global scale -> nvfp4_quantize, and to the
+oracle's amax, global scale and quantization."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_scaled_precision_05_b200 import api
+from block_scaled_precision_05_b200 import workloads as wl
+from tests._gpu import DEV, down, up_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(rows, K, seed, std=0.02):
+    rng = np.random.default_rng(seed)
+    return wl.f32_to_bf16_bits((rng.standard_normal((rows, K)) * std).astype(np.float32))
+
+
+def _three_launches(w, fmax):
+    a = api.amax(w)
+    gs, inv = api.nvfp4_global_scale(a, fmax)
+    return api.nvfp4_quantize(w, gs), gs, inv, a
+
+
+def _assert_same(fused, ref):
+    (q1, g1, i1, a1), (q2, g2, i2, a2) = fused, ref
+    assert torch.equal(q1.codes, q2.codes)
+    assert torch.equal(q1.sf, q2.sf)
+    for x, y in ((g1, g2), (i1, i2), (a1, a2)):
+        assert torch.equal(x, y), (x, y)
+
+
+SHAPES = [(1, 64), (7, 128), (130, 1536), (300, 5120), (1000, 13824), (5120, 5120), (13824, 5120), (333, 576)]
+
+
+@pytest.mark.parametrize("N,K", SHAPES)
+@pytest.mark.parametrize("fmax", [api.FP8_FP4_MAX, api.FP8_FP4_MAX_4OVER6])
+def test_matches_three_launches(N, K, fmax):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(N * 7 + K)
+    w = (torch.randn((N, K), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    fused = api.nvfp4_quantize_weight(w, fmax)
+    ref = _three_launches(w, fmax)
+    assert api.device_status() == 0
+    _assert_same(fused, ref)
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (130, 1536), (257, 640)])
+def test_matches_oracle(N, K):
+    W = _bf16(N, K, seed=N + K)
+    q, gs, inv, a = api.nvfp4_quantize_weight(up_bf16(W))
+    assert api.device_status() == 0
+    a_ref = oracle.amax_bf16(W)
+    g_ref = oracle.nvfp4_global_scale(a_ref)
+    assert down(a)[0] == np.float32(a_ref)
+    assert down(gs)[0] == g_ref and down(inv)[0] == np.float32(1.0) / g_ref
+    codes, sf = oracle.nvfp4_quantize(W, g_ref)
+    assert np.array_equal(down(q.codes), codes)
+    assert np.array_equal(down(q.sf), sf)
+
+
+def test_special_values_and_zero_weight():
+    W = _bf16(200, 256, seed=5)
+    W[3, 7] = 0x7F80   # +inf counts as the largest finite value
+    W[9, 0] = 0x7FC1   # NaN counts as 0
+    W[11, 1] = 0x0001  # subnormal
+    w = up_bf16(W)
+    _assert_same(api.nvfp4_quantize_weight(w), _three_launches(w, api.FP8_FP4_MAX))
+    z = torch.zeros((130, 128), dtype=torch.bfloat16, device=DEV)
+    q, gs, inv, a = api.nvfp4_quantize_weight(z)
+    assert down(a)[0] == 0.0 and down(gs)[0] == 1.0 and down(inv)[0] == 1.0
+    assert not q.codes.any() and not q.sf.any()
+    assert api.device_status() == 0
+
+
+def test_f16_weight():
+    rng = np.random.default_rng(8)
+    W = (rng.standard_normal((300, 1024)) * 30).astype(np.float16).view(np.uint16)
+    W[0, 5] = 0xFC00  # -inf -> 65504
+    w = torch.from_numpy(W.view(np.int16)).view(torch.float16).to(DEV)
+    fused = api.nvfp4_quantize_weight(w)
+    _assert_same(fused, _three_launches(w, api.FP8_FP4_MAX))
+    g_ref = oracle.nvfp4_global_scale(oracle.amax_f16(W))
+    assert down(fused[1])[0] == g_ref
+    codes, sf = oracle.nvfp4_quantize(W, g_ref, fmt="f16")
+    assert np.array_equal(down(fused[0].codes), codes) and np.array_equal(down(fused[0].sf), sf)
+
+
+def test_strided_rows():
+    g = torch.Generator(device=DEV)
+    g.manual_seed(3)
+    big = (torch.randn((700, 1600), generator=g, device=DEV) * 0.05).to(torch.bfloat16)
+    w = big[:, :1536]
+    assert w.stride(0) == 1600
+    _assert_same(api.nvfp4_quantize_weight(w), _three_launches(w.contiguous(), api.FP8_FP4_MAX))
+
+
+def test_consecutive_calls_reuse_the_workspace():
+    """The grid barrier leaves its arrival count at 0: many calls in a row, on
+    weights of different sizes, each match their own three-launch result."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(11)
+    ws = [(torch.randn(s, generator=g, device=DEV) * sc).to(torch.bfloat16)
+          for s, sc in (((512, 1024), 0.02), ((3, 64), 5.0), ((2048, 5120), 0.01), ((512, 1024), 0.3))]
+    fused = [api.nvfp4_quantize_weight(w) for w in ws for _ in range(2)]
+    torch.cuda.synchronize()
+    for j, f in enumerate(fused):
+        _assert_same(f, _three_launches(ws[j // 2], api.FP8_FP4_MAX))
+    for ws_t in api._WEIGHT_WS.values():
+        assert int(ws_t[:4].view(torch.int32)[0]) == 0
+    assert api.device_status() == 0
+
+
+def test_graph_replay():
+    g = torch.Generator(device=DEV)
+    g.manual_seed(12)
+    w = (torch.randn((1024, 5120), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    q, gs, inv, a = api.nvfp4_quantize_weight(w)  # sets up the workspace outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        out = api.nvfp4_quantize_weight(w)
+    for scale in (0.5, 3.0):
+        w.mul_(scale)
+        graph.replay()
+        torch.cuda.synchronize()
+        _assert_same(out, _three_launches(w, api.FP8_FP4_MAX))
+    assert api.device_status() == 0
+
+
+def test_layer_uses_it():
+    W = _bf16(384, 1024, seed=21)
+    layer = api.NVFP4Linear(up_bf16(W))
+    g_ref = oracle.nvfp4_global_scale(oracle.amax_bf16(W))
+    assert down(layer.gs_w)[0] == g_ref
+    codes, sf = oracle.nvfp4_quantize(W, g_ref)
+    assert np.array_equal(down(layer.weight.codes), codes) and np.array_equal(down(layer.weight.sf), sf)
