@@ -44,6 +44,8 @@ SIGNATURES = {
     "nvfp4_quantize_weight": (_i32, [_vp, _i32, _i64, _i64, _i64, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                      _vp]),
     "bsp_nvfp4_quantize_weight_workspace_bytes": (_i32, [_i32, _vp]),
+    "nvfp4_quantize_weight_static": (_i32, [_vp, _i32, _i64, _i64, _i64, ctypes.c_float, _vp, _vp, _vp, _vp, _vp,
+                                            _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_f16": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_ex": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),

@@ -1091,6 +1091,30 @@ int run_nvfp4_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t l
   return BSP_OK;
 }
 
+// Scratch of nvfp4_quantize_weight_static: a file-scope device array (no
+// allocation by anyone), the header and one word per block for grids of up to
+// kStaticWeightWsBlocks blocks.
+constexpr int64_t kStaticWeightWsBlocks = 4096;
+constexpr int64_t kStaticWeightWsBytes = kWeightWsHeader + 4 * kStaticWeightWsBlocks;
+static __device__ __align__(256) uint8_t g_weight_ws[kStaticWeightWsBytes];
+
+// Its address on device dev.id, looked up once per device; the first call
+// also clears the barrier header on `stream` (the array is zero at module load
+// as well).  Not thread-safe; the first call must come before any stream
+// capture (the symbol lookup may load the module).
+int static_weight_ws(const DeviceInfo& dev, cudaStream_t stream, void** out) {
+  static void* addr[64] = {};
+  if (dev.id < 0 || dev.id >= 64) return BSP_ERR_INVALID_ARG;
+  if (!addr[dev.id]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_weight_ws) != cudaSuccess) return launch_status();
+    if (cudaMemsetAsync(p, 0, kWeightWsHeader, stream) != cudaSuccess) return launch_status();
+    addr[dev.id] = p;
+  }
+  *out = addr[dev.id];
+  return BSP_OK;
+}
+
 }  // namespace
 }  // namespace bsp
 
@@ -1239,6 +1263,26 @@ int nvfp4_quantize_weight(const uint16_t* w, int w_dtype, int64_t N, int64_t K, 
   if (w_dtype != BSP_IN_BF16) return BSP_ERR_INVALID_ARG;
   return run_nvfp4_quantize_weight<InBf16>(w, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf, workspace,
                                            workspace_bytes, stream);
+}
+
+int nvfp4_quantize_weight_static(const uint16_t* w, int w_dtype, int64_t N, int64_t K, int64_t ld_w,
+                                 float fp8_fp4_max, float* amax, float* gs, float* inv_gs, uint8_t* codes, uint8_t* sf,
+                                 bsp_stream_t stream) {
+  if (w_dtype != BSP_IN_BF16 && w_dtype != BSP_IN_F16) return BSP_ERR_INVALID_ARG;
+  // the host checks of nvfp4_quantize_weight, before the set-up touches the device
+  if (N < 0 || K <= 0 || K % 64 != 0 || ld_w < K) return BSP_ERR_INVALID_ARG;
+  if (!(fp8_fp4_max > 0.0f) || !(fp8_fp4_max <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
+  if ((N > 0 && !w) || !codes || !sf || !gs || !inv_gs) return BSP_ERR_INVALID_ARG;
+  int64_t need = 0;
+  int st = bsp_nvfp4_quantize_weight_workspace_bytes(w_dtype, &need);
+  if (st != BSP_OK) return st;
+  if (need > kStaticWeightWsBytes) return BSP_ERR_INVALID_ARG;  // grid larger than the static scratch holds
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != BSP_OK) return st;
+  void* ws = nullptr;
+  if ((st = static_weight_ws(dev, stream, &ws)) != BSP_OK) return st;
+  return nvfp4_quantize_weight(w, w_dtype, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf, ws,
+                               kStaticWeightWsBytes, stream);
 }
 
 int bsp_nvfp4_global_scale(const float* amax, float* gs, float* inv_gs, bsp_stream_t stream) {

@@ -198,6 +198,22 @@ int nvfp4_quantize_weight(const uint16_t *w, int w_dtype, int64_t N, int64_t K, 
  * w_dtype (a header and one word per block of its grid).  Host-only. */
 int bsp_nvfp4_quantize_weight_workspace_bytes(int w_dtype, int64_t *bytes);
 
+/* nvfp4_quantize_weight with no workspace argument and no allocation: its
+ * scratch is a static device array inside the library (16,640 bytes: the
+ * barrier header and one word per block for grids of up to 4096 blocks).  The
+ * pages have no counterpart; it serves callers that can provide neither
+ * scratch memory nor an allocator.  Results are those of
+ * nvfp4_quantize_weight.
+ *   Arguments and errors as nvfp4_quantize_weight, less the workspace; also
+ *   INVALID_ARG if this device's grid needs more scratch than the array holds.
+ * The first call on each device looks up the array's address
+ * (cudaGetSymbolAddress) and clears its barrier header on `stream`; make that
+ * first call before any stream capture.  There is one array per device:
+ * calls that overlap in time (other streams, other host threads) race. */
+int nvfp4_quantize_weight_static(const uint16_t *w, int w_dtype, int64_t N, int64_t K, int64_t ld_w,
+                                 float fp8_fp4_max, float *amax, float *gs, float *inv_gs, uint8_t *codes,
+                                 uint8_t *sf, bsp_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * NVFP4 quantization (nvfp4_config.py: fastvideo_fp4::nvfp4_quantize and
  * _nvfp4_quantize; module docstring: e2m1 elements, group size 16, e4m3

@@ -98,6 +98,11 @@ def test_host_validation_rejects_bad_arguments():
     assert qw(p, 0, 4, 64, 68, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_ALIGNMENT  # ld % 8
     assert L.bsp_nvfp4_quantize_weight_workspace_bytes(0, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_nvfp4_quantize_weight_workspace_bytes(5, p) == nat.BSP_ERR_INVALID_ARG
+    qs = L.nvfp4_quantize_weight_static
+    assert qs(p, 0, 4, 48, 48, 2688.0, None, p, p, p, p, None) == nat.BSP_ERR_INVALID_ARG  # K % 64
+    assert qs(p, 3, 4, 64, 64, 2688.0, None, p, p, p, p, None) == nat.BSP_ERR_INVALID_ARG  # dtype
+    assert qs(p, 0, 4, 64, 64, float("inf"), None, p, p, p, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert qs(p, 0, 4, 64, 64, 2688.0, None, None, p, p, p, None) == nat.BSP_ERR_INVALID_ARG  # no gs
 
 
 def test_no_gpu_means_an_error_not_a_fallback():
