@@ -135,13 +135,38 @@ __device__ __forceinline__ float global_scale_from_mag(uint32_t mag) {
   return mag == 0u ? 1.0f : __fdiv_rn(2688.0f, In::value(mag));
 }
 
-// NVFP4 scale byte and reciprocal of one group with amax bit pattern `mag`.
+// fl32(x / 6) for x a bf16 or fp16 magnitude: the product with fl32(1/6),
+// corrected once by the fma residual.  For 0 and every positive finite bf16 and
+// fp16 value this equals the correctly rounded quotient (checked exhaustively
+// against exact rationals); +inf (the amax of a group holding an infinity)
+// gives +inf.
+__device__ __forceinline__ float div6_rn(float x) {
+  constexpr float kSixth = 0x1.555556p-3f;  // fl32(1/6)
+  const float q = __fmul_rn(x, kSixth);
+  const float c = __fmaf_rn(__fmaf_rn(-q, 6.0f, x), kSixth, q);
+  return x == __int_as_float(0x7F800000) ? x : c;
+}
+
+// fl32(gs / e4m3(b)) for every scale byte b (0 for b = 0): the decode factor
+// of a per-tensor scale, built once per block so that a group looks it up
+// instead of dividing.  Ends with a block barrier.  Used by the kernels whose
+// time is instruction issue rather than DRAM (the fused RMSNorm ones and the
+// short-row one); in the K % 64 streaming kernels it measured slower.
+__device__ __forceinline__ void build_inv_table(float* tab, float gs) {
+  for (uint32_t i = threadIdx.x; i < 256u; i += blockDim.x)
+    tab[i] = i == 0u ? 0.0f : __fdiv_rn(gs, e4m3_pos_to_f32(i));
+  __syncthreads();
+}
+
+// NVFP4 scale byte and reciprocal of one group with amax bit pattern `mag`
+// (inv_tab: build_inv_table(gs), or NULL to divide).
 template <class In>
-__device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sfb, float& inv) {
+__device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sfb, float& inv,
+                                            const float* inv_tab = nullptr) {
   const float amax = In::value(mag);
-  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+  const float s = __fmul_rn(div6_rn(amax), gs);
   sfb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
-  inv = (sfb == 0u) ? 0.0f : __fdiv_rn(gs, e4m3_pos_to_f32(sfb));
+  inv = inv_tab ? inv_tab[sfb] : ((sfb == 0u) ? 0.0f : __fdiv_rn(gs, e4m3_pos_to_f32(sfb)));
 }
 
 // Eight elements (one 16-byte chunk) times inv -> eight e2m1 codes in one
@@ -207,7 +232,7 @@ __device__ __forceinline__ float row_scale_pass(const uint16_t* __restrict__ row
 // the first step.
 template <class In, class L, int U>
 __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uint8_t* sp, bool live, float gs,
-                                            bool store_sf) {
+                                            bool store_sf, const float* inv_tab) {
   uint4 v[U][2];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
@@ -218,7 +243,7 @@ __device__ __forceinline__ void nvfp4_steps(const uint16_t* lp, uint8_t* cp, uin
   for (int u = 0; u < U; ++u) {
     uint32_t sfb;
     float inv;
-    nvfp4_scale<In>(group_mag16<In>(v[u][0], v[u][1]), gs, sfb, inv);
+    nvfp4_scale<In>(group_mag16<In>(v[u][0], v[u][1]), gs, sfb, inv, inv_tab);
     uint2 w;
     w.x = nvfp4_codes8<In>(v[u][0], inv);
     w.y = nvfp4_codes8<In>(v[u][1], inv);
@@ -244,6 +269,8 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs = __ldg(gs_ptr);
   const bool quad_lead = (lane & 3u) == 0u;
+  __shared__ float inv_tab[256];
+  build_inv_table(inv_tab, gs);
   for (int64_t r0 = 2 * warp; r0 < Mp; r0 += 2 * nwarps) {
     uint4 v[2][S][2];
 #pragma unroll
@@ -268,7 +295,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_quant_short_kernel(
       for (int st = 0; st < S; ++st) {
         uint32_t sfb;
         float inv;
-        nvfp4_scale<In>(group_mag16<In>(v[h][st][0], v[h][st][1]), gs, sfb, inv);
+        nvfp4_scale<In>(group_mag16<In>(v[h][st][0], v[h][st][1]), gs, sfb, inv, inv_tab);
         uint2 w;
         w.x = nvfp4_codes8<In>(v[h][st][0], inv);
         w.y = nvfp4_codes8<In>(v[h][st][1], inv);
@@ -363,7 +390,8 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
 // tensor (live false) only writes its zero scale bytes.
 template <class In, class L, int U = kUnroll>
 __device__ __forceinline__ void nvfp4_row_k64(const uint16_t* row, int64_t K, int64_t r, bool live, float gs,
-                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, uint32_t lane) {
+                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, uint32_t lane,
+                                              const float* inv_tab) {
   const int64_t groups = K >> 4;
   const int64_t steps = groups >> 5;  // full warp steps (32 groups) per row
   const int64_t rem = groups & 31;    // groups of a last, partial step (a multiple of 4)
@@ -374,13 +402,13 @@ __device__ __forceinline__ void nvfp4_row_k64(const uint16_t* row, int64_t K, in
   constexpr int kStepSf = 8 * L::kTileBytes;  // a warp step covers 8 scale tiles
   int64_t st = 0;
   for (; st + U <= steps; st += U)
-    nvfp4_steps<In, L, U>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
+    nvfp4_steps<In, L, U>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead, inv_tab);
   for (; st < steps; ++st)
-    nvfp4_steps<In, L, 1>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead);
+    nvfp4_steps<In, L, 1>(lp + st * 512, cp + st * 256, sp + st * kStepSf, live, gs, quad_lead, inv_tab);
   if (rem) {
     const bool in = lane < rem;  // groups beyond the row end are predicated off
     nvfp4_steps<In, L, 1>(in ? lp + st * 512 : lp, in ? cp + st * 256 : cp, in ? sp + st * kStepSf : sp, live && in,
-                          gs, in && quad_lead);
+                          gs, in && quad_lead, inv_tab);
   }
 }
 
@@ -399,7 +427,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_k64_kernel(
     const uint16_t* row = x + r * ld_x;
     float gs = gs_tensor;
     if (kPerRow && live) gs = row_scale_pass<In>(row, K, r, row_gs, row_inv);
-    nvfp4_row_k64<In, L>(row, K, r, live, gs, codes, sf, lane);
+    nvfp4_row_k64<In, L>(row, K, r, live, gs, codes, sf, lane, nullptr);
   }
 }
 
@@ -499,6 +527,8 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+  __shared__ float inv_tab[256];
+  if constexpr (!kPerRow) build_inv_table(inv_tab, gs_tensor);
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const int64_t sfb_row = L::row_base(r, cols4 >> 2);
@@ -535,7 +565,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
         const uint4 y0 = rmsnorm8(ldg16(row + c * 16), ldg16(gamma + c * 16), rstd);
         const uint4 y1 = rmsnorm8(ldg16(row + c * 16 + 8), ldg16(gamma + c * 16 + 8), rstd);
         float inv;
-        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv);
+        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, kPerRow ? nullptr : inv_tab);
         uint2 w;
         w.x = nvfp4_codes8<InBf16>(y0, inv);
         w.y = nvfp4_codes8<InBf16>(y1, inv);
@@ -570,6 +600,8 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+  __shared__ float inv_tab[256];
+  if constexpr (!kPerRow) build_inv_table(inv_tab, gs_tensor);
   const bool quad_lead = (lane & 3u) == 0u;
   const uint16_t* gp = gamma + lane * 16;  // re-read per row from L1 (registers go to rows in flight)
   for (int64_t r0 = R * warp; r0 < Mp; r0 += R * nwarps) {
@@ -621,7 +653,7 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant
         const uint4 y1 = rmsnorm8(v[h][s][1], ldg16(gp + s * 512 + 8), rs);
         uint32_t sfb;
         float inv;
-        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv);
+        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, kPerRow ? nullptr : inv_tab);
         uint2 w;
         w.x = nvfp4_codes8<InBf16>(y0, inv);
         w.y = nvfp4_codes8<InBf16>(y1, inv);
@@ -921,7 +953,8 @@ __global__ void __launch_bounds__(kQuantThreads, BSP_WQ_MIN_BLOCKS) nvfp4_weight
   for (int64_t i = warp; i < Np; i += nwarps) {
     const int64_t r = Np - 1 - i;
     const bool live = r < N;
-    nvfp4_row_k64<In, Sf128x4, BSP_WQ_ROW_STEPS>(w + (live ? r : 0) * ld_w, K, r, live, gs, codes, sf, lane);
+    nvfp4_row_k64<In, Sf128x4, BSP_WQ_ROW_STEPS>(w + (live ? r : 0) * ld_w, K, r, live, gs, codes, sf, lane,
+                                                 nullptr);
   }
 }
 
