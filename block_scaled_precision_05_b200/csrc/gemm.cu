@@ -87,10 +87,11 @@ enum Kind : int { kNVF4 = 0, kMXF8 = 1 };
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
-template <int KIND>
+template <int KIND, int BN_ = 256>
 struct Cfg {
   static constexpr int BM = 128;                        // accumulator rows (tensor-memory lanes)
-  static constexpr int BN = 256;                        // output tile columns
+  static constexpr int BN = BN_;                        // output tile columns (256, or 128 for few tiles)
+  static_assert(BN == 256 || BN == 128, "tile width");
   static constexpr int ROW_BYTES = KIND == kNVF4 ? BSP_GEMM_NVF4_ROW_BYTES : 128;  // K bytes per row per stage
   static constexpr int MMAS = ROW_BYTES / 32;                                    // per stage, 32 bytes of K each
   static constexpr int ATOMS = KIND == kNVF4 ? ROW_BYTES / 32 : 1;  // 128x4 scale tiles per 128 rows per stage
@@ -158,12 +159,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int KIND>
-__global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
+template <int KIND, int BN>
+__global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                             const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-  using C = Cfg<KIND>;
+  using C = Cfg<KIND, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
@@ -919,11 +920,11 @@ int encode_output(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
 
-template <int KIND>
+template <int KIND, int BN>
 int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                 int64_t row_bytes, int64_t tiles_per_band, const CUtensorMap& tmD, GemmParams p,
                 cudaStream_t stream) {
-  using C = Cfg<KIND>;
+  using C = Cfg<KIND, BN>;
   CUtensorMap tmA, tmB, tmSFA, tmSFB;
   int st;
   if ((st = encode_operand(&tmA, A, p.M, row_bytes, C::BM, C::ROW_BYTES)) != BSP_OK) return st;
@@ -932,7 +933,7 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
   if ((st = encode_scales(&tmSFB, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, C::B_BANDS)) != BSP_OK)
     return st;
   p.num_kb = static_cast<int>(ceil_div(row_bytes, C::ROW_BYTES));
-  auto kernel = blockscaled_gemm_kernel<KIND>;
+  auto kernel = blockscaled_gemm_kernel<KIND, BN>;
   static bool attr_set[64] = {};
   if (!attr_set[dev.id]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
@@ -1031,7 +1032,11 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
     if (M <= 64) return launch_skinny<KIND, 64>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
     return launch_skinny<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
   }
-  return launch_gemm<KIND>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
+  // 128-column tiles when they still fit in one wave: twice the CTAs stream B
+  // (for small M the weight stream, not the tensor pipe, sets the time)
+  if (ceil_div(M, 128) * ceil_div(N, 128) <= dev.sm_count)
+    return launch_gemm<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
+  return launch_gemm<KIND, 256>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
 }
 
 }  // namespace
