@@ -58,13 +58,38 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(src: str) -> str:
+    """C/CUDA source without comments and with whitespace runs collapsed, so
+    that an edit of comments alone keeps the hash of the kernels."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif src[i] == '"':  # string literal: kept as is
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash() -> str:
+    """Identifies the kernel sources (csrc/*.cu, *.cuh, *.h; comments and
+    layout ignored) that a committed ncu capture was taken on."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "block_scaled_precision_05_b200", "csrc")
     for name in sorted(os.listdir(cdir)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(cdir, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(cdir, name), encoding="utf-8") as f:
+                h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -35,9 +35,12 @@
 //   (roles by warp index: 0 producer, 1 MMA, 2-9 epilogue, 10-13 scales)
 // Output tiles are 128 x 256 with one accumulator (256 tensor-memory
 // columns): two accumulators of 256 columns would leave no room for the stages'
-// scale factors, and 128-column tiles measured slower (an N = 128 block-scaled
-// MMA takes about as long to issue as an N = 256 one), so the next tile's MMAs
-// wait until the epilogue has read the accumulator, which it does first thing.
+// scale factors, and 128-column tiles with two accumulators measured slower (an
+// N = 128 block-scaled MMA takes about as long to issue as an N = 256 one), so
+// the next tile's MMAs wait until the epilogue has read the accumulator, which
+// it does first thing.  When the 128 x 128 tiles of a GEMM fit in one wave
+// (small M), the kernel is instantiated with BN = 128: twice the CTAs then
+// stream the weight, which sets the time there.
 // Tensor memory: the accumulator; then, per pipeline stage, the stage's
 // scale factors (a scale column may only be rewritten once the stage's MMAs
 // have completed, which the stage's empty barrier already guarantees).
@@ -528,12 +531,12 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Skinny M (M <= 128, e.g. per-token decode-like batches against a large
-// weight): the GEMM is bound by streaming the weight from HBM, so it is run
-// transposed, D^T = B A^T.  The weight is the MMA's 128-row operand (tiles of
-// 128 weight rows, so ~N/128 CTAs stream disjoint weight panels through a deep
-// pipeline of small stages) and the BNA <= 128 activation rows are the MMA's N
-// side.  Same roles as the main kernel: warp 0 producer, warp 1 MMA issuer,
+// Skinny M (M <= BSP_GEMM_SKINNY_MAX_M, and M <= 64 with 8x4 activation
+// scales; e.g. per-token decode-like batches against a large weight): the GEMM
+// is bound by streaming the weight from HBM, so it is run transposed,
+// D^T = B A^T.  The weight is the MMA's 128-row operand (tiles of 128 weight
+// rows, so ~N/128 CTAs stream disjoint weight panels through a deep pipeline of
+// small stages) and the BNA <= 128 activation rows are the MMA's N side.  Same roles as the main kernel: warp 0 producer, warp 1 MMA issuer,
 // warps 2-5 scale factors, warps 6-9 epilogue (lane = output column n, one
 // TMEM column per activation row m; each warp writes 32 consecutive n of a
 // row of D per instruction).
