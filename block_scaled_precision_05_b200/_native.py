@@ -27,6 +27,14 @@ BSP_SF_LAYOUT_8X4 = 1
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 
+BSP_WEIGHT_BATCH_MAX = 256
+
+
+class BspWeightDesc(ctypes.Structure):
+    """bsp_weight_desc of include/bsp.h (one weight of nvfp4_quantize_weights)."""
+    _fields_ = [("w", _vp), ("N", _i64), ("K", _i64), ("ld_w", _i64), ("amax", _vp), ("gs", _vp), ("inv_gs", _vp),
+                ("codes", _vp), ("sf", _vp)]
+
 # name -> (restype, argtypes), one entry per function declared in include/bsp.h
 SIGNATURES = {
     "bsp_status_string": (ctypes.c_char_p, [_i32]),
@@ -46,6 +54,7 @@ SIGNATURES = {
     "bsp_nvfp4_quantize_weight_workspace_bytes": (_i32, [_i32, _vp]),
     "nvfp4_quantize_weight_static": (_i32, [_vp, _i32, _i64, _i64, _i64, ctypes.c_float, _vp, _vp, _vp, _vp, _vp,
                                             _vp]),
+    "nvfp4_quantize_weights": (_i32, [_vp, _i32, _i32, ctypes.c_float, _vp, _i64, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_f16": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_ex": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),

@@ -251,6 +251,46 @@ def nvfp4_quantize_weight(w: torch.Tensor, fp8_fp4_max: float = FP8_FP4_MAX, out
     return out, gs, inv, am
 
 
+def nvfp4_quantize_weights(weights, fp8_fp4_max: float = FP8_FP4_MAX):
+    """nvfp4_quantize_weight for a list of [N, K] weights of one dtype (K % 64
+    == 0), up to BSP_WEIGHT_BATCH_MAX per launch: the load-time conversion of a
+    model's linears in one cooperative launch per chunk.  Returns one
+    (NVFP4Tensor, gs, 1/gs, amax) per weight, bit-identical to
+    nvfp4_quantize_weight on it."""
+    ws_in = []
+    for w in weights:
+        _require_cuda(w)
+        w = coerce_input(w)
+        if w.dim() != 2 or w.shape[1] % 64 != 0:
+            raise ValueError(f"nvfp4_quantize_weights expects [N, K] weights with K % 64 == 0, got {tuple(w.shape)}")
+        ws_in.append(w if w.stride(1) == 1 else w.contiguous())
+    if not ws_in:
+        return []
+    dtypes = {w.dtype for w in ws_in}
+    devices = {w.device for w in ws_in}
+    if len(dtypes) != 1 or len(devices) != 1:
+        raise ValueError("nvfp4_quantize_weights expects weights of one dtype on one device")
+    dev = ws_in[0].device
+    w_dtype = nat.BSP_IN_F16 if ws_in[0].dtype == torch.float16 else nat.BSP_IN_BF16
+    work = _weight_workspace(dev, w_dtype)
+    results = []
+    for c0 in range(0, len(ws_in), nat.BSP_WEIGHT_BATCH_MAX):
+        chunk = ws_in[c0:c0 + nat.BSP_WEIGHT_BATCH_MAX]
+        descs = (nat.BspWeightDesc * len(chunk))()
+        for d, w in zip(descs, chunk):
+            N, K = w.shape
+            q = NVFP4Tensor(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                            torch.empty(nvfp4_sf_bytes(N, K), dtype=torch.uint8, device=dev), K)
+            gs, inv, am = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(3))
+            d.w, d.N, d.K, d.ld_w = w.data_ptr(), N, K, w.stride(0)
+            d.amax, d.gs, d.inv_gs, d.codes, d.sf = am.data_ptr(), gs.data_ptr(), inv.data_ptr(), \
+                q.codes.data_ptr(), q.sf.data_ptr()
+            results.append((q, gs, inv, am))
+        nat.check(nat.lib().nvfp4_quantize_weights(ctypes.addressof(descs), len(chunk), w_dtype, float(fp8_fp4_max),
+                                                   _ptr(work), work.numel(), _stream()), "nvfp4_quantize_weights")
+    return results
+
+
 def nvfp4_rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
                            global_sf: torch.Tensor | None = None, per_row: bool = False,
                            out: NVFP4Tensor | None = None, rstd_out: torch.Tensor | None = None) -> NVFP4Tensor:

@@ -841,6 +841,7 @@ __global__ void global_scale_kernel(const float* __restrict__ amax, float fp8_fp
 // kWeightWsHeader.
 // ---------------------------------------------------------------------------
 constexpr int64_t kWeightWsHeader = 256;
+constexpr int kWeightBatchMax = BSP_WEIGHT_BATCH_MAX;  // weights per nvfp4_quantize_weights call
 #ifndef BSP_WQ_AMAX_LOADS
 #define BSP_WQ_AMAX_LOADS 8  // 16-byte loads in flight per thread in the amax phase
 #endif
@@ -900,20 +901,14 @@ __device__ __forceinline__ uint32_t block_max(uint32_t m) {
   return warp_max(m);
 }
 
+// Phase 1: this block's max|w| (sanitized magnitudes as in amax_kernel), the
+// block's threads striding over the whole grid's share.
 template <class In>
-__global__ void __launch_bounds__(kQuantThreads, BSP_WQ_MIN_BLOCKS) nvfp4_weight_kernel(
-    const uint16_t* __restrict__ w, int64_t N, int64_t Np, int64_t K, int64_t ld_w, float fp8_fp4_max,
-    float* __restrict__ amax_out, float* __restrict__ gs_out, float* __restrict__ inv_out, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ sf, uint8_t* __restrict__ ws, uint32_t* __restrict__ err) {
-  uint32_t* count = reinterpret_cast<uint32_t*>(ws);
-  uint32_t* gen = count + 1;
-  uint32_t* part = reinterpret_cast<uint32_t*>(ws + kWeightWsHeader);
+__device__ __forceinline__ uint32_t weight_block_amax(const uint16_t* __restrict__ w, int64_t N, int64_t K,
+                                                      int64_t ld_w) {
   const uint32_t lane = lane_id();
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t warp = tid >> 5, nwarps = nthreads >> 5;
-
-  // 1. max|w| (sanitized magnitudes as in amax_kernel)
   uint32_t m = 0;
   if (ld_w == K) {
     constexpr int A = BSP_WQ_AMAX_LOADS;
@@ -928,17 +923,18 @@ __global__ void __launch_bounds__(kQuantThreads, BSP_WQ_MIN_BLOCKS) nvfp4_weight
     }
     for (; i < nvec; i += nthreads) m = max(m, max_sane_mag8<In>(ldg16(w + i * 8)));
   } else {
-    for (int64_t r = warp; r < N; r += nwarps)
+    for (int64_t r = tid >> 5; r < N; r += nthreads >> 5)
       for (int64_t c = lane * 8; c < K; c += 256) m = max(m, max_sane_mag8<In>(ldg16(w + r * ld_w + c)));
   }
-  m = block_max(m);
-  if (threadIdx.x == 0) part[blockIdx.x] = m;
+  return block_max(m);
+}
 
-  // 2.
-  if (!grid_barrier(count, gen, gridDim.x, err)) return;
-
-  // 3. (the words are read through L2: other SMs wrote them)
-  m = 0;
+// Phase 3: amax from the blocks' words (read through L2: other SMs wrote
+// them) and gs exactly as bsp_nvfp4_global_scale_max; block 0 stores them.
+template <class In>
+__device__ __forceinline__ float weight_global_scale(const uint32_t* part, float fp8_fp4_max, float* amax_out,
+                                                     float* gs_out, float* inv_out) {
+  uint32_t m = 0;
   for (int64_t i = threadIdx.x; i < gridDim.x; i += blockDim.x) m = max(m, __ldcg(part + i));
   m = block_max(m);
   const float amax = m == 0u ? 0.0f : In::value(m);
@@ -948,13 +944,61 @@ __global__ void __launch_bounds__(kQuantThreads, BSP_WQ_MIN_BLOCKS) nvfp4_weight
     if (gs_out) *gs_out = gs;
     if (inv_out) *inv_out = __fdiv_rn(1.0f, gs);
   }
+  return gs;
+}
 
-  // 4.
-  for (int64_t i = warp; i < Np; i += nwarps) {
+// Phase 4: the rows, last row first, one warp per row.
+template <class In>
+__device__ __forceinline__ void weight_rows(const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ld_w,
+                                            float gs, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  const int64_t Np = (N + 127) / 128 * 128;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < Np; i += nwarps) {
     const int64_t r = Np - 1 - i;
     const bool live = r < N;
-    nvfp4_row_k64<In, Sf128x4, BSP_WQ_ROW_STEPS>(w + (live ? r : 0) * ld_w, K, r, live, gs, codes, sf, lane,
+    nvfp4_row_k64<In, Sf128x4, BSP_WQ_ROW_STEPS>(w + (live ? r : 0) * ld_w, K, r, live, gs, codes, sf, lane_id(),
                                                  nullptr);
+  }
+}
+
+template <class In>
+__global__ void __launch_bounds__(kQuantThreads, BSP_WQ_MIN_BLOCKS) nvfp4_weight_kernel(
+    const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ld_w, float fp8_fp4_max,
+    float* __restrict__ amax_out, float* __restrict__ gs_out, float* __restrict__ inv_out, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ sf, uint8_t* __restrict__ ws, uint32_t* __restrict__ err) {
+  uint32_t* count = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* part = reinterpret_cast<uint32_t*>(ws + kWeightWsHeader);
+  const uint32_t m = weight_block_amax<In>(w, N, K, ld_w);                      // 1.
+  if (threadIdx.x == 0) part[blockIdx.x] = m;
+  if (!grid_barrier(count, count + 1, gridDim.x, err)) return;                  // 2.
+  const float gs = weight_global_scale<In>(part, fp8_fp4_max, amax_out, gs_out, inv_out);  // 3.
+  weight_rows<In>(w, N, K, ld_w, gs, codes, sf);                                 // 4.
+}
+
+// Many weights in one launch: the phases of nvfp4_weight_kernel per weight,
+// one grid barrier each.  A block that has quantized its rows of weight j goes
+// on to the amax of weight j + 1 while others finish, so one weight's tail
+// overlaps the next one's reads.  The blocks' words alternate between two
+// slots: slot j % 2 is rewritten (for weight j + 2) only after the barrier of
+// weight j + 1, which every block passes after reading it.
+struct WeightBatch {
+  int count;
+  bsp_weight_desc d[kWeightBatchMax];
+};
+
+template <class In>
+__global__ void __launch_bounds__(kQuantThreads, 3) nvfp4_weights_kernel(
+    const __grid_constant__ WeightBatch batch, float fp8_fp4_max, uint8_t* __restrict__ ws, uint32_t* __restrict__ err) {
+  uint32_t* count = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* part = reinterpret_cast<uint32_t*>(ws + kWeightWsHeader);
+  for (int j = 0; j < batch.count; ++j) {
+    const bsp_weight_desc& d = batch.d[j];
+    uint32_t* slot = part + (j & 1) * gridDim.x;
+    const uint32_t m = weight_block_amax<In>(d.w, d.N, d.K, d.ld_w);
+    if (threadIdx.x == 0) slot[blockIdx.x] = m;
+    if (!grid_barrier(count, count + 1, gridDim.x, err)) return;
+    const float gs = weight_global_scale<In>(slot, fp8_fp4_max, d.amax, d.gs, d.inv_gs);
+    weight_rows<In>(d.w, d.N, d.K, d.ld_w, gs, d.codes, d.sf);
   }
 }
 
@@ -1083,11 +1127,15 @@ int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, co
 template <class In>
 int weight_grid(const DeviceInfo& dev, int* grid) {
   int per_sm = 0;
+  int per_sm_batch = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_weight_kernel<In>, kQuantThreads, 0) !=
           cudaSuccess ||
-      per_sm < 1)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_batch, nvfp4_weights_kernel<In>, kQuantThreads, 0) !=
+          cudaSuccess ||
+      per_sm < 1 || per_sm_batch < 1)
     return (cudaGetLastError(), BSP_ERR_CUDA);
-  *grid = dev.sm_count * per_sm;
+  // one grid for both kernels (they share the workspace layout): the smaller residency
+  *grid = dev.sm_count * (per_sm < per_sm_batch ? per_sm : per_sm_batch);
   return BSP_OK;
 }
 
@@ -1107,7 +1155,7 @@ int run_nvfp4_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t l
   if (st != BSP_OK) return st;
   int grid = 0;
   if ((st = weight_grid<In>(dev, &grid)) != BSP_OK) return st;
-  if (ws_bytes < kWeightWsHeader + 4 * static_cast<int64_t>(grid)) return BSP_ERR_INVALID_ARG;
+  if (ws_bytes < kWeightWsHeader + 4 * static_cast<int64_t>(grid)) return BSP_ERR_INVALID_ARG;  // one slot used here
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -1117,9 +1165,48 @@ int run_nvfp4_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t l
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const int64_t Np = round_up(N, 128);
-  if (cudaLaunchKernelEx(&cfg, nvfp4_weight_kernel<In>, w, N, Np, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf,
+  if (cudaLaunchKernelEx(&cfg, nvfp4_weight_kernel<In>, w, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf,
                          static_cast<uint8_t*>(ws), dev.err_word) != cudaSuccess)
+    return launch_status();
+  return BSP_OK;
+}
+
+template <class In>
+int run_nvfp4_quantize_weights(const bsp_weight_desc* descs, int count, float fp8_fp4_max, void* ws, int64_t ws_bytes,
+                               cudaStream_t stream) {
+  if (count < 0 || count > kWeightBatchMax || (count > 0 && !descs) || !ws) return BSP_ERR_INVALID_ARG;
+  if (!(fp8_fp4_max > 0.0f) || !(fp8_fp4_max <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
+  WeightBatch batch;
+  batch.count = count;
+  for (int j = 0; j < count; ++j) {
+    const bsp_weight_desc& d = descs[j];
+    if (d.N < 0 || d.K <= 0 || d.K % 64 != 0 || d.ld_w < d.K) return BSP_ERR_INVALID_ARG;
+    if ((d.N > 0 && !d.w) || !d.codes || !d.sf || !d.gs || !d.inv_gs) return BSP_ERR_INVALID_ARG;
+    if ((d.w && !aligned16(d.w)) || !aligned16(d.codes) || !aligned16(d.sf) || d.ld_w % 8 != 0 ||
+        (reinterpret_cast<uintptr_t>(d.gs) & 3u) || (reinterpret_cast<uintptr_t>(d.inv_gs) & 3u) ||
+        (reinterpret_cast<uintptr_t>(d.amax) & 3u))
+      return BSP_ERR_ALIGNMENT;
+    batch.d[j] = d;
+  }
+  if (!aligned16(ws)) return BSP_ERR_ALIGNMENT;
+  if (count == 0) return BSP_OK;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  int grid = 0;
+  if ((st = weight_grid<In>(dev, &grid)) != BSP_OK) return st;
+  if (ws_bytes < kWeightWsHeader + 8 * static_cast<int64_t>(grid)) return BSP_ERR_INVALID_ARG;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeCooperative;  // all blocks resident at once, or no launch
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, nvfp4_weights_kernel<In>, batch, fp8_fp4_max, static_cast<uint8_t*>(ws),
+                         dev.err_word) != cudaSuccess)
     return launch_status();
   return BSP_OK;
 }
@@ -1283,7 +1370,7 @@ int bsp_nvfp4_quantize_weight_workspace_bytes(int w_dtype, int64_t* bytes) {
   int grid = 0;
   st = w_dtype == BSP_IN_F16 ? weight_grid<InF16>(dev, &grid) : weight_grid<InBf16>(dev, &grid);
   if (st != BSP_OK) return st;
-  *bytes = kWeightWsHeader + 4 * static_cast<int64_t>(grid);
+  *bytes = kWeightWsHeader + 8 * static_cast<int64_t>(grid);  // two slots: enough for nvfp4_quantize_weights too
   return BSP_OK;
 }
 
@@ -1316,6 +1403,14 @@ int nvfp4_quantize_weight_static(const uint16_t* w, int w_dtype, int64_t N, int6
   if ((st = static_weight_ws(dev, stream, &ws)) != BSP_OK) return st;
   return nvfp4_quantize_weight(w, w_dtype, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf, ws,
                                kStaticWeightWsBytes, stream);
+}
+
+int nvfp4_quantize_weights(const bsp_weight_desc* descs, int count, int w_dtype, float fp8_fp4_max, void* workspace,
+                           int64_t workspace_bytes, bsp_stream_t stream) {
+  if (w_dtype == BSP_IN_F16)
+    return run_nvfp4_quantize_weights<InF16>(descs, count, fp8_fp4_max, workspace, workspace_bytes, stream);
+  if (w_dtype != BSP_IN_BF16) return BSP_ERR_INVALID_ARG;
+  return run_nvfp4_quantize_weights<InBf16>(descs, count, fp8_fp4_max, workspace, workspace_bytes, stream);
 }
 
 int bsp_nvfp4_global_scale(const float* amax, float* gs, float* inv_gs, bsp_stream_t stream) {

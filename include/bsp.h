@@ -194,9 +194,39 @@ int nvfp4_quantize_weight(const uint16_t *w, int w_dtype, int64_t N, int64_t K, 
                           float *amax, float *gs, float *inv_gs, uint8_t *codes, uint8_t *sf, void *workspace,
                           int64_t workspace_bytes, bsp_stream_t stream);
 
-/* Workspace bytes nvfp4_quantize_weight needs on the current device for
- * w_dtype (a header and one word per block of its grid).  Host-only. */
+/* Workspace bytes nvfp4_quantize_weight and nvfp4_quantize_weights need on
+ * the current device for w_dtype (a 256-byte header and two words per block of
+ * their grid).  Host-only. */
 int bsp_nvfp4_quantize_weight_workspace_bytes(int w_dtype, int64_t *bytes);
+
+/* One weight of an nvfp4_quantize_weights call: the arguments of
+ * nvfp4_quantize_weight that differ from weight to weight (all device
+ * pointers; amax may be NULL). */
+#define BSP_WEIGHT_BATCH_MAX 256
+typedef struct bsp_weight_desc {
+    const uint16_t *w;       /* [N, K], row stride ld_w elements, 16-byte aligned */
+    int64_t N, K, ld_w;      /* N >= 0, K % 64 == 0, ld_w >= K, ld_w % 8 == 0 */
+    float *amax, *gs, *inv_gs;
+    uint8_t *codes, *sf;
+} bsp_weight_desc;
+
+/* nvfp4_quantize_weight for up to BSP_WEIGHT_BATCH_MAX weights of one input
+ * format and one fp8_fp4_max in a single cooperative launch: per weight the
+ * amax, a grid barrier, gs and the quantization, with one weight's last rows
+ * overlapping the next weight's amax reads (the load-time conversion of a
+ * model's linears, nvfp4_qat_config.py convert_model_to_fp4, as one call).
+ * Results are bit-identical to nvfp4_quantize_weight on each weight.
+ *   descs    : HOST array of count descriptors (copied into the launch; the
+ *              caller may reuse it as soon as the call returns)
+ *   count    : 0 .. BSP_WEIGHT_BATCH_MAX (0: nothing launched)
+ *   workspace: as nvfp4_quantize_weight (its size from
+ *              bsp_nvfp4_quantize_weight_workspace_bytes; the two entries may
+ *              share one workspace if their calls do not overlap in time)
+ * Errors: INVALID_ARG or ALIGNMENT for any descriptor as nvfp4_quantize_weight
+ * (nothing launched), CUDA if the launch fails; a barrier wait that runs out
+ * raises the device error word. */
+int nvfp4_quantize_weights(const bsp_weight_desc *descs, int count, int w_dtype, float fp8_fp4_max, void *workspace,
+                           int64_t workspace_bytes, bsp_stream_t stream);
 
 /* nvfp4_quantize_weight with no workspace argument and no allocation: its
  * scratch is a static device array inside the library (16,640 bytes: the

@@ -98,6 +98,22 @@ def test_host_validation_rejects_bad_arguments():
     assert qw(p, 0, 4, 64, 68, 2688.0, None, p, p, p, p, p, 1 << 20, None) == nat.BSP_ERR_ALIGNMENT  # ld % 8
     assert L.bsp_nvfp4_quantize_weight_workspace_bytes(0, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_nvfp4_quantize_weight_workspace_bytes(5, p) == nat.BSP_ERR_INVALID_ARG
+    qb = L.nvfp4_quantize_weights
+    descs = (nat.BspWeightDesc * 2)()
+    for d in descs:
+        d.w, d.N, d.K, d.ld_w, d.gs, d.inv_gs, d.codes, d.sf = 0x10000, 4, 64, 64, 0x10000, 0x10000, 0x10000, 0x10000
+    da = ctypes.addressof(descs)
+    assert qb(da, nat.BSP_WEIGHT_BATCH_MAX + 1, 0, 2688.0, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # count
+    assert qb(da, -1, 0, 2688.0, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG
+    assert qb(None, 2, 0, 2688.0, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG
+    assert qb(da, 2, 2, 2688.0, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # dtype
+    assert qb(da, 2, 0, 0.0, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG
+    assert qb(da, 2, 0, 2688.0, None, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # no workspace
+    assert qb(da, 0, 0, 2688.0, p, 1 << 20, None) == nat.BSP_OK  # empty batch: nothing launched
+    descs[1].K = 48
+    assert qb(da, 2, 0, 2688.0, p, 1 << 20, None) == nat.BSP_ERR_INVALID_ARG  # K % 64 of the second weight
+    descs[1].K, descs[1].w = 64, 0x10008
+    assert qb(da, 2, 0, 2688.0, p, 1 << 20, None) == nat.BSP_ERR_ALIGNMENT
     qs = L.nvfp4_quantize_weight_static
     assert qs(p, 0, 4, 48, 48, 2688.0, None, p, p, p, p, None) == nat.BSP_ERR_INVALID_ARG  # K % 64
     assert qs(p, 3, 4, 64, 64, 2688.0, None, p, p, p, p, None) == nat.BSP_ERR_INVALID_ARG  # dtype

@@ -1,4 +1,5 @@
-"""Load-time weight conversion in one kernel (nvfp4_quantize_weight) on the GPU.
+"""Load-time weight conversion in one kernel (nvfp4_quantize_weight, and
+nvfp4_quantize_weights for many weights in one launch) on the GPU.
 
 The entry fuses the weight path of sgl-project sglang nvfp4_online.py
 (_quantize_weight_nvfp4: amax, gs = e4m3_max * 6 / amax, quantize) into one
@@ -141,3 +142,54 @@ def test_layer_uses_it():
     assert down(layer.gs_w)[0] == g_ref
     codes, sf = oracle.nvfp4_quantize(W, g_ref)
     assert np.array_equal(down(layer.weight.codes), codes) and np.array_equal(down(layer.weight.sf), sf)
+
+
+def test_batch_matches_single_launches():
+    """nvfp4_quantize_weights: one launch over mixed weights (ragged, L2-sized,
+    larger than L2, a strided view, an all-zero weight) equals the
+    single-weight entry on each."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(21)
+    big = (torch.randn((700, 1600), generator=g, device=DEV) * 0.05).to(torch.bfloat16)
+    weights = [(torch.randn(s, generator=g, device=DEV) * sc).to(torch.bfloat16)
+               for s, sc in (((5120, 5120), 0.02), ((130, 1536), 1.0), ((7, 128), 3.0), ((13824, 5120), 0.02),
+                             ((1000, 576), 0.5))]
+    weights += [big[:, :1536], torch.zeros((129, 64), dtype=torch.bfloat16, device=DEV)]
+    for fmax in (api.FP8_FP4_MAX, api.FP8_FP4_MAX_4OVER6):
+        batch = api.nvfp4_quantize_weights(weights, fmax)
+        for w, b in zip(weights, batch):
+            _assert_same(b, api.nvfp4_quantize_weight(w, fmax))
+    assert api.device_status() == 0
+
+
+def test_batch_chunks_and_f16():
+    """More weights than one launch takes (split into chunks), and fp16."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(22)
+    n = 300
+    weights = [(torch.randn((3 + i % 5, 64 * (1 + i % 3)), generator=g, device=DEV) * (0.1 + i)).to(torch.float16)
+               for i in range(n)]
+    batch = api.nvfp4_quantize_weights(weights)
+    assert len(batch) == n
+    for w, b in zip(weights, batch):
+        _assert_same(b, api.nvfp4_quantize_weight(w))
+    assert api.device_status() == 0
+
+
+def test_batch_graph_replay():
+    g = torch.Generator(device=DEV)
+    g.manual_seed(23)
+    weights = [(torch.randn(s, generator=g, device=DEV) * 0.02).to(torch.bfloat16) for s in ((1024, 5120), (256, 1536))]
+    api.nvfp4_quantize_weights(weights)  # sets up the workspace outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        outs = api.nvfp4_quantize_weights(weights)
+    for scale in (0.5, 7.0):
+        for w in weights:
+            w.mul_(scale)
+        graph.replay()
+        torch.cuda.synchronize()
+        for w, b in zip(weights, outs):
+            _assert_same(b, api.nvfp4_quantize_weight(w))
+    assert api.device_status() == 0
