@@ -22,6 +22,8 @@
 // scale bytes of a 128x4 tile row gathered by shuffles into one 4-byte store.
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "bsp_device.cuh"
 #include "bsp_internal.h"
 
@@ -1220,11 +1222,13 @@ static __device__ __align__(256) uint8_t g_weight_ws[kStaticWeightWsBytes];
 
 // Its address on device dev.id, looked up once per device; the first call
 // also clears the barrier header on `stream` (the array is zero at module load
-// as well).  Not thread-safe; the first call must come before any stream
-// capture (the symbol lookup may load the module).
+// as well).  The set-up is serialised by a lock; the first call must come
+// before any stream capture (the symbol lookup may load the module).
 int static_weight_ws(const DeviceInfo& dev, cudaStream_t stream, void** out) {
   static void* addr[64] = {};
+  static std::mutex mu;
   if (dev.id < 0 || dev.id >= 64) return BSP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev.id]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_weight_ws) != cudaSuccess) return launch_status();

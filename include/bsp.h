@@ -237,9 +237,10 @@ int nvfp4_quantize_weights(const bsp_weight_desc *descs, int count, int w_dtype,
  *   Arguments and errors as nvfp4_quantize_weight, less the workspace; also
  *   INVALID_ARG if this device's grid needs more scratch than the array holds.
  * The first call on each device looks up the array's address
- * (cudaGetSymbolAddress) and clears its barrier header on `stream`; make that
- * first call before any stream capture.  There is one array per device:
- * calls that overlap in time (other streams, other host threads) race. */
+ * (cudaGetSymbolAddress) and clears its barrier header on `stream` (under a
+ * lock); make that first call before any stream capture.  There is one array
+ * per device: calls that overlap in time (other streams, other host threads)
+ * race. */
 int nvfp4_quantize_weight_static(const uint16_t *w, int w_dtype, int64_t N, int64_t K, int64_t ld_w,
                                  float fp8_fp4_max, float *amax, float *gs, float *inv_gs, uint8_t *codes,
                                  uint8_t *sf, bsp_stream_t stream);
