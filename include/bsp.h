@@ -177,7 +177,8 @@ int bsp_nvfp4_alpha(const float *gs_x, const float *gs_w, float *alpha, bsp_stre
  *   amax         : fp32 [1] max|w| (NaN 0, +-inf the largest finite), or NULL
  *   gs, inv_gs   : fp32 [1], as bsp_nvfp4_global_scale_max
  *   codes, sf    : outputs as nvfp4_quantize (N rows; round_up(N, 128) rows of
- *                  scales, the padding rows zero)
+ *                  scales, the padding rows zero); non-NULL even when N = 0
+ *                  (a zero-row weight still gets its amax 0, gs 1, inv_gs 1)
  *   workspace    : device memory of workspace_bytes >= the size that
  *                  bsp_nvfp4_quantize_weight_workspace_bytes reports for this
  *                  device and w_dtype, 16-byte aligned, its first 4 bytes zero
