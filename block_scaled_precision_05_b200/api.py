@@ -233,8 +233,8 @@ def nvfp4_quantize_weight(w: torch.Tensor, fp8_fp4_max: float = FP8_FP4_MAX, out
     overlap in time (one stream, or ordered streams)."""
     _require_cuda(w)
     w = coerce_input(w)
-    if w.dim() != 2 or w.shape[1] % 64 != 0:
-        raise ValueError(f"nvfp4_quantize_weight expects [N, K] with K % 64 == 0, got {tuple(w.shape)}")
+    if w.dim() != 2 or w.shape[1] % 64 != 0 or w.shape[0] == 0:
+        raise ValueError(f"nvfp4_quantize_weight expects [N, K] with N > 0 and K % 64 == 0, got {tuple(w.shape)}")
     if w.stride(1) != 1:
         w = w.contiguous()
     N, K = w.shape
@@ -261,8 +261,9 @@ def nvfp4_quantize_weights(weights, fp8_fp4_max: float = FP8_FP4_MAX):
     for w in weights:
         _require_cuda(w)
         w = coerce_input(w)
-        if w.dim() != 2 or w.shape[1] % 64 != 0:
-            raise ValueError(f"nvfp4_quantize_weights expects [N, K] weights with K % 64 == 0, got {tuple(w.shape)}")
+        if w.dim() != 2 or w.shape[1] % 64 != 0 or w.shape[0] == 0:
+            raise ValueError(f"nvfp4_quantize_weights expects [N, K] weights with N > 0 and K % 64 == 0, "
+                             f"got {tuple(w.shape)}")
         ws_in.append(w if w.stride(1) == 1 else w.contiguous())
     if not ws_in:
         return []
