@@ -1214,8 +1214,8 @@ int run_nvfp4_quantize_weights(const bsp_weight_desc* descs, int count, float fp
 }
 
 // Scratch of nvfp4_quantize_weight_static: a file-scope device array (no
-// allocation by anyone), the header and one word per block for grids of up to
-// kStaticWeightWsBlocks blocks.
+// allocation by anyone) that holds the reported workspace size (header and two
+// words per block) for grids of up to kStaticWeightWsBlocks / 2 blocks.
 constexpr int64_t kStaticWeightWsBlocks = 4096;
 constexpr int64_t kStaticWeightWsBytes = kWeightWsHeader + 4 * kStaticWeightWsBlocks;
 static __device__ __align__(256) uint8_t g_weight_ws[kStaticWeightWsBytes];

@@ -230,8 +230,9 @@ int nvfp4_quantize_weights(const bsp_weight_desc *descs, int count, int w_dtype,
                            int64_t workspace_bytes, bsp_stream_t stream);
 
 /* nvfp4_quantize_weight with no workspace argument and no allocation: its
- * scratch is a static device array inside the library (16,640 bytes: the
- * barrier header and one word per block for grids of up to 4096 blocks).  The
+ * scratch is a static device array inside the library (16,640 bytes: room
+ * for the size bsp_nvfp4_quantize_weight_workspace_bytes reports up to grids
+ * of 2048 blocks; a B200 grid is 444).  The
  * pages have no counterpart; it serves callers that can provide neither
  * scratch memory nor an allocator.  Results are those of
  * nvfp4_quantize_weight.
