@@ -129,3 +129,15 @@ def test_no_gpu_means_an_error_not_a_fallback():
     p = ctypes.c_void_p(0x10000)
     st = L.nvfp4_quantize(p, 4, 32, 32, p, 0, None, None, p, p, None)
     assert st in (nat.BSP_ERR_CUDA, nat.BSP_ERR_UNSUPPORTED_DEVICE)
+
+
+def test_weight_descriptor_layout():
+    """The ctypes mirror of bsp_weight_desc has the header's layout (nine
+    8-byte fields in declaration order, 72 bytes, no padding)."""
+    names = ["w", "N", "K", "ld_w", "amax", "gs", "inv_gs", "codes", "sf"]
+    assert [f[0] for f in nat.BspWeightDesc._fields_] == names
+    assert ctypes.sizeof(nat.BspWeightDesc) == 72
+    for i, n in enumerate(names):
+        assert getattr(nat.BspWeightDesc, n).offset == 8 * i
+    src = open(HEADER).read()
+    assert "#define BSP_WEIGHT_BATCH_MAX 256" in src and nat.BSP_WEIGHT_BATCH_MAX == 256
