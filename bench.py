@@ -82,16 +82,31 @@ def _code_only(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-def source_hash() -> str:
-    """Identifies the kernel sources (csrc/*.cu, *.cuh, *.h; comments and
-    layout ignored) that a committed ncu capture was taken on."""
+# the sources each timed kernel is compiled from (its own file and the shared headers)
+KERNEL_SOURCES = {
+    "nvfp4_gemm": ("gemm.cu", "bsp_device.cuh", "bsp_internal.h"),
+    "mxfp8_gemm": ("gemm.cu", "bsp_device.cuh", "bsp_internal.h"),
+    "nvfp4_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h"),
+    "nvfp4_rmsnorm_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h"),
+    "mxfp8_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h"),
+}
+
+
+def source_hash(files=None) -> str:
+    """Identifies kernel sources (by default every csrc/*.cu, *.cuh, *.h;
+    comments and layout ignored) that a committed ncu capture was taken on."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "block_scaled_precision_05_b200", "csrc")
-    for name in sorted(os.listdir(cdir)):
+    names = sorted(files) if files else sorted(os.listdir(cdir))
+    for name in names:
         if name.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(cdir, name), encoding="utf-8") as f:
                 h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
+
+
+def kernel_source_hash(kernel: str) -> str:
+    return source_hash(KERNEL_SOURCES.get(kernel))
 
 
 def max_over_ranks(ms: float, world: int, device) -> float:
@@ -120,7 +135,7 @@ def traffic_for(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 

@@ -25,3 +25,18 @@ def test_source_hash_ignores_comments_and_layout():
     assert bench._code_only("int a = 1;") != bench._code_only("int a = 2;")
     h = bench.source_hash()
     assert len(h) == 16 and h == bench.source_hash()
+
+
+def test_traffic_entries_are_keyed_to_their_kernels_sources():
+    import json
+    import os
+    assert bench.kernel_source_hash("nvfp4_gemm") == bench.kernel_source_hash("mxfp8_gemm")
+    assert bench.kernel_source_hash("nvfp4_gemm") != bench.kernel_source_hash("nvfp4_quantize")
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        t = json.load(f)
+    for workload, entries in t.items():
+        if workload.startswith("_"):
+            continue
+        for kernel, e in entries.items():
+            assert tuple(e["sources"]) == bench.KERNEL_SOURCES[kernel]
+            assert e["read"] + e["write"] == e["dram_bytes_per_launch"]
