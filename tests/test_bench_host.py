@@ -39,4 +39,4 @@ def test_traffic_entries_are_keyed_to_their_kernels_sources():
             continue
         for kernel, e in entries.items():
             assert tuple(e["sources"]) == bench.KERNEL_SOURCES[kernel]
-            assert e["read"] + e["write"] == e["dram_bytes_per_launch"]
+            assert abs(e["read"] + e["write"] - e["dram_bytes_per_launch"]) <= 1  # each averaged, then truncated
