@@ -2,23 +2,25 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
-Default workload (N=1): the Wan-2.1-1.3B-shaped attention projection as an NVFP4
-W4A4 linear layer, A bf16 [32760, 1536] (N(0,1) with 0.1% x50 outliers),
-W [1536, 1536] ~N(0, 1/sqrt(1536)), bias [1536] ~N(0, 0.01), static activation
-scale 1.0; the weight is quantized once before timing (load time).  One step =
-quantize A (NVFP4 kernel) + block-scaled GEMM with alpha and bias fused (tcgen05
-kernel), inputs resident in HBM; the K timed steps are replayed as one CUDA graph
-with timing events recorded as graph nodes around each step (the per-kernel split
-comes from a second graph with an event between the two kernels).
-`value` = 2*M*N*K per step / step time (TFLOP/s) summed over ranks; L2 is
-flushed (256 MiB write) before every timed step, outside the timed events.
+Default workload (N=1): the Wan-2.1-14B-shaped FFN as two NVFP4 W4A4 linear
+layers, fc_in A bf16 [32760, 5120] ~N(0,1) x W [13824, 5120]^T ~N(0, 1/sqrt(5120)),
+then fc_out A bf16 [32760, 13824] (GELU-shaped) x W [5120, 13824]^T
+~N(0, 1/sqrt(13824)); static activation scale 1.0; weights quantized once
+before timing (load time).  One step = for each layer, quantize its resident
+input (NVFP4 kernel) and run the block-scaled GEMM with alpha fused (tcgen05
+kernel); the K timed steps are replayed as one CUDA graph with timing events
+recorded as graph nodes around each step (the per-kernel split comes from a
+second graph with events between the kernels).  `value` = sum of 2*M*N*K over
+the layers per step / step time (TFLOP/s), summed over ranks; L2 is flushed
+(256 MiB write) before every timed step, outside the timed events.
 
-Other --config values (wan14_in, wan14_out, mxfp8, skinny_m<M>, tiny) time the
-corresponding workload the same way; --config loadtime times the load-time
-conversion of the 240 weights of a 40-block DiT stack (GB/s).
+Other --config values (wan13, wan14_in, wan14_out, mxfp8, skinny_m<M>, tiny)
+time the corresponding one-layer workload the same way; --config loadtime times
+the load-time conversion of the 240 weights of a 40-block DiT stack (GB/s).
 
 --impl reference times the CPU oracle (oracle/, plain C + numpy float64) on a
-bounded row sample of the same workload, on the host cores.
+bounded row sample of every layer of the same workload, on the host cores; the
+default run's cpu_baseline times the same oracle step.
 
 Under torchrun (N > 1) every rank runs the same workload on its own GPU
 (replicas; the path has no exchange step), timing is the max over ranks, and
@@ -214,29 +216,51 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- workloads
-def make_workload(name: str):
+def make_workloads(name: str):
+    """[(Linear, kind)] of the layers one step runs, in order."""
     from block_scaled_precision_05_b200 import workloads as wl
+    if name == "wan14":  # the FFN: fc_in then fc_out, each on its own resident input
+        return [(wl.wan14_in(), "nvfp4"), (wl.wan14_out(), "nvfp4")]
     if name == "wan13":
-        return wl.wan13(), "nvfp4"
+        return [(wl.wan13(), "nvfp4")]
     if name == "tiny":
-        return wl.tiny(), "nvfp4"
+        return [(wl.tiny(), "nvfp4")]
     if name in ("wan14_in", "wan14_out"):
-        return getattr(wl, name)(), "nvfp4"
+        return [(getattr(wl, name)(), "nvfp4")]
     if name == "mxfp8":
-        return wl.mxfp8(), "mxfp8"
+        return [(wl.mxfp8(), "mxfp8")]
     if name.startswith("skinny_m"):
-        return wl.skinny(int(name[len("skinny_m"):])), "nvfp4"
+        return [(wl.skinny(int(name[len("skinny_m"):])), "nvfp4")]
     raise SystemExit(f"unknown --config {name}")
 
 
+def make_workload(name: str):
+    """The single layer of a one-layer configuration."""
+    layers = make_workloads(name)
+    if len(layers) != 1:
+        raise SystemExit(f"--config {name} has {len(layers)} layers")
+    return layers[0]
+
+
 NORM_EPS = 1e-6
+WORKLOAD_TITLES = {
+    "wan14": "Wan-2.1-14B-shaped FFN, NVFP4 W4A4: fc_in A[32760,5120] x W[13824,5120]^T, then fc_out "
+             "A[32760,13824] x W[5120,13824]^T (fc_out input: GELU-shaped, resident)",
+}
 
 
 def norm_gamma(lin):
-    """Seeded RMSNorm weight for --norm rmsnorm: 1 + 0.2 N(0, 1), bf16 bits."""
+    """Seeded norm weight for --norm rmsnorm / layernorm: 1 + 0.2 N(0, 1), bf16 bits."""
     from block_scaled_precision_05_b200 import workloads as wl
     rng = np.random.default_rng(77)
     return wl.f32_to_bf16_bits((1.0 + 0.2 * rng.standard_normal(lin.K)).astype(np.float32))
+
+
+def norm_beta(lin):
+    """Seeded LayerNorm bias for --norm layernorm: 0.1 N(0, 1), bf16 bits."""
+    from block_scaled_precision_05_b200 import workloads as wl
+    rng = np.random.default_rng(78)
+    return wl.f32_to_bf16_bits((0.1 * rng.standard_normal(lin.K)).astype(np.float32))
 
 
 def apply_input_format(lin, kind, fmt):
@@ -252,14 +276,29 @@ def apply_input_format(lin, kind, fmt):
     return lin
 
 
-def describe(lin, kind):
-    d = {"workload": f"{lin.name}: {kind.upper()} linear A[{lin.M},{lin.K}] x W[{lin.N},{lin.K}]^T"
-                     + (" + bias" if lin.bias is not None else "")
-                     + (" (per-token activation scales)" if lin.per_token else ""),
-         "M": lin.M, "N": lin.N, "K": lin.K,
-         "l2": "flushed before every timed step (256 MiB write, outside the timed events)",
-         "timing": "K steps in one CUDA graph, CUDA events as graph nodes around each step's two kernels; "
-                   "per-kernel split from a second graph with an event also between them"}
+def describe(layers, args):
+    """The `config` object of the JSON line; identical in both arms."""
+    lines = [f"{lin.name}: {kind.upper()} linear A[{lin.M},{lin.K}] x W[{lin.N},{lin.K}]^T"
+             + (" + bias" if lin.bias is not None else "")
+             + (" (per-token activation scales)" if lin.per_token else "") for lin, kind in layers]
+    d = {"workload": WORKLOAD_TITLES.get(args.config, "; ".join(lines))}
+    if len(layers) > 1:
+        d["layers"] = lines
+    lin0, kind0 = layers[0]
+    if len(layers) == 1:
+        d.update({"M": lin0.M, "N": lin0.N, "K": lin0.K})
+    d["flop_per_step"] = int(sum(lin.flops for lin, _ in layers))
+    d["l2"] = "flushed before every timed step (256 MiB write, outside the timed events)"
+    d["parallelism"] = "replicas (one process per GPU, no exchange)"
+    d["activation_dtype"] = "fp16" if args.input == "f16" else "bf16"
+    if kind0 == "nvfp4":
+        d["activation_sf_layout"] = args.sf_layout
+        d["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
+    if args.norm == "rmsnorm":
+        d["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
+    elif args.norm == "layernorm":
+        d["producer"] = (f"LayerNorm (gamma 1+0.2N(0,1), beta 0.1N(0,1), eps {NORM_EPS:g}) fused into the "
+                         "quantizer")
     return d
 
 
@@ -271,7 +310,166 @@ def quant_bytes(M, K, kind, sf_layout="128x4"):
     return M * K * 2 + M * K + (-(-M // 128) * 128) * (-(-(K // 32) // 4) * 4)
 
 
+def skinny_gemm_bytes(M, N, K, kind):
+    """Algorithmic HBM bytes of a GEMM that streams the weight once (M <= 128):
+    operand codes, their scales and the bf16 output."""
+    c, g = (0.5, 16) if kind == "nvfp4" else (1.0, 32)
+    return int((M * K + N * K) * c + (M + N) * (K // g) + 2 * M * N)
+
+
+def quant_kernel_name(kind, norm):
+    return {"rmsnorm": "nvfp4_rmsnorm_quantize", "layernorm": "nvfp4_layernorm_quantize"}.get(norm,
+                                                                                              f"{kind}_quantize")
+
+
+def roofline_of(parts, peaks, peak_src, traffic):
+    """Roofline of the dominant kernel.  `parts` lists per layer (lin, kind,
+    q_ms, g_ms, q_bytes); the kernel with the most time over the step is the
+    dominant one, and for several layers its figures are the step's totals
+    (achieved = work over all its launches / their summed duration, traffic =
+    mean per launch)."""
+    q_tot = sum(p[2] for p in parts)
+    g_tot = sum(p[3] for p in parts)
+    kind = parts[0][1]
+    if all(p[0].M <= 128 for p in parts):
+        gb = sum(skinny_gemm_bytes(p[0].M, p[0].N, p[0].K, p[1]) for p in parts)
+        a = gb / (g_tot * 1e-3) / 1e9
+        return {"kernel": f"{kind}_gemm", "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(a / peaks["hbm_gbs"], 4), "traffic": traffic("gemm"),
+                "peak_source": f"{peak_src}: hbm_gbs",
+                "algorithmic": f"{gb // len(parts)} bytes per launch (operand codes + scales + output)"}
+    if g_tot >= q_tot:
+        ratio = FP4_PER_BF16 if kind == "nvfp4" else FP8_PER_BF16
+        peak = peaks["bf16_tflops"] * ratio
+        flops = sum(p[0].flops for p in parts)
+        a = flops / (g_tot * 1e-3) / 1e12
+        per = "; ".join(f"{p[0].name} {p[0].flops:.4g}" for p in parts)
+        return {"kernel": f"{kind}_gemm", "bound": "tensor", "achieved": round(a, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(a / peak, 4), "traffic": traffic("gemm"),
+                "peak_source": f"{peak_src}: bf16_tflops (burst) x {ratio:g} nominal {kind} ratio",
+                "algorithmic": f"2*M*N*K flop per launch ({per})"}
+    qb = sum(p[4] for p in parts)
+    a = qb / (q_tot * 1e-3) / 1e9
+    return {"kernel": "quantize", "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(a / peaks["hbm_gbs"], 4), "traffic": traffic("quantize"),
+            "peak_source": f"{peak_src}: hbm_gbs", "algorithmic": f"{qb // len(parts)} bytes per launch"}
+
+
 # --------------------------------------------------------------------------- our arm
+class LayerRun:
+    """One layer of the timed step on the device: its resident input, the
+    weight quantized at load time, preallocated outputs, and the two launches."""
+
+    def __init__(self, lin, kind, args, dev):
+        import torch
+
+        from block_scaled_precision_05_b200 import api
+        self.api, self.lin, self.kind, self.args, self.dev = api, lin, kind, args, dev
+        self.a_dtype = torch.float16 if lin.fmt == "f16" else torch.bfloat16
+        self.A = self.up(lin.A, self.a_dtype)
+        self.gamma = self.beta = None
+        if args.norm != "none":
+            if kind != "nvfp4" or lin.fmt != "bf16":
+                raise SystemExit(f"--norm {args.norm} applies to the bf16 NVFP4 workloads")
+            self.gamma = self.up(norm_gamma(lin))
+            if args.norm == "layernorm":
+                self.beta = self.up(norm_beta(lin))
+        W = self.up(lin.W)
+        bias = None if lin.bias is None else self.up(lin.bias)
+        if kind == "nvfp4":
+            self.layer = api.NVFP4Linear(W, bias, per_token=lin.per_token, four_over_six=args.four_over_six)
+        else:
+            self.layer = api.MXFP8Linear(W, bias)
+        del W
+        M, K = lin.M, lin.K
+        if kind == "nvfp4" and args.sf_layout == "8x4" and (M > 64 or args.norm != "none"):
+            raise SystemExit("--sf-layout 8x4 applies to NVFP4 workloads with M <= 64 and no fused norm")
+        self.xq = self.new_xq()
+        self.D = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
+        self.qname = quant_kernel_name(kind, args.norm)
+
+    def up(self, a, dtype=None):
+        import torch
+        dtype = dtype or torch.bfloat16
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dtype).to(self.dev)
+
+    def new_xq(self):
+        import torch
+        api, lin, M, K = self.api, self.lin, self.lin.M, self.lin.K
+        if self.kind == "nvfp4":
+            xq = api.NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=self.dev),
+                                 torch.empty(api.nvfp4_sf_bytes(M, K, self.args.sf_layout), dtype=torch.uint8,
+                                             device=self.dev), K, sf_layout=self.args.sf_layout)
+            if lin.per_token:
+                xq.row_gs = torch.empty(M, dtype=torch.float32, device=self.dev)
+                xq.row_inv_gs = torch.empty(M, dtype=torch.float32, device=self.dev)
+            return xq
+        return api.MXFP8Tensor(torch.empty((M, K), dtype=torch.uint8, device=self.dev),
+                               torch.empty(api.mxfp8_sf_bytes(M, K), dtype=torch.uint8, device=self.dev), K)
+
+    def quantize(self, x=None, out=None):
+        api, args, lin, layer = self.api, self.args, self.lin, self.layer
+        x = self.A if x is None else x
+        out = self.xq if out is None else out
+        gs = None if lin.per_token else getattr(layer, "gs_x", None)
+        if args.norm == "rmsnorm":
+            api.nvfp4_rmsnorm_quantize(x, self.gamma, NORM_EPS, gs, per_row=lin.per_token, out=out)
+        elif args.norm == "layernorm":
+            api.nvfp4_layernorm_quantize(x, self.gamma, self.beta, NORM_EPS, gs, per_row=lin.per_token, out=out)
+        elif self.kind == "nvfp4":
+            api.nvfp4_quantize(x, gs, per_row=lin.per_token, out=out, sf_layout=args.sf_layout)
+        else:
+            api.mxfp8_quantize(x, out=out)
+
+    def gemm(self, a=None, b=None, out=None):
+        api, layer = self.api, self.layer
+        a = self.xq if a is None else a
+        b = layer.weight if b is None else b
+        out = self.D if out is None else out
+        if self.kind == "nvfp4":
+            api.nvfp4_gemm(a, b, layer.alpha, a.row_inv_gs if self.lin.per_token else None, layer.bias, out=out)
+        else:
+            api.mxfp8_gemm(a, b, None, layer.bias, out=out)
+
+    def call(self, x):
+        """The public layer call (e2e): quantize (or norm + quantize) and GEMM."""
+        layer, args = self.layer, self.args
+        if args.norm == "rmsnorm":
+            return layer(x, pre_quantized=layer.rmsnorm_quantize_input(x, self.gamma, NORM_EPS))
+        if args.norm == "layernorm":
+            return layer(x, pre_quantized=layer.layernorm_quantize_input(x, self.gamma, self.beta, NORM_EPS))
+        if self.kind == "nvfp4":
+            return layer(x, sf_layout=args.sf_layout)
+        return layer(x)
+
+    @property
+    def w_bytes(self):
+        w = self.layer.weight
+        return (w.codes.numel() if self.kind == "nvfp4" else w.q.numel()) + w.sf.numel()
+
+    @property
+    def a_bytes(self):
+        x = self.xq
+        return (x.codes.numel() if self.kind == "nvfp4" else x.q.numel()) + x.sf.numel()
+
+    def clone_xq(self):
+        import torch
+        x = self.xq
+        if self.kind == "nvfp4":
+            t = self.api.NVFP4Tensor(torch.empty_like(x.codes), torch.empty_like(x.sf), self.lin.K,
+                                     sf_layout=x.sf_layout)
+            if self.lin.per_token:
+                t.row_gs, t.row_inv_gs = torch.empty_like(x.row_gs), torch.empty_like(x.row_inv_gs)
+            return t
+        return self.api.MXFP8Tensor(torch.empty_like(x.q), torch.empty_like(x.sf), self.lin.K)
+
+    def clone_weight(self):
+        w, K = self.layer.weight, self.lin.K
+        if self.kind == "nvfp4":
+            return self.api.NVFP4Tensor(w.codes.clone(), w.sf.clone(), K)
+        return self.api.MXFP8Tensor(w.q.clone(), w.sf.clone(), K)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -280,89 +478,56 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    lin, kind = make_workload(args.config)
-    lin = apply_input_format(lin, kind, args.input)
-    a_dtype = torch.float16 if lin.fmt == "f16" else torch.bfloat16
-
-    def up(a, dtype=torch.bfloat16):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dtype).to(dev)
-
-    A = up(lin.A, a_dtype)
-    if args.norm == "rmsnorm":
-        if kind != "nvfp4" or lin.fmt != "bf16":
-            raise SystemExit("--norm rmsnorm applies to the bf16 NVFP4 workloads")
-        gamma = up(norm_gamma(lin))
-    W = up(lin.W)
-    bias = None if lin.bias is None else up(lin.bias)
-    if kind == "nvfp4":
-        layer = api.NVFP4Linear(W, bias, per_token=lin.per_token, four_over_six=args.four_over_six)
-    else:
-        layer = api.MXFP8Linear(W, bias)
-    del W
-    M, N, K = lin.M, lin.N, lin.K
-    flops = 2.0 * M * N * K
+    specs = [(apply_input_format(lin, kind, args.input), kind) for lin, kind in make_workloads(args.config)]
+    runs = [LayerRun(lin, kind, args, dev) for lin, kind in specs]
+    flops = float(sum(r.lin.flops for r in runs))
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    # preallocated outputs: the timed step launches exactly our two kernels
-    if kind == "nvfp4":
-        if args.sf_layout == "8x4" and (M > 64 or args.norm == "rmsnorm"):
-            raise SystemExit("--sf-layout 8x4 applies to NVFP4 workloads with M <= 64 and no fused norm")
-        xq = api.NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
-                             torch.empty(api.nvfp4_sf_bytes(M, K, args.sf_layout), dtype=torch.uint8, device=dev), K,
-                             sf_layout=args.sf_layout)
-        if lin.per_token:
-            xq.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
-            xq.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
-    else:
-        xq = api.MXFP8Tensor(torch.empty((M, K), dtype=torch.uint8, device=dev),
-                             torch.empty(api.mxfp8_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
-    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-
-    def quantize():
-        if args.norm == "rmsnorm":
-            api.nvfp4_rmsnorm_quantize(A, gamma, NORM_EPS, None if lin.per_token else layer.gs_x,
-                                       per_row=lin.per_token, out=xq)
-        elif kind == "nvfp4":
-            api.nvfp4_quantize(A, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=xq,
-                               sf_layout=args.sf_layout)
-        else:
-            api.mxfp8_quantize(A, out=xq)
-
-    def gemm():
-        if kind == "nvfp4":
-            api.nvfp4_gemm(xq, layer.weight, layer.alpha, xq.row_inv_gs if lin.per_token else None, layer.bias,
-                           out=D)
-        else:
-            api.mxfp8_gemm(xq, layer.weight, None, layer.bias, out=D)
+    if args.profile_launches:
+        # a short eager run for a profiler capture: set-up, then N steps
+        for _ in range(args.profile_launches):
+            for r in runs:
+                r.quantize()
+                r.gemm()
+        torch.cuda.synchronize()
+        if api.device_status() != 0:
+            raise RuntimeError("device error word set")
+        return {"profile_launches": args.profile_launches, "config": args.config,
+                "layers": [r.lin.name for r in runs]}
 
     for _ in range(args.warmup):
         flush.zero_()
-        quantize()
-        gemm()
+        for r in runs:
+            r.quantize()
+            r.gemm()
     torch.cuda.synchronize()
     if api.device_status() != 0:
         raise RuntimeError("device error word set during warm-up")
 
     # The timed region is one CUDA graph holding all K steps back to back: per
-    # step an L2 flush, then a timing event, the quantize and GEMM launches and a
-    # second timing event (events are graph nodes; no Python/ctypes launch
-    # latency inside the measured intervals).  The library is capturable (no
-    # allocation, no host synchronisation).  A second graph of the same steps
-    # with an event also between the two kernels gives the per-kernel split for
-    # the roofline; every event interval on this device carries a launch floor
-    # of about 6 us (an empty kernel between two event nodes reads 6.1 us).
+    # step an L2 flush, then a timing event, every layer's quantize and GEMM
+    # launches and a second timing event (events are graph nodes; no Python or
+    # ctypes launch latency inside the measured intervals).  The library is
+    # capturable (no allocation, no host synchronisation).  A second graph of
+    # the same steps with an event also between every two kernels gives the
+    # per-kernel split; every event interval on this device carries a launch
+    # floor of about 6 us (an empty kernel between two event nodes reads 6.1 us).
+    nk = 2 * len(runs)
+
     def step(evs, split):  # records on the current (capturing) stream
         flush.zero_()
         evs[0].record()
-        quantize()
-        if split:
-            evs[1].record()
-        gemm()
-        evs[2].record()
+        for i, r in enumerate(runs):
+            r.quantize()
+            if split:
+                evs[2 * i + 1].record()
+            r.gemm()
+            if split or i == len(runs) - 1:
+                evs[2 * i + 2].record()
 
     def graph_of(steps, split):
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nk + 1)] for _ in range(steps)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for s in range(steps):
@@ -385,11 +550,11 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier(device_ids=[local_rank])
     g_split.replay()  # untimed for the step value: per-kernel durations only
     torch.cuda.synchronize()
-    step_ms = [ev[s][0].elapsed_time(ev[s][2]) for s in range(args.steps)]
-    t_q = [ev_split[s][0].elapsed_time(ev_split[s][1]) for s in range(args.steps)]
-    t_g = [ev_split[s][1].elapsed_time(ev_split[s][2]) for s in range(args.steps)]
-    total_ms = float(sum(step_ms))
-    total_ms = max_over_ranks(total_ms, world, dev)
+    step_ms = [ev[s][0].elapsed_time(ev[s][nk]) for s in range(args.steps)]
+    split_ms = [[statistics.mean(ev_split[s][j].elapsed_time(ev_split[s][j + 1]) for s in range(args.steps))
+                 for j in range(nk)]]
+    split_ms = split_ms[0]
+    total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
     if api.device_status() != 0:
         raise RuntimeError("device error word set during timing")
     ms_per_step = total_ms / args.steps
@@ -404,23 +569,22 @@ def run_ours(args, rank, world, local_rank):
     # event-interval floor of about 6 us per kernel and is reported beside it.
     # R launches last about 2 ms in all (4 to 24), short enough to stay a burst
     # like the timed steps rather than a sustained power-capped loop.
-    def launches_for(step_ms):
-        return int(min(24, max(4, 2.0 / max(step_ms, 1e-3))))
+    def launches_for(ms):
+        return int(min(24, max(4, 2.0 / max(ms, 1e-3))))
 
-    q_step_ms, g_step_ms = statistics.mean(t_q), statistics.mean(t_g)
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
 
     def rotations(streamed_bytes):
         return int(min(8, max(2, -(-3 * l2_bytes // max(1, streamed_bytes)))))
 
     def back_to_back(launch, n_rot, R):
-        for r in range(n_rot):
-            launch(r)
+        for i in range(n_rot):
+            launch(i)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for r in range(R):
-                launch(r % n_rot)
+            for i in range(R):
+                launch(i % n_rot)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         g.replay()
         torch.cuda.synchronize()
@@ -431,103 +595,71 @@ def run_ours(args, rank, world, local_rank):
         del g
         return e0.elapsed_time(e1) / R
 
-    # the GEMM streams A (large M) or the weight (skinny M) from DRAM
-    w_bytes = layer.weight.codes.numel() + layer.weight.sf.numel() if kind == "nvfp4" else \
-        layer.weight.q.numel() + layer.weight.sf.numel()
-    a_bytes = xq.codes.numel() + xq.sf.numel() if kind == "nvfp4" else xq.q.numel() + xq.sf.numel()
-    rotate_weight = w_bytes > a_bytes
-    nq = rotations(A.numel() * A.element_size())  # bf16 inputs of the quantizer
-    nx = max(nq, 1 if rotate_weight else rotations(a_bytes))  # quantized activations
-    A_rot = [A] + [A.clone() for _ in range(nq - 1)]
-    if kind == "nvfp4":
-        xq_rot = [xq] + [api.NVFP4Tensor(torch.empty_like(xq.codes), torch.empty_like(xq.sf), K,
-                                          sf_layout=xq.sf_layout) for _ in range(nx - 1)]
-        for t in xq_rot[1:]:
-            if lin.per_token:
-                t.row_gs, t.row_inv_gs = torch.empty_like(xq.row_gs), torch.empty_like(xq.row_inv_gs)
-    else:
-        xq_rot = [xq] + [api.MXFP8Tensor(torch.empty_like(xq.q), torch.empty_like(xq.sf), K) for _ in range(nx - 1)]
+    b2b = []  # per layer: (quantize ms, GEMM ms, R_q, R_g)
+    for i, r in enumerate(runs):
+        # the GEMM streams A (large M) or the weight (skinny M) from DRAM
+        rotate_weight = r.w_bytes > r.a_bytes
+        nq = rotations(r.A.numel() * r.A.element_size())
+        nx = max(nq, 1 if rotate_weight else rotations(r.a_bytes))
+        A_rot = [r.A] + [r.A.clone() for _ in range(nq - 1)]
+        xq_rot = [r.xq] + [r.clone_xq() for _ in range(nx - 1)]
+        R_q, R_g = launches_for(split_ms[2 * i]), launches_for(split_ms[2 * i + 1])
+        q_ms = back_to_back(lambda j: r.quantize(A_rot[j % nq], xq_rot[j]), nx, max(R_q, nx))
+        ng = rotations(max(r.w_bytes, r.a_bytes))
+        w_rot = [r.layer.weight] + [r.clone_weight() for _ in range(ng - 1)] if rotate_weight else None
+        D_rot = [r.D] + [torch.empty_like(r.D) for _ in range(min(ng, 2) - 1)]
 
-    def quant_launch(r):
-        x, out = A_rot[r % nq], xq_rot[r]
-        if args.norm == "rmsnorm":
-            api.nvfp4_rmsnorm_quantize(x, gamma, NORM_EPS, None if lin.per_token else layer.gs_x,
-                                       per_row=lin.per_token, out=out)
-        elif kind == "nvfp4":
-            api.nvfp4_quantize(x, None if lin.per_token else layer.gs_x, per_row=lin.per_token, out=out,
-                               sf_layout=args.sf_layout)
-        else:
-            api.mxfp8_quantize(x, out=out)
+        def gemm_launch(j):
+            a = r.xq if rotate_weight else xq_rot[j]
+            b = w_rot[j] if rotate_weight else None
+            r.gemm(a, b, D_rot[j % len(D_rot)])
 
-    R_q, R_g = launches_for(q_step_ms), launches_for(g_step_ms)
-    q_b2b_ms = back_to_back(quant_launch, nx, max(R_q, nx))  # also fills every quantized buffer
-    ng = rotations(max(w_bytes, a_bytes))
-    if rotate_weight:
-        w = layer.weight
-        if kind == "nvfp4":
-            w_rot = [w] + [api.NVFP4Tensor(w.codes.clone(), w.sf.clone(), K) for _ in range(ng - 1)]
-        else:
-            w_rot = [w] + [api.MXFP8Tensor(w.q.clone(), w.sf.clone(), K) for _ in range(ng - 1)]
-    D_rot = [D] + [torch.empty_like(D) for _ in range(min(ng, 2) - 1)]
+        g_ms = back_to_back(gemm_launch, ng if rotate_weight else nx, R_g)
+        del A_rot, xq_rot, D_rot, w_rot
+        torch.cuda.empty_cache()
+        b2b.append((max_over_ranks(q_ms, world, dev), max_over_ranks(g_ms, world, dev), R_q, R_g))
 
-    def gemm_launch(r):
-        a = xq if rotate_weight else xq_rot[r]
-        b = w_rot[r] if rotate_weight else layer.weight
-        out = D_rot[r % len(D_rot)]
-        if kind == "nvfp4":
-            api.nvfp4_gemm(a, b, layer.alpha, a.row_inv_gs if lin.per_token else None, layer.bias, out=out)
-        else:
-            api.mxfp8_gemm(a, b, None, layer.bias, out=out)
-
-    g_b2b_ms = back_to_back(gemm_launch, ng if rotate_weight else nx, R_g)
-    del A_rot, xq_rot, D_rot
-    if rotate_weight:
-        del w_rot
-    q_b2b_ms = max_over_ranks(q_b2b_ms, world, dev)
-    g_b2b_ms = max_over_ranks(g_b2b_ms, world, dev)
-
-    # ---- end to end through the public API: every step copies its input from
-    # pinned host memory and its result back to pinned host memory.  With large
-    # copies the steps are pipelined as a serving loop would run them: the
-    # copy-in of step i+1 and the copy-out of step i-1 run on their own streams
-    # while step i computes (two device input buffers, two host output
-    # buffers).  With small copies (skinny M) the extra stream bookkeeping costs
-    # more host time than it hides, and the steps run on one stream.
-    A_host = torch.from_numpy(np.ascontiguousarray(lin.A).view(np.int16)).view(a_dtype).pin_memory()
-    D_host = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    A_dev = [torch.empty_like(A) for _ in range(2)]
+    # ---- end to end through the public API: every step copies each layer's
+    # input from pinned host memory and its result back to pinned host memory.
+    # With large copies the steps are pipelined as a serving loop would run
+    # them: the copy-in of step i+1 and the copy-out of step i-1 run on their
+    # own streams while step i computes (two device input buffers and two host
+    # output buffers per layer).  With small copies (skinny M) the extra stream
+    # bookkeeping costs more host time than it hides, and the steps run on one
+    # stream.
+    A_host = [torch.from_numpy(np.ascontiguousarray(r.lin.A).view(np.int16)).view(r.a_dtype).pin_memory()
+              for r in runs]
+    D_host = [[torch.empty((r.lin.M, r.lin.N), dtype=torch.bfloat16).pin_memory() for _ in range(2)] for r in runs]
+    A_dev = [[torch.empty_like(r.A) for _ in range(2)] for r in runs]
     e2e_steps = max(2, min(args.steps, 20))
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
-
-    pipelined = A.numel() * 2 + M * N * 2 > (16 << 20)
+    h2d = sum(a.numel() * a.element_size() for a in A_host)
+    d2h = sum(d[0].numel() * 2 for d in D_host)
+    pipelined = h2d + d2h > (16 << 20)
 
     def e2e_step(i):
         b = i % 2
         if not pipelined:
-            A_dev[0].copy_(A_host, non_blocking=True)
-            if args.norm == "rmsnorm":
-                y = layer(A_dev[0], pre_quantized=layer.rmsnorm_quantize_input(A_dev[0], gamma, NORM_EPS))
-            else:
-                y = layer(A_dev[0], sf_layout=args.sf_layout) if kind == "nvfp4" else layer(A_dev[0])
-            D_host[0].copy_(y, non_blocking=True)
+            for li, r in enumerate(runs):
+                A_dev[li][0].copy_(A_host[li], non_blocking=True)
+                D_host[li][0].copy_(r.call(A_dev[li][0]), non_blocking=True)
             return
         with torch.cuda.stream(s_in):
             if i >= 2:
-                s_in.wait_event(ev_comp[b])  # step i-2 has finished reading A_dev[b]
-            A_dev[b].copy_(A_host, non_blocking=True)
+                s_in.wait_event(ev_comp[b])  # step i-2 has finished reading A_dev[.][b]
+            for li in range(len(runs)):
+                A_dev[li][b].copy_(A_host[li], non_blocking=True)
             ev_in[b].record(s_in)
         stream.wait_event(ev_in[b])
-        if args.norm == "rmsnorm":
-            y = layer(A_dev[b], pre_quantized=layer.rmsnorm_quantize_input(A_dev[b], gamma, NORM_EPS))
-        else:
-            y = layer(A_dev[b], sf_layout=args.sf_layout) if kind == "nvfp4" else layer(A_dev[b])
+        ys = [r.call(A_dev[li][b]) for li, r in enumerate(runs)]
         ev_comp[b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp[b])
-            D_host[b].copy_(y, non_blocking=True)  # in order after step i-2's copy of D_host[b]
-            y.record_stream(s_out)
+            for li, y in enumerate(ys):
+                D_host[li][b].copy_(y, non_blocking=True)  # in order after step i-2's copy of D_host[.][b]
+                y.record_stream(s_out)
 
     def e2e_run(n):
         e0, e1, e_out = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -553,71 +685,57 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
-    q_ms, g_ms = q_b2b_ms, g_b2b_ms
-    qb = quant_bytes(M, K, kind, args.sf_layout)
-    q_gbs = qb / (q_ms * 1e-3) / 1e9
-    g_tflops = flops / (g_ms * 1e-3) / 1e12
-    ratio = FP4_PER_BF16 if kind == "nvfp4" else FP8_PER_BF16
-    tensor_peak = peaks["bf16_tflops"] * ratio
-    hbm_peak = peaks["hbm_gbs"]
-    wname = args.config + ("_rmsnorm" if args.norm == "rmsnorm" else "")
-    qname = "nvfp4_rmsnorm_quantize" if args.norm == "rmsnorm" else f"{kind}_quantize"
-    if M <= 128:
-        # skinny M: the GEMM streams the weight once; bound by HBM
-        gb = (M * K + N * K) * (0.5 if kind == "nvfp4" else 1.0) + (M + N) * (K // 16 if kind == "nvfp4" else K // 32) \
-            + 2 * M * N
-        g_gbs = gb / (g_ms * 1e-3) / 1e9
-        roof = {"kernel": f"{kind}_gemm", "bound": "hbm", "achieved": round(g_gbs, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(g_gbs / hbm_peak, 4), "traffic": traffic_for(f"{kind}_gemm", wname),
-                "peak_source": f"{peak_src}: hbm_gbs",
-                "algorithmic": f"{int(gb)} bytes per launch (operand codes + scales + output)"}
-    elif g_ms >= q_ms:
-        roof = {"kernel": f"{kind}_gemm", "bound": "tensor", "achieved": round(g_tflops, 1),
-                "peak": round(tensor_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / tensor_peak, 4),
-                "traffic": traffic_for(f"{kind}_gemm", wname),
-                "peak_source": f"{peak_src}: bf16_tflops (burst) x {ratio:g} nominal {kind} ratio",
-                "algorithmic": f"2*M*N*K = {flops:.4g} flop per launch"}
-    else:
-        roof = {"kernel": qname, "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4), "traffic": traffic_for(qname, wname),
-                "peak_source": f"{peak_src}: hbm_gbs", "algorithmic": f"{qb} bytes per launch"}
+    parts = [(r.lin, r.kind, q, g, quant_bytes(r.lin.M, r.lin.K, r.kind, args.sf_layout))
+             for r, (q, g, _, _) in zip(runs, b2b)]
+    wsuffix = {"rmsnorm": "_rmsnorm", "layernorm": "_layernorm"}.get(args.norm, "")
 
-    cfg = describe(lin, kind)
-    cfg["parallelism"] = f"replicas x{world}"
-    cfg["activation_dtype"] = "fp16" if lin.fmt == "f16" else "bf16"
-    if kind == "nvfp4":
-        cfg["activation_sf_layout"] = args.sf_layout
-    if args.norm == "rmsnorm":
-        cfg["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
-    if kind == "nvfp4":
-        cfg["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
+    def traffic(which):
+        vals = [traffic_for(f"{r.kind}_gemm" if which == "gemm" else r.qname, r.lin.name + wsuffix) for r in runs]
+        return None if any(v is None for v in vals) else int(sum(vals) / len(vals))
+
+    roof = roofline_of(parts, peaks, peak_src, traffic)
+    if roof["kernel"] == "quantize":
+        roof["kernel"] = runs[0].qname
+    hbm_peak = peaks["hbm_gbs"]
+    kernels = {}
+    for i, (r, (q_ms, g_ms, R_q, R_g)) in enumerate(zip(runs, b2b)):
+        ratio = FP4_PER_BF16 if r.kind == "nvfp4" else FP8_PER_BF16
+        tensor_peak = peaks["bf16_tflops"] * ratio
+        qb = parts[i][4]
+        g_tflops = r.lin.flops / (g_ms * 1e-3) / 1e12
+        entry = {r.qname: {"ms": round(q_ms, 5), "GB/s": round(qb / (q_ms * 1e-3) / 1e9, 1),
+                           "frac_hbm": round(qb / (q_ms * 1e-3) / 1e9 / hbm_peak, 4)},
+                 f"{r.kind}_gemm": {"ms": round(g_ms, 5), "TFLOP/s": round(g_tflops, 1),
+                                    "frac_tensor_peak": round(g_tflops / tensor_peak, 4)},
+                 "launches_back_to_back": [R_q, R_g],
+                 "per_step_event_split_ms": [round(split_ms[2 * i], 5), round(split_ms[2 * i + 1], 5)]}
+        if r.lin.M <= 128:
+            gb = skinny_gemm_bytes(r.lin.M, r.lin.N, r.lin.K, r.kind)
+            entry[f"{r.kind}_gemm"]["frac_hbm"] = round(gb / (g_ms * 1e-3) / 1e9 / hbm_peak, 4)
+        kernels[r.lin.name] = entry
+    kernels["timing"] = ("each kernel launched R times back to back in one CUDA graph between two events (about "
+                         "2 ms), operands rotated through buffers totalling > 3x L2 so each launch streams from "
+                         "DRAM; per_step_event_split_ms: events around each kernel inside the timed steps, each "
+                         "interval carrying a ~6 us event/launch floor")
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "nvfp4" if kind == "nvfp4" else "mxfp8", "data": "synthetic (seeded numpy)",
-        "config": cfg, "roofline": roof,
-        "kernels": {
-            qname: {"ms": round(q_ms, 5), "GB/s": round(q_gbs, 1), "frac_hbm": round(q_gbs / hbm_peak, 4)},
-            f"{kind}_gemm": {"ms": round(g_ms, 5), "TFLOP/s": round(g_tflops, 1),
-                             "frac_tensor_peak": round(g_tflops / tensor_peak, 4)},
-            "timing": f"{R_q} / {R_g} launches back to back in one CUDA graph between two events (about 2 ms), "
-                      "operands rotated through buffers totalling > 3x L2 so each launch streams from DRAM",
-            "per_step_event_split_ms": {qname: round(q_step_ms, 5), f"{kind}_gemm": round(g_step_ms, 5),
-                                        "note": "events around each kernel inside the timed steps; each "
-                                                "interval carries a ~6 us event/launch floor"},
-        },
+        "vs_baseline": None, "dtype": "nvfp4" if runs[0].kind == "nvfp4" else "mxfp8",
+        "data": "synthetic (seeded numpy)", "config": describe(specs, args), "roofline": roof,
+        "kernels": kernels,
         "e2e": {"value": round(whole_job_rate(flops, world, 1, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(A_host.numel() * 2), "d2h_bytes_per_step": int(D_host[0].numel() * 2),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e_ms, 4), "runs_ms_per_step": [round(v, 4) for v in e2e_runs],
                 "steps_per_run": e2e_steps,
                 "pipelining": ("each step's copy-in, compute and copy-out on three streams; consecutive steps "
                                "overlap") if pipelined else "none (one stream; small copies)"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": nk * args.steps,
+        "timing": ("K steps in one CUDA graph, CUDA events as graph nodes around each step's kernels; L2 flushed "
+                   "before every step outside the events"),
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = oracle_baseline(lin, kind, budget_s=args.cpu_budget, four_over_six=args.four_over_six,
-                                              norm=args.norm)
+        out["cpu_baseline"] = oracle_baseline(specs, args)
     return out
 
 
@@ -750,7 +868,8 @@ def run_loadtime(args, rank, world, local_rank):
 
 # --------------------------------------------------------------------------- oracle arm
 def oracle_step(lin, kind, rows, wq, norm=None):
-    """The oracle's linear layer on `rows` of A: quantize, decode, float64 GEMM, epilogue."""
+    """The oracle's linear layer on `rows` of A: (norm,) quantize, decode,
+    float64 GEMM, epilogue, bf16 rounding."""
     import oracle
     K = lin.K
     A = lin.A[rows]
@@ -759,6 +878,9 @@ def oracle_step(lin, kind, rows, wq, norm=None):
         fmt = getattr(lin, "fmt", "bf16")
         if norm == "rmsnorm":
             A = oracle.rmsnorm_bf16(A, norm_gamma(lin), oracle.rmsnorm_rstd(A, NORM_EPS))
+        elif norm == "layernorm":
+            mean, rstd = oracle.layernorm_stats(A, NORM_EPS)
+            A = oracle.layernorm_bf16(A, norm_gamma(lin), norm_beta(lin), mean, rstd)
         if lin.per_token:
             gs, inv = oracle.row_global_scales(A, fmt=fmt)
             ca, sa = oracle.nvfp4_quantize(A, gs, per_row=True, fmt=fmt)
@@ -794,24 +916,56 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_baseline(lin, kind, budget_s=10.0, four_over_six=False, norm=None):
-    """Times the oracle on a bounded row sample, scaled to TFLOP/s."""
-    wq = oracle_weights(lin, kind, four_over_six)
-    rng = np.random.default_rng(123)
-    rows = np.sort(rng.choice(lin.M, size=min(lin.M, 128), replace=False))
-    t0 = time.perf_counter()
-    oracle_step(lin, kind, rows, wq, norm)
-    dt = time.perf_counter() - t0
-    n = int(min(lin.M, max(128, 128 * budget_s / max(dt, 1e-3))))
-    rows = np.sort(rng.choice(lin.M, size=n, replace=False))
-    t0 = time.perf_counter()
-    oracle_step(lin, kind, rows, wq, norm)
-    dt = time.perf_counter() - t0
-    flops = 2.0 * n * lin.N * lin.K
-    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": max(os.cpu_count() or 1, blas_threads()),
-            "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"{n} random rows of A (of {lin.M}): quantize + decode + float64 GEMM + epilogue + bf16 "
-                      f"rounding; weight quantized beforehand (load time)"}
+def oracle_rows(args, M):
+    """Rows of A per layer that one oracle step processes: --ref-rows, or by
+    default up to 128 (about a second of oracle work per Wan-14B layer)."""
+    if args.ref_rows:
+        return min(M, args.ref_rows)
+    return M if M <= 128 else 128
+
+
+class OracleRunner:
+    """The oracle's step over the same layers as the GPU step: each step takes
+    a fresh random sample of rows of every layer's A (seeded) and runs the whole
+    path on them.  Used, unchanged, by the reference arm and by cpu_baseline,
+    so both report the same work per step."""
+
+    def __init__(self, specs, args, seed=7):
+        self.specs, self.args = specs, args
+        self.wq = [oracle_weights(lin, kind, args.four_over_six) for lin, kind in specs]
+        self.n = [oracle_rows(args, lin.M) for lin, _ in specs]
+        self.rng = np.random.default_rng(seed)
+        self.flops = 2.0 * sum(n * lin.N * lin.K for n, (lin, _) in zip(self.n, specs))
+
+    def step(self):
+        for (lin, kind), wq, n in zip(self.specs, self.wq, self.n):
+            rows = np.sort(self.rng.choice(lin.M, size=n, replace=False))
+            oracle_step(lin, kind, rows, wq, self.args.norm)
+
+    def sample(self):
+        parts = [f"{n} random rows of {lin.name} A (of {lin.M})" for n, (lin, _) in zip(self.n, self.specs)]
+        return ("per step " + ", ".join(parts) + ": quantize + decode + float64 GEMM + epilogue + bf16 rounding; "
+                "weights quantized beforehand (load time); plain C + numpy oracle")
+
+    def timed(self, steps, warmup):
+        for _ in range(warmup):
+            self.step()
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            self.step()
+        return time.perf_counter() - t0
+
+
+def oracle_baseline(specs, args):
+    """cpu_baseline: the reference arm's oracle step, timed for about
+    --cpu-budget seconds (at least one step after one warm-up step)."""
+    orc = OracleRunner(specs, args)
+    t1 = orc.timed(1, 1)
+    steps = int(max(1, min(50, args.cpu_budget / max(t1, 1e-3))))
+    dt = t1 + (orc.timed(steps - 1, 0) if steps > 1 else 0.0)
+    return {"value": round(orc.flops * steps / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": max(os.cpu_count() or 1, blas_threads()), "kind": "oracle", "steps": steps,
+            "seconds": round(dt, 2), "sample": orc.sample()}
 
 
 def run_reference_loadtime(args):
@@ -848,39 +1002,21 @@ def run_reference_loadtime(args):
 
 
 def run_reference(args):
+    """The oracle on the host cores as the reference arm: the same layers, a
+    bounded row sample of each per step (the same runner as cpu_baseline)."""
     if args.config == "loadtime":
         return run_reference_loadtime(args)
-    lin, kind = make_workload(args.config)
-    lin = apply_input_format(lin, kind, args.input)
-    wq = oracle_weights(lin, kind, args.four_over_six)
-    rng = np.random.default_rng(7)
-    n = min(lin.M, args.ref_rows)
-    for _ in range(args.warmup):
-        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq, args.norm)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(lin, kind, np.sort(rng.choice(lin.M, size=n, replace=False)), wq, args.norm)
-    dt = time.perf_counter() - t0
-    flops = 2.0 * n * lin.N * lin.K * args.steps
-    value = flops / dt / 1e12
+    specs = [(apply_input_format(lin, kind, args.input), kind) for lin, kind in make_workloads(args.config)]
+    orc = OracleRunner(specs, args)
+    dt = orc.timed(args.steps, args.warmup)
+    value = orc.flops * args.steps / dt / 1e12
     cores = max(os.cpu_count() or 1, blas_threads())
-    sample = (f"{n} random rows of A per step (of {lin.M}): quantize + decode + float64 GEMM + epilogue + bf16 "
-              f"rounding; weight quantized beforehand (load time)")
-    cfg = describe(lin, kind)
-    cfg["parallelism"] = "host cores"
-    cfg["activation_dtype"] = "fp16" if lin.fmt == "f16" else "bf16"
-    if kind == "nvfp4":
-        cfg["activation_sf_layout"] = args.sf_layout
-    if args.norm == "rmsnorm":
-        cfg["producer"] = f"RMSNorm (gamma 1+0.2N(0,1), eps {NORM_EPS:g}) fused into the quantizer"
-    if kind == "nvfp4":
-        cfg["weight_global_scale"] = "256*6/amax (4over6)" if args.four_over_six else "448*6/amax"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64 (oracle)", "data": "synthetic (seeded numpy)", "config": cfg,
+            "dtype": "f64 (oracle)", "data": "synthetic (seeded numpy)", "config": describe(specs, args),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": orc.sample()},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -890,18 +1026,21 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="wan13")
+    ap.add_argument("--config", default="wan14")
     ap.add_argument("--sf-layout", choices=["128x4", "8x4"], default="128x4",
                     help="activation scale layout of the NVFP4 workloads (8x4: M <= 64)")
     ap.add_argument("--norm", choices=["none", "rmsnorm"], default="none",
-                    help="NVFP4 workloads: fuse an RMSNorm of the activation into the quantizer")
+                    help="NVFP4 workloads: fuse a norm of the activation into the quantizer")
     ap.add_argument("--input", choices=["bf16", "f16"], default="bf16",
                     help="activation dtype of the NVFP4 workloads (f16: the bf16 values rounded to fp16)")
     ap.add_argument("--four-over-six", action="store_true",
                     help="NVFP4 weight global scale 256*6/amax (the 4over6 setting) instead of 448*6/amax")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--ref-rows", type=int, default=256, help="rows per oracle step for --impl reference")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="rows of each layer's A per oracle step (reference arm and cpu_baseline; 0: up to 128)")
+    ap.add_argument("--profile-launches", type=int, default=0,
+                    help="set up, run this many untimed eager steps and exit (for a profiler capture)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--blocks", type=int, default=40, help="DiT blocks for --config loadtime")
     args = ap.parse_args()

@@ -138,10 +138,11 @@ __device__ __forceinline__ float global_scale_from_mag(uint32_t mag) {
 }
 
 // fl32(x / 6) for x a bf16 or fp16 magnitude: the product with fl32(1/6),
-// corrected once by the fma residual.  For 0 and every positive finite bf16 and
-// fp16 value this equals the correctly rounded quotient (checked exhaustively
-// against exact rationals); +inf (the amax of a group holding an infinity)
-// gives +inf.
+// corrected once by the fma residual r = x - 6q (a residual-corrected
+// reciprocal product in the manner of Markstein's division: q' = q + r/6 with
+// r exact by the fma).  For 0 and every positive finite bf16 and fp16 value
+// this equals the correctly rounded quotient (checked exhaustively against
+// exact rationals); +inf (the amax of a group holding an infinity) gives +inf.
 __device__ __forceinline__ float div6_rn(float x) {
   constexpr float kSixth = 0x1.555556p-3f;  // fl32(1/6)
   const float q = __fmul_rn(x, kSixth);
@@ -838,8 +839,8 @@ __global__ void global_scale_kernel(const float* __restrict__ amax, float fp8_fp
 //      smaller than L2 is read from DRAM once).
 // The grid is one co-resident wave (a cooperative launch where the runtime
 // allows it), so every block reaches the barrier.
-// Workspace: [0] arrivals at the barrier (0 outside it; must be 0 before the
-// first launch), [1] barrier generation, then one word per block from byte
+// Workspace: [0] arrivals at the barrier, [1] barrier generation (both set to
+// 0 on the stream before every launch), then one word per block from byte
 // kWeightWsHeader.
 // ---------------------------------------------------------------------------
 constexpr int64_t kWeightWsHeader = 256;
@@ -1158,6 +1159,9 @@ int run_nvfp4_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t l
   int grid = 0;
   if ((st = weight_grid<In>(dev, &grid)) != BSP_OK) return st;
   if (ws_bytes < kWeightWsHeader + 4 * static_cast<int64_t>(grid)) return BSP_ERR_INVALID_ARG;  // one slot used here
+  // the barrier words start at 0 whatever an earlier call left (one that timed
+  // out leaves its arrival count behind)
+  if (cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), stream) != cudaSuccess) return launch_status();
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -1198,6 +1202,7 @@ int run_nvfp4_quantize_weights(const bsp_weight_desc* descs, int count, float fp
   int grid = 0;
   if ((st = weight_grid<In>(dev, &grid)) != BSP_OK) return st;
   if (ws_bytes < kWeightWsHeader + 8 * static_cast<int64_t>(grid)) return BSP_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), stream) != cudaSuccess) return launch_status();  // barrier words
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -1220,11 +1225,13 @@ constexpr int64_t kStaticWeightWsBlocks = 4096;
 constexpr int64_t kStaticWeightWsBytes = kWeightWsHeader + 4 * kStaticWeightWsBlocks;
 static __device__ __align__(256) uint8_t g_weight_ws[kStaticWeightWsBytes];
 
-// Its address on device dev.id, looked up once per device; the first call
-// also clears the barrier header on `stream` (the array is zero at module load
-// as well).  The set-up is serialised by a lock; the first call must come
-// before any stream capture (the symbol lookup may load the module).
-int static_weight_ws(const DeviceInfo& dev, cudaStream_t stream, void** out) {
+// Its address on device dev.id, looked up once per device (the launch clears
+// the barrier words before every call).  The set-up is serialised by a lock;
+// the first call must come before any stream capture (the symbol lookup may
+// load the module).  The cached address belongs to the device's primary
+// context: after cudaDeviceReset the entry is not to be called again in the
+// same process.
+int static_weight_ws(const DeviceInfo& dev, void** out) {
   static void* addr[64] = {};
   static std::mutex mu;
   if (dev.id < 0 || dev.id >= 64) return BSP_ERR_INVALID_ARG;
@@ -1232,7 +1239,6 @@ int static_weight_ws(const DeviceInfo& dev, cudaStream_t stream, void** out) {
   if (!addr[dev.id]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_weight_ws) != cudaSuccess) return launch_status();
-    if (cudaMemsetAsync(p, 0, kWeightWsHeader, stream) != cudaSuccess) return launch_status();
     addr[dev.id] = p;
   }
   *out = addr[dev.id];
@@ -1404,7 +1410,7 @@ int nvfp4_quantize_weight_static(const uint16_t* w, int w_dtype, int64_t N, int6
   DeviceInfo dev;
   if ((st = current_device(&dev)) != BSP_OK) return st;
   void* ws = nullptr;
-  if ((st = static_weight_ws(dev, stream, &ws)) != BSP_OK) return st;
+  if ((st = static_weight_ws(dev, &ws)) != BSP_OK) return st;
   return nvfp4_quantize_weight(w, w_dtype, N, K, ld_w, fp8_fp4_max, amax, gs, inv_gs, codes, sf, ws,
                                kStaticWeightWsBytes, stream);
 }

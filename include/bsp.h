@@ -181,10 +181,11 @@ int bsp_nvfp4_alpha(const float *gs_x, const float *gs_w, float *alpha, bsp_stre
  *                  (a zero-row weight still gets its amax 0, gs 1, inv_gs 1)
  *   workspace    : device memory of workspace_bytes >= the size that
  *                  bsp_nvfp4_quantize_weight_workspace_bytes reports for this
- *                  device and w_dtype, 16-byte aligned, its first 4 bytes zero
- *                  before the first call; each call leaves them zero again.
- *                  Owned by the caller; calls that overlap in time on one
- *                  workspace race.
+ *                  device and w_dtype, 16-byte aligned, any content: the call
+ *                  sets its two barrier words to 0 on `stream` before the
+ *                  launch, so a workspace left behind by a call that timed out
+ *                  is fit for the next call.  Owned by the caller; calls that
+ *                  overlap in time on one workspace race.
  * Launched cooperatively (every block resident at once).  Errors:
  * INVALID_ARG (sizes, modes, NULL pointers, workspace too small), ALIGNMENT,
  * UNSUPPORTED_DEVICE, CUDA (the launch failed, e.g. a cooperative launch the
@@ -239,10 +240,12 @@ int nvfp4_quantize_weights(const bsp_weight_desc *descs, int count, int w_dtype,
  *   Arguments and errors as nvfp4_quantize_weight, less the workspace; also
  *   INVALID_ARG if this device's grid needs more scratch than the array holds.
  * The first call on each device looks up the array's address
- * (cudaGetSymbolAddress) and clears its barrier header on `stream` (under a
- * lock); make that first call before any stream capture.  There is one array
- * per device: calls that overlap in time (other streams, other host threads)
- * race. */
+ * (cudaGetSymbolAddress, under a lock) and keeps it for the life of the
+ * process; make that first call before any stream capture.  Every call clears
+ * the barrier words on `stream` before its launch.  The address belongs to
+ * the device's primary context: after cudaDeviceReset this entry must not be
+ * called again in the same process.  There is one array per device: calls
+ * that overlap in time (other streams, other host threads) race. */
 int nvfp4_quantize_weight_static(const uint16_t *w, int w_dtype, int64_t N, int64_t K, int64_t ld_w,
                                  float fp8_fp4_max, float *amax, float *gs, float *inv_gs, uint8_t *codes,
                                  uint8_t *sf, bsp_stream_t stream);

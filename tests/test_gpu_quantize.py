@@ -30,6 +30,75 @@ def _data(M, K, seed, kind="normal"):
 
 SHAPES = [(1, 16), (1, 64), (7, 48), (128, 256), (129, 64), (130, 80), (300, 1536), (257, 5120), (64, 13824)]
 
+# Dispatch branches of the quantize launchers (each instantiated for bf16 and
+# fp16 input and for 128x4 and 8x4 scale tiles) and the bit-exact tests that
+# reach each of them:
+#
+# nvfp4_quantize / _f16 / _ex (run_nvfp4_quantize):
+#   K % 64 == 0, per-row, round_up(M) <= resident blocks (at most 148 x 8)
+#       nvfp4_quant_rowblock_kernel     test_nvfp4_quantize_per_row_bit_exact (M <= 300),
+#                                       test_dispatch_branch_bit_exact[rowblock-*]
+#   K % 64 == 0, per-row, more rows
+#       nvfp4_quant_k64_kernel<true>    test_dispatch_branch_bit_exact[k64-per-row-*] (M = 4100)
+#   per-tensor, K == 1024
+#       nvfp4_quant_short_kernel<S=2>   test_dispatch_branch_bit_exact[short-1024-*]
+#   per-tensor, K == 1536
+#       nvfp4_quant_short_kernel<S=3>   test_nvfp4_quantize_per_tensor_bit_exact (300, 1536),
+#                                       test_dispatch_branch_bit_exact[short-1536-*]
+#   per-tensor, other K % 64 == 0
+#       nvfp4_quant_k64_kernel<false>   test_nvfp4_quantize_per_tensor_bit_exact (K 64, 256, 5120, 13824)
+#   K % 64 != 0 (per-tensor / per-row)
+#       nvfp4_quant_generic_kernel      both SHAPES tests at K = 16, 48, 80
+# nvfp4_rmsnorm_quantize (tests/test_gpu_rmsnorm.py):
+#   K == 1536 / 2048                    nvfp4_rmsnorm_quant_short_kernel<per_row, S=3 / 4>
+#   other K                             nvfp4_rmsnorm_quant_kernel<per_row>
+# mxfp8_quantize:
+#   K % 128 == 0                        mxfp8_quant_k128_kernel   test_mxfp8_quantize_bit_exact (K 128, 5120, 13824)
+#   other K % 32 == 0                   mxfp8_quant_generic_kernel test_mxfp8_quantize_bit_exact (K 32, 96, 160)
+BRANCH_CASES = [
+    # (name, M, K, per_row)
+    ("short-1024", 1, 1024, False), ("short-1024", 129, 1024, False), ("short-1024", 300, 1024, False),
+    ("short-1024", 4100, 1024, False), ("short-1536", 4100, 1536, False),
+    ("rowblock", 129, 1024, True), ("rowblock", 300, 5120, True),
+    ("k64-per-row", 4100, 1024, True), ("k64-per-row", 4100, 5120, True),
+]
+
+
+def _f16_bits(M, K, seed):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((M, K)) * 3.0).astype(np.float32)
+    x[rng.random((M, K)) < 0.001] *= 50.0
+    bits = x.astype(np.float16).view(np.uint16)
+    flat = bits.reshape(-1)
+    flat[rng.integers(0, flat.size, flat.size // 50)] = 0x8203  # negative subnormal
+    flat[rng.integers(0, flat.size, flat.size // 200)] = 0x7BFF  # 65504
+    return bits
+
+
+@pytest.mark.parametrize("name,M,K,per_row", BRANCH_CASES, ids=[f"{c[0]}-{c[1]}x{c[2]}" for c in BRANCH_CASES])
+@pytest.mark.parametrize("fmt", ["bf16", "f16"])
+@pytest.mark.parametrize("layout", ["128x4", "8x4"])
+def test_dispatch_branch_bit_exact(name, M, K, per_row, fmt, layout):
+    seed = M * 13 + K + (7 if fmt == "f16" else 0)
+    if fmt == "f16":
+        x = _f16_bits(M, K, seed)
+        xt = torch.from_numpy(np.ascontiguousarray(x)).view(torch.float16).to(DEV)
+    else:
+        x = _data(M, K, seed=seed, kind="special")
+        xt = up_bf16(x)
+    if per_row:
+        q = api.nvfp4_quantize(xt, per_row=True, sf_layout=layout)
+        gs, inv = oracle.row_global_scales(x, fmt=fmt)
+        assert np.array_equal(down(q.row_gs).view(np.uint32), gs.view(np.uint32))
+        assert np.array_equal(down(q.row_inv_gs).view(np.uint32), inv.view(np.uint32))
+        codes, sf = oracle.nvfp4_quantize(x, gs, per_row=True, fmt=fmt, layout=layout)
+    else:
+        g = np.float32(0.37109375) if M % 2 else np.float32(291.5)
+        q = api.nvfp4_quantize(xt, torch.tensor([g], device=DEV), sf_layout=layout)
+        codes, sf = oracle.nvfp4_quantize(x, g, fmt=fmt, layout=layout)
+    assert np.array_equal(down(q.codes), codes)
+    assert np.array_equal(down(q.sf), sf)
+
 
 @pytest.mark.parametrize("M,K", SHAPES)
 @pytest.mark.parametrize("gs", [1.0, 0.37109375, 291.5])

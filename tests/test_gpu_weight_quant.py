@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import oracle
+from block_scaled_precision_05_b200 import _native as nat
 from block_scaled_precision_05_b200 import api
 from block_scaled_precision_05_b200 import workloads as wl
 from tests._gpu import DEV, down, up_bf16
@@ -115,6 +116,32 @@ def test_consecutive_calls_reuse_the_workspace():
         _assert_same(f, _three_launches(ws[j // 2], api.FP8_FP4_MAX))
     for ws_t in api._WEIGHT_WS.values():
         assert int(ws_t[:4].view(torch.int32)[0]) == 0
+    assert api.device_status() == 0
+
+
+def test_workspace_left_by_a_timed_out_call_is_fit_for_the_next():
+    """A barrier wait that runs out leaves a non-zero arrival count (and stale
+    block words) in the workspace.  Each call clears the barrier words on its
+    stream before the launch, so a later call on that workspace is still
+    correct.  The stale state is written by the host here; nothing waits."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(13)
+    w = (torch.randn((3000, 5120), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn((700, 1024), generator=g, device=DEV) * 2.0).to(torch.bfloat16)
+    api.nvfp4_quantize_weight(w)  # sets up the per-device workspace
+    torch.cuda.synchronize()
+    ws = api._weight_workspace(DEV, nat.BSP_IN_BF16)
+    words = ws.view(torch.int32)
+    for stale in ((5, 3), (443, 0)):  # arrivals short of the grid, and one short of releasing
+        words[0], words[1] = stale
+        words[64:] = 0x7F7F0000  # block words of a larger amax than any here
+        f1 = api.nvfp4_quantize_weight(w)
+        words[0] = stale[0]
+        f2 = api.nvfp4_quantize_weights([w2])[0]
+        torch.cuda.synchronize()
+        _assert_same(f1, _three_launches(w, api.FP8_FP4_MAX))
+        _assert_same(f2, _three_launches(w2, api.FP8_FP4_MAX))
+        assert int(words[0]) == 0
     assert api.device_status() == 0
 
 
