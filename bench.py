@@ -88,9 +88,10 @@ def _code_only(src: str) -> str:
 KERNEL_SOURCES = {
     "nvfp4_gemm": ("gemm.cu", "bsp_device.cuh", "bsp_internal.h"),
     "mxfp8_gemm": ("gemm.cu", "bsp_device.cuh", "bsp_internal.h"),
-    "nvfp4_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h"),
-    "nvfp4_rmsnorm_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h"),
-    "mxfp8_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h"),
+    "nvfp4_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h", "norm_stats.cuh"),
+    "nvfp4_rmsnorm_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h", "norm_stats.cuh"),
+    "nvfp4_layernorm_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h", "norm_stats.cuh"),
+    "mxfp8_quantize": ("quantize.cu", "bsp_device.cuh", "bsp_internal.h", "norm_stats.cuh"),
 }
 
 
@@ -1029,7 +1030,7 @@ def main():
     ap.add_argument("--config", default="wan14")
     ap.add_argument("--sf-layout", choices=["128x4", "8x4"], default="128x4",
                     help="activation scale layout of the NVFP4 workloads (8x4: M <= 64)")
-    ap.add_argument("--norm", choices=["none", "rmsnorm"], default="none",
+    ap.add_argument("--norm", choices=["none", "rmsnorm", "layernorm"], default="none",
                     help="NVFP4 workloads: fuse a norm of the activation into the quantizer")
     ap.add_argument("--input", choices=["bf16", "f16"], default="bf16",
                     help="activation dtype of the NVFP4 workloads (f16: the bf16 values rounded to fp16)")

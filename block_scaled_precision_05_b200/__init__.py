@@ -19,7 +19,9 @@ from .api import (  # noqa: F401
     nvfp4_alpha,
     nvfp4_gemm,
     nvfp4_global_scale,
+    nvfp4_layernorm_quantize,
     nvfp4_quantize,
+    nvfp4_rmsnorm_quantize,
     nvfp4_sf_bytes,
 )
 from ._native import BSPError, LIB_PATH  # noqa: F401

@@ -24,6 +24,8 @@ BSP_IN_BF16 = 0
 BSP_IN_F16 = 1
 BSP_SF_LAYOUT_128X4 = 0
 BSP_SF_LAYOUT_8X4 = 1
+BSP_NORM_RMS = 0
+BSP_NORM_LAYER = 1
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 
@@ -60,6 +62,8 @@ SIGNATURES = {
     "nvfp4_quantize_ex": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_rmsnorm_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, ctypes.c_float, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
                                       _vp]),
+    "nvfp4_layernorm_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, ctypes.c_float, _vp, _i32, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "nvfp4_gemm_ex": (_i32, [_vp, _vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "mxfp8_quantize": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
@@ -68,6 +72,7 @@ SIGNATURES = {
     "bsp_debug_encode_e2m1": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_debug_encode_e4m3": (_i32, [_vp, _i64, _vp, _vp]),
     "bsp_debug_wait_timeout": (_i32, [_i64, _vp]),
+    "bsp_debug_norm_stats": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
 }
 
 

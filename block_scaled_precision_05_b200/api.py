@@ -324,6 +324,61 @@ def nvfp4_rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e
     return out
 
 
+def nvfp4_layernorm_quantize(x: torch.Tensor, gamma: torch.Tensor | None = None, beta: torch.Tensor | None = None,
+                             eps: float = 1e-6, global_sf: torch.Tensor | None = None, per_row: bool = False,
+                             out: NVFP4Tensor | None = None, mean_out: torch.Tensor | None = None,
+                             rstd_out: torch.Tensor | None = None) -> NVFP4Tensor:
+    """LayerNorm(x) (* gamma + beta, each optional), rounded to bf16 and
+    quantized to NVFP4 in one kernel (the normalised activation is never
+    written).  bf16 x [..., K], gamma / beta [K] or None."""
+    _require_cuda(x, gamma, beta, global_sf, mean_out, rstd_out)
+    if x.dtype != torch.bfloat16 or any(t is not None and t.dtype != torch.bfloat16 for t in (gamma, beta)):
+        raise TypeError("nvfp4_layernorm_quantize expects bf16 x, gamma and beta")
+    x2 = _as_2d(x)
+    M, K = x2.shape
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        if t is not None and (t.numel() != K or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous [{K}] tensor")
+    for name, t in (("mean_out", mean_out), ("rstd_out", rstd_out)):
+        if t is not None and (t.dtype != torch.float32 or t.numel() != M):
+            raise ValueError(f"{name} must be an fp32 [{M}] tensor")
+    dev = x2.device
+    if out is None:
+        out = NVFP4Tensor(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev), K)
+        if per_row:
+            out.row_gs = torch.empty(M, dtype=torch.float32, device=dev)
+            out.row_inv_gs = torch.empty(M, dtype=torch.float32, device=dev)
+    if not per_row and global_sf is None:
+        raise ValueError("per-tensor quantization needs global_sf (fp32 device tensor)")
+    st = nat.lib().nvfp4_layernorm_quantize(
+        _ptr(x2), M, K, x2.stride(0), _ptr(gamma), _ptr(beta), float(eps), None if per_row else _ptr(global_sf),
+        nat.BSP_SF_PER_ROW if per_row else nat.BSP_SF_PER_TENSOR,
+        _ptr(out.row_gs) if per_row else None, _ptr(out.row_inv_gs) if per_row else None, _ptr(mean_out),
+        _ptr(rstd_out), _ptr(out.codes), _ptr(out.sf), _stream())
+    nat.check(st, "nvfp4_layernorm_quantize")
+    return out
+
+
+def norm_stats(x: torch.Tensor, norm: str = "rms", exact_only: bool = False):
+    """Diagnostic: the fused norms' row statistics alone (bsp_debug_norm_stats).
+    Returns (ms,) for "rms" or (mean, var) for "layer", each fp32 [M], and the
+    int32 [M] path flags (1 where the exact integer sums decided the row)."""
+    _require_cuda(x)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("norm_stats expects bf16 x")
+    x2 = _as_2d(x)
+    M, K = x2.shape
+    dev = x2.device
+    s0 = torch.empty(M, dtype=torch.float32, device=dev)
+    s1 = torch.empty(M, dtype=torch.float32, device=dev) if norm == "layer" else None
+    path = torch.empty(M, dtype=torch.int32, device=dev)
+    kind = {"rms": nat.BSP_NORM_RMS, "layer": nat.BSP_NORM_LAYER}[norm]
+    nat.check(nat.lib().bsp_debug_norm_stats(_ptr(x2), M, K, x2.stride(0), kind, int(exact_only), _ptr(s0), _ptr(s1),
+                                             _ptr(path), _stream()), "bsp_debug_norm_stats")
+    return ((s0,) if s1 is None else (s0, s1)), path
+
+
 def mxfp8_quantize(x: torch.Tensor, out: MXFP8Tensor | None = None) -> MXFP8Tensor:
     """Quantize bf16 [..., K] to MXFP8 along K (leading dims flattened)."""
     _require_cuda(x)
@@ -447,6 +502,15 @@ class NVFP4Linear:
         result as `pre_quantized` (the fused norm+quant producer)."""
         return nvfp4_rmsnorm_quantize(coerce_bf16(x), coerce_bf16(gamma).contiguous(), eps,
                                       None if self.per_token else self.gs_x, per_row=self.per_token)
+
+    def layernorm_quantize_input(self, x: torch.Tensor, gamma: torch.Tensor | None = None,
+                                 beta: torch.Tensor | None = None, eps: float = 1e-6) -> NVFP4Tensor:
+        """LayerNorm(x) (* gamma + beta) quantized for this layer in one kernel:
+        pass the result as `pre_quantized` (the fused norm+quant producer)."""
+        g = None if gamma is None else coerce_bf16(gamma).contiguous()
+        b = None if beta is None else coerce_bf16(beta).contiguous()
+        return nvfp4_layernorm_quantize(coerce_bf16(x), g, b, eps, None if self.per_token else self.gs_x,
+                                        per_row=self.per_token)
 
     def __call__(self, x: torch.Tensor, pre_quantized: NVFP4Tensor | None = None,
                  out_dtype: torch.dtype = torch.bfloat16, sf_layout: str = "128x4") -> torch.Tensor:

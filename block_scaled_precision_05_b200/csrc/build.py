@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(PKG, "libbsp.so")
 SOURCES = ["common.cu", "quantize.cu", "gemm.cu"]
-HEADERS = ["bsp_device.cuh", "bsp_internal.h"]
+HEADERS = ["bsp_device.cuh", "bsp_internal.h", "norm_stats.cuh"]
 
 
 def nvcc() -> str:

@@ -26,6 +26,7 @@
 
 #include "bsp_device.cuh"
 #include "bsp_internal.h"
+#include "norm_stats.cuh"
 
 namespace bsp {
 namespace {
@@ -471,40 +472,24 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// RMSNorm fused into the NVFP4 quantizer (the producer of a pre-quantized
+// Norms fused into the NVFP4 quantizer (the producer of a pre-quantized
 // activation: hao-ai-lab-FastVideo nvfp4_config.py, NVFP4QuantizeMethod.apply
 // with `pre_quantized` from a fused norm+quant call).  Per row:
-//   ms   = mean(x^2)  (relative error <= 2^-24: pairs of exact squares added in
-//          fp32, the pair sums in fp64, one rounding to fp32 at the end)
-//   rstd = fl32(1 / sqrt(fl32(ms + eps)))     (correctly rounded)
-//   y_k  = bf16(fl32(fl32(x_k * rstd) * gamma_k))
-// and y is quantized exactly as nvfp4_quantize quantizes a bf16 input, so the
-// result equals RMSNorm to bf16 followed by nvfp4_quantize, without writing y.
-// One warp per row: pass 1 the sum of squares, pass 2 (per-token scales) the
-// row amax of y, pass 3 the groups; passes 2 and 3 re-read the row from cache.
+//   RMSNorm   ms = mean(x^2), rstd = fl32(1 / sqrt(fl32(ms + eps)))
+//             y_k = bf16(fl32(fl32(x_k * rstd) * gamma_k))
+//   LayerNorm mean, var = the row's mean and population variance,
+//             rstd = fl32(1 / sqrt(fl32(var + eps)))
+//             y_k = bf16(fl32(fl32(fl32(fl32(x_k - mean) * rstd) * gamma_k) + beta_k))
+//             (gamma 1 and beta -0 when absent: both are exact identities)
+// with the statistics the exact values rounded once to fp32 (norm_stats.cuh),
+// and rstd correctly rounded.  y is then quantized exactly as nvfp4_quantize
+// quantizes a bf16 input, so the result equals the norm to bf16 followed by
+// nvfp4_quantize, without writing y.  One warp per row.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ double warp_sum_f64(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-  return v;
-}
+constexpr int kNormWarps = kQuantThreads / 32;
+constexpr uint32_t kBf16OnePair = 0x3F803F80u, kBf16NegZeroPair = 0x80008000u;
 
-// Sum of squares of 8 bf16 values: the squares of a pair are added with one
-// fp32 rounding (fma of the exact second square onto the exact first), the
-// four pair sums in fp64.  Relative error <= 2^-24 (all terms are
-// non-negative), at half the fp32-to-fp64 conversions of a per-element fp64 sum.
-__device__ __forceinline__ double sumsq8(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  double s = 0.0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = InBf16::values2(w[i]);
-    s += static_cast<double>(__fmaf_rn(f.y, f.y, __fmul_rn(f.x, f.x)));
-  }
-  return s;
-}
-
-// Eight normalised outputs as bf16 pairs: bf16(fl32(fl32(x * rstd) * gamma)).
+// Eight normalised outputs as bf16 pairs (RMSNorm).
 __device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, float rstd) {
   const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
   const float2 r2 = make_float2(rstd, rstd);
@@ -519,19 +504,112 @@ __device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, floa
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <class L, bool kPerRow>
-__global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
+// Eight normalised outputs as bf16 pairs (LayerNorm).
+__device__ __forceinline__ uint4 layernorm8(const uint4& xv, const uint4& gv, const uint4& bv, float mean,
+                                            float rstd) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+  const float2 nm2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 d = __fadd2_rn(InBf16::values2(xw[i]), nm2);  // x - mean, rounded once
+    const float2 y = __fadd2_rn(__fmul2_rn(__fmul2_rn(d, r2), InBf16::values2(gw[i])), InBf16::values2(bw[i]));
+    const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
+    memcpy(&o[i], &h, 4);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The per-row parameters of either norm and its elementwise map.
+struct NormRow {
+  float mean;  // LayerNorm only
+  float rstd;
+};
+
+template <bool kLN>
+__device__ __forceinline__ uint4 norm8(const uint4& xv, const uint4& gv, const uint4& bv, const NormRow& p) {
+  if constexpr (kLN)
+    return layernorm8(xv, gv, bv, p.mean, p.rstd);
+  else
+    return rmsnorm8(xv, gv, p.rstd);
+}
+
+// Exact row statistics from the row in global memory (the rare path; the row
+// is re-read): ms, or mean and var.
+template <bool kLN>
+__device__ __noinline__ void norm_row_exact(const uint16_t* __restrict__ row, int64_t K,
+                                            normstats::ExactSums* xs, float* a, float* b) {
+  const uint32_t lane = lane_id();
+  normstats::exact_clear(xs);
+  for (int64_t g = lane; g < (K >> 4); g += 32) {
+    normstats::exact_add8(xs, ldg16(row + g * 16), kLN);
+    normstats::exact_add8(xs, ldg16(row + g * 16 + 8), kLN);
+  }
+  __syncwarp();
+  float ea = 0.0f, eb = 0.0f;
+  if (lane == 0) {
+    if constexpr (kLN)
+      normstats::exact_mean_var(xs, static_cast<uint32_t>(K), &ea, &eb);
+    else
+      ea = normstats::exact_ms(xs, static_cast<uint32_t>(K));
+  }
+  *a = __shfl_sync(kFull, ea, 0);
+  *b = __shfl_sync(kFull, eb, 0);
+  __syncwarp();
+}
+
+// Row statistics.  `each(f)` applies f to each of this lane's 16-byte chunks
+// of the row (any order; the chunks of the 32 lanes cover the row once);
+// `row` is the row in global memory, re-read by the exact path.
+template <bool kLN, class Each>
+__device__ __forceinline__ NormRow norm_row_stats(Each each, const uint16_t* row, int64_t K, double rK, float eps,
+                                                  normstats::ExactSums* xs) {
+  NormRow p;
+  if constexpr (!kLN) {
+    double acc = 0.0;
+    each([&](const uint4& v) { acc = normstats::sumsq8(v, acc); });
+    acc = normstats::warp_sum(acc);
+    float ms, unused;
+    if (!normstats::ms_fast(acc, K, rK, &ms)) norm_row_exact<false>(row, K, xs, &ms, &unused);  // warp-uniform
+    p.mean = 0.0f;
+    p.rstd = __frsqrt_rn(__fadd_rn(ms, eps));
+  } else {
+    double s1 = 0.0, s2 = 0.0;
+    each([&](const uint4& v) { normstats::sums8(v, s1, s2); });
+    s1 = normstats::warp_sum(s1);
+    s2 = normstats::warp_sum(s2);
+    float mean, var;
+    if (!normstats::ln_fast(s1, s2, K, rK, &mean, &var)) norm_row_exact<true>(row, K, xs, &mean, &var);  // warp-uniform
+    p.mean = mean;
+    p.rstd = __frsqrt_rn(__fadd_rn(var, eps));
+  }
+  return p;
+}
+
+__device__ __forceinline__ uint4 ldg16_or(const uint16_t* p, uint32_t fill) {
+  return p ? ldg16(p) : make_uint4(fill, fill, fill, fill);
+}
+
+// Any K % 16 == 0: the statistics pass(es), then (per-token scales) the row
+// amax of y, then the groups; the later passes re-read the row from cache.
+template <class L, bool kPerRow, bool kLN>
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const uint16_t* __restrict__ gamma,
-    float eps, const float* __restrict__ gs_ptr, float* __restrict__ row_gs, float* __restrict__ row_inv,
-    float* __restrict__ row_rstd, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+    const uint16_t* __restrict__ beta, float eps, const float* __restrict__ gs_ptr, float* __restrict__ row_gs,
+    float* __restrict__ row_inv, float* __restrict__ row_mean, float* __restrict__ row_rstd,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
   allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   const uint32_t lane = lane_id();
   const int64_t groups = K >> 4, cols4 = (groups + 3) & ~int64_t(3);
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+  const double rK = 1.0 / static_cast<double>(K);
   __shared__ float inv_tab[256];
+  __shared__ normstats::ExactSums xsum[kNormWarps];
   if constexpr (!kPerRow) build_inv_table(inv_tab, gs_tensor);
+  normstats::ExactSums* xs = &xsum[threadIdx.x >> 5];
+  const uint16_t* bt = kLN ? beta : nullptr;
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const int64_t sfb_row = L::row_base(r, cols4 >> 2);
@@ -540,21 +618,26 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
       continue;
     }
     const uint16_t* row = x + r * ld_x;
-    double acc = 0.0;
-    for (int64_t g = lane; g < groups; g += 32) acc += sumsq8(ldg16(row + g * 16)) + sumsq8(ldg16(row + g * 16 + 8));
-    acc = warp_sum_f64(acc);
-    const float ms = __double2float_rn(acc / static_cast<double>(K));
-    const float rstd = __frsqrt_rn(__fadd_rn(ms, eps));
-    if (row_rstd != nullptr && lane == 0) row_rstd[r] = rstd;
-
+    auto each = [&](auto f) {
+      for (int64_t g = lane; g < groups; g += 32) {
+        f(ldg16(row + g * 16));
+        f(ldg16(row + g * 16 + 8));
+      }
+    };
+    const NormRow p = norm_row_stats<kLN>(each, row, K, rK, eps, xs);
+    if (lane == 0) {
+      if (row_rstd) row_rstd[r] = p.rstd;
+      if (kLN && row_mean) row_mean[r] = p.mean;
+    }
+    auto y8 = [&](int64_t c) {  // normalised elements [c, c + 8) as bf16 pairs
+      return norm8<kLN>(ldg16(row + c), ldg16_or(gamma ? gamma + c : nullptr, kBf16OnePair),
+                        ldg16_or(bt ? bt + c : nullptr, kBf16NegZeroPair), p);
+    };
     float gs = gs_tensor;
     if (kPerRow) {
       uint32_t mag = 0;
-      for (int64_t g = lane; g < groups; g += 32) {
-        const uint4 y0 = rmsnorm8(ldg16(row + g * 16), ldg16(gamma + g * 16), rstd);
-        const uint4 y1 = rmsnorm8(ldg16(row + g * 16 + 8), ldg16(gamma + g * 16 + 8), rstd);
-        mag = max(mag, max(max_sane_mag8<InBf16>(y0), max_sane_mag8<InBf16>(y1)));
-      }
+      for (int64_t g = lane; g < groups; g += 32)
+        mag = max(mag, max(max_sane_mag8<InBf16>(y8(g * 16)), max_sane_mag8<InBf16>(y8(g * 16 + 8))));
       mag = warp_max(mag);
       gs = global_scale_from_mag<InBf16>(mag);
       if (lane == 0) {
@@ -565,8 +648,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
     for (int64_t c = lane; c < cols4; c += 32) {
       uint32_t sfb = 0;
       if (c < groups) {
-        const uint4 y0 = rmsnorm8(ldg16(row + c * 16), ldg16(gamma + c * 16), rstd);
-        const uint4 y1 = rmsnorm8(ldg16(row + c * 16 + 8), ldg16(gamma + c * 16 + 8), rstd);
+        const uint4 y0 = y8(c * 16), y1 = y8(c * 16 + 8);
         float inv;
         nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, kPerRow ? nullptr : inv_tab);
         uint2 w;
@@ -582,20 +664,22 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_rmsnorm_quant_kernel(
 // K = 512 * S (S = 3, 4: the Wan-1.3B hidden size 1536 among them): the same
 // arithmetic with every row read from DRAM once and kept in registers.  Lane
 // l holds elements [512 s + 16 l, 512 s + 16 l + 16) of the row for s < S (one
-// group of 16 per slab); gamma is re-read per row (it stays in L1).  A warp
-// loads R rows before working on the first, like nvfp4_quant_short_kernel.
-// Rows [M, Mp) are scale padding: y = 0, so their scale bytes are 0.
+// group of 16 per slab); gamma (and beta) are re-read per row (they stay in
+// L1).  A warp loads R rows before working on the first, like
+// nvfp4_quant_short_kernel.  Rows [M, Mp) are scale padding: y = 0, so their
+// scale bytes are 0.
 #ifndef BSP_RMSNORM_ROWS
 #define BSP_RMSNORM_ROWS 1  // rows in flight per warp at K = 1536
 #endif
 #ifndef BSP_RMSNORM_MIN_BLOCKS
 #define BSP_RMSNORM_MIN_BLOCKS 3  // resident blocks per SM the K = 1536 kernel is compiled for
 #endif
-template <bool kPerRow, int S, int R, int kMinBlocks>
-__global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant_short_kernel(
-    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const uint16_t* __restrict__ gamma, float eps,
-    const float* __restrict__ gs_ptr, float* __restrict__ row_gs, float* __restrict__ row_inv,
-    float* __restrict__ row_rstd, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+template <bool kPerRow, bool kLN, int S, int R, int kMinBlocks>
+__global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_short_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, const uint16_t* __restrict__ gamma,
+    const uint16_t* __restrict__ beta, float eps, const float* __restrict__ gs_ptr, float* __restrict__ row_gs,
+    float* __restrict__ row_inv, float* __restrict__ row_mean, float* __restrict__ row_rstd,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
   using L = Sf128x4;
   allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
   constexpr int64_t K = 512 * S;
@@ -603,10 +687,14 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float gs_tensor = kPerRow ? 1.0f : __ldg(gs_ptr);
+  constexpr double rK = 1.0 / static_cast<double>(K);
   __shared__ float inv_tab[256];
+  __shared__ normstats::ExactSums xsum[kNormWarps];
   if constexpr (!kPerRow) build_inv_table(inv_tab, gs_tensor);
+  normstats::ExactSums* xs = &xsum[threadIdx.x >> 5];
   const bool quad_lead = (lane & 3u) == 0u;
-  const uint16_t* gp = gamma + lane * 16;  // re-read per row from L1 (registers go to rows in flight)
+  const uint16_t* gp = gamma ? gamma + lane * 16 : nullptr;  // re-read per row from L1
+  const uint16_t* bp = (kLN && beta) ? beta + lane * 16 : nullptr;
   for (int64_t r0 = R * warp; r0 < Mp; r0 += R * nwarps) {
     uint4 v[R][S][2];
 #pragma unroll
@@ -625,22 +713,32 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant
       const int64_t r = r0 + h;
       if (r >= Mp) break;
       const bool live = r < M;
-      double acc = 0.0;
+      NormRow p{0.0f, 0.0f};
+      if (live) {  // warp-uniform
+        auto each = [&](auto f) {
 #pragma unroll
-      for (int s = 0; s < S; ++s) acc += sumsq8(v[h][s][0]) + sumsq8(v[h][s][1]);
-      acc = warp_sum_f64(acc);
-      const float ms = __double2float_rn(acc / static_cast<double>(K));
-      const float rstd = __frsqrt_rn(__fadd_rn(ms, eps));
-      if (live && row_rstd != nullptr && lane == 0) row_rstd[r] = rstd;
-      const float rs = live ? rstd : 0.0f;
+          for (int s = 0; s < S; ++s) {
+            f(v[h][s][0]);
+            f(v[h][s][1]);
+          }
+        };
+        p = norm_row_stats<kLN>(each, x + r * ld_x, K, rK, eps, xs);
+        if (lane == 0) {
+          if (row_rstd) row_rstd[r] = p.rstd;
+          if (kLN && row_mean) row_mean[r] = p.mean;
+        }
+      }
       // y is recomputed where it is needed rather than held (register pressure)
+      auto y8 = [&](int s, int half) {
+        return norm8<kLN>(v[h][s][half], ldg16_or(gp ? gp + s * 512 + half * 8 : nullptr, kBf16OnePair),
+                          ldg16_or(bp ? bp + s * 512 + half * 8 : nullptr, kBf16NegZeroPair), p);
+      };
       float gs = gs_tensor;
       if (kPerRow) {
         uint32_t mag = 0;
 #pragma unroll
         for (int s = 0; s < S; ++s)
-          mag = max(mag, max(max_sane_mag8<InBf16>(rmsnorm8(v[h][s][0], ldg16(gp + s * 512), rs)),
-                             max_sane_mag8<InBf16>(rmsnorm8(v[h][s][1], ldg16(gp + s * 512 + 8), rs))));
+          mag = max(mag, max(max_sane_mag8<InBf16>(y8(s, 0)), max_sane_mag8<InBf16>(y8(s, 1))));
         mag = warp_max(mag);
         gs = global_scale_from_mag<InBf16>(mag);
         if (live && lane == 0) {
@@ -652,8 +750,7 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant
       uint8_t* sp = sf + L::row_base(r, K >> 6) + (lane >> 2) * L::kTileBytes;
 #pragma unroll
       for (int s = 0; s < S; ++s) {
-        const uint4 y0 = rmsnorm8(v[h][s][0], ldg16(gp + s * 512), rs);
-        const uint4 y1 = rmsnorm8(v[h][s][1], ldg16(gp + s * 512 + 8), rs);
+        const uint4 y0 = y8(s, 0), y1 = y8(s, 1);
         uint32_t sfb;
         float inv;
         nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, kPerRow ? nullptr : inv_tab);
@@ -667,6 +764,55 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_rmsnorm_quant
         if (quad_lead)
           *reinterpret_cast<uint32_t*>(sp + s * 8 * L::kTileBytes) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
+    }
+  }
+}
+
+// Row statistics alone (diagnostic entry bsp_debug_norm_stats): per row the
+// RMSNorm ms, or the LayerNorm mean and var, each as the fast decision with its
+// exact fallback (exact_only = false) or always from the exact sums; path[r]
+// = 1 where the exact sums were used.
+template <bool kLN>
+__global__ void __launch_bounds__(kQuantThreads) norm_stats_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                                    int64_t K, int64_t ld_x, bool exact_only,
+                                                                    float* __restrict__ stat0,
+                                                                    float* __restrict__ stat1, int* __restrict__ path) {
+  const uint32_t lane = lane_id();
+  const int64_t groups = K >> 4;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const double rK = 1.0 / static_cast<double>(K);
+  __shared__ normstats::ExactSums xsum[kNormWarps];
+  normstats::ExactSums* xs = &xsum[threadIdx.x >> 5];
+  for (int64_t r = warp; r < M; r += nwarps) {
+    const uint16_t* row = x + r * ld_x;
+    auto each = [&](auto f) {
+      for (int64_t g = lane; g < groups; g += 32) {
+        f(ldg16(row + g * 16));
+        f(ldg16(row + g * 16 + 8));
+      }
+    };
+    float a = 0.0f, b = 0.0f;
+    bool fast = false;
+    if (!exact_only) {
+      if constexpr (kLN) {
+        double s1 = 0.0, s2 = 0.0;
+        each([&](const uint4& v) { normstats::sums8(v, s1, s2); });
+        s1 = normstats::warp_sum(s1);
+        s2 = normstats::warp_sum(s2);
+        fast = normstats::ln_fast(s1, s2, K, rK, &a, &b);
+      } else {
+        double acc = 0.0;
+        each([&](const uint4& v) { acc = normstats::sumsq8(v, acc); });
+        acc = normstats::warp_sum(acc);
+        fast = normstats::ms_fast(acc, K, rK, &a);
+      }
+    }
+    if (!fast) norm_row_exact<kLN>(row, K, xs, &a, &b);
+    if (lane == 0) {
+      stat0[r] = a;
+      if (stat1) stat1[r] = b;
+      if (path) path[r] = fast ? 0 : 1;
     }
   }
 }
@@ -1245,6 +1391,61 @@ int static_weight_ws(const DeviceInfo& dev, void** out) {
   return BSP_OK;
 }
 
+// Largest K of the fused norms: the exact path's digit counts and its 32-bit
+// divisor (K for the mean of squares, K^2 for the variance) bound it.
+constexpr int64_t norm_max_k(bool ln) { return ln ? 32768 : (int64_t(1) << 20); }
+
+template <bool kLN>
+int run_norm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const uint16_t* gamma,
+                      const uint16_t* beta, float eps, const float* global_sf, int sf_mode, float* row_gs,
+                      float* row_inv_gs, float* row_mean, float* row_rstd, uint8_t* codes, uint8_t* sf,
+                      cudaStream_t stream) {
+  if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K || K > norm_max_k(kLN)) return BSP_ERR_INVALID_ARG;
+  if (sf_mode != BSP_SF_PER_TENSOR && sf_mode != BSP_SF_PER_ROW) return BSP_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !(eps <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
+  if (M == 0) return BSP_OK;
+  if (!x || !codes || !sf || (sf_mode == BSP_SF_PER_TENSOR && !global_sf)) return BSP_ERR_INVALID_ARG;
+  if (!aligned16(x) || (gamma && !aligned16(gamma)) || (beta && !aligned16(beta)) || !aligned16(codes) ||
+      !aligned16(sf) || ld_x % 8 != 0)
+    return BSP_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  int st = current_device(&dev);
+  if (st != BSP_OK) return st;
+  const int64_t Mp = round_up(M, 128);
+  const bool per_row = sf_mode == BSP_SF_PER_ROW;
+  float* rg = per_row ? row_gs : nullptr;
+  float* ri = per_row ? row_inv_gs : nullptr;
+  // K = 1536 / 2048: rows in registers (at K = 1024 the multi-pass kernel
+  // below measured as fast)
+  if (K == 1536 || K == 2048) {
+    auto launch = [&](auto k, int64_t rows_per_warp) {
+      k<<<grid_for_rows(dev, k, ceil_div(Mp, rows_per_warp)), kQuantThreads, 0, stream>>>(
+          x, M, Mp, ld_x, gamma, beta, eps, global_sf, rg, ri, row_mean, row_rstd, codes, sf);
+    };
+    switch (K / 512) {
+#define BSP_NORM_CASE(S_, R_, B_)                                                                      \
+  case S_:                                                                                            \
+    per_row ? launch(nvfp4_norm_quant_short_kernel<true, kLN, S_, R_, B_>, R_)                        \
+            : launch(nvfp4_norm_quant_short_kernel<false, kLN, S_, R_, B_>, R_);                      \
+    break;
+      BSP_NORM_CASE(3, BSP_RMSNORM_ROWS, BSP_RMSNORM_MIN_BLOCKS)
+      BSP_NORM_CASE(4, 1, 2)
+#undef BSP_NORM_CASE
+    }
+    return launch_status();
+  }
+  if (per_row) {
+    auto k = nvfp4_norm_quant_kernel<Sf128x4, true, kLN>;
+    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, beta, eps, global_sf, rg, ri,
+                                                               row_mean, row_rstd, codes, sf);
+  } else {
+    auto k = nvfp4_norm_quant_kernel<Sf128x4, false, kLN>;
+    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, beta, eps, global_sf, rg, ri,
+                                                               row_mean, row_rstd, codes, sf);
+  }
+  return launch_status();
+}
+
 }  // namespace
 }  // namespace bsp
 
@@ -1282,46 +1483,35 @@ int nvfp4_quantize_ex(const uint16_t* x, int x_dtype, int64_t M, int64_t K, int6
 int nvfp4_rmsnorm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const uint16_t* gamma, float eps,
                            const float* global_sf, int sf_mode, float* row_gs, float* row_inv_gs, float* row_rstd,
                            uint8_t* codes, uint8_t* sf, bsp_stream_t stream) {
-  if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K) return BSP_ERR_INVALID_ARG;
-  if (sf_mode != BSP_SF_PER_TENSOR && sf_mode != BSP_SF_PER_ROW) return BSP_ERR_INVALID_ARG;
-  if (!(eps >= 0.0f) || !(eps <= 3.4028234663852886e38f)) return BSP_ERR_INVALID_ARG;
+  if (!gamma && M > 0) return BSP_ERR_INVALID_ARG;
+  return run_norm_quantize<false>(x, M, K, ld_x, gamma, nullptr, eps, global_sf, sf_mode, row_gs, row_inv_gs, nullptr,
+                                  row_rstd, codes, sf, stream);
+}
+
+int nvfp4_layernorm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const uint16_t* gamma,
+                             const uint16_t* beta, float eps, const float* global_sf, int sf_mode, float* row_gs,
+                             float* row_inv_gs, float* row_mean, float* row_rstd, uint8_t* codes, uint8_t* sf,
+                             bsp_stream_t stream) {
+  return run_norm_quantize<true>(x, M, K, ld_x, gamma, beta, eps, global_sf, sf_mode, row_gs, row_inv_gs, row_mean,
+                                 row_rstd, codes, sf, stream);
+}
+
+int bsp_debug_norm_stats(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, int norm, int exact_only, float* stat0,
+                         float* stat1, int* path, bsp_stream_t stream) {
+  if (norm != BSP_NORM_RMS && norm != BSP_NORM_LAYER) return BSP_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || K % 16 != 0 || ld_x < K || K > norm_max_k(norm == BSP_NORM_LAYER)) return BSP_ERR_INVALID_ARG;
   if (M == 0) return BSP_OK;
-  if (!x || !gamma || !codes || !sf || (sf_mode == BSP_SF_PER_TENSOR && !global_sf)) return BSP_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(gamma) || !aligned16(codes) || !aligned16(sf) || ld_x % 8 != 0)
-    return BSP_ERR_ALIGNMENT;
+  if (!x || !stat0 || (norm == BSP_NORM_LAYER && !stat1)) return BSP_ERR_INVALID_ARG;
+  if (!aligned16(x) || ld_x % 8 != 0) return BSP_ERR_ALIGNMENT;
   DeviceInfo dev;
   int st = current_device(&dev);
   if (st != BSP_OK) return st;
-  const int64_t Mp = round_up(M, 128);
-  // K = 1536 / 2048: rows in registers (at K = 1024 the three-pass kernel below
-  // measured as fast)
-  if (K == 1536 || K == 2048) {
-    const bool per_row = sf_mode == BSP_SF_PER_ROW;
-    auto launch = [&](auto k, int64_t rows_per_warp) {
-      k<<<grid_for_rows(dev, k, ceil_div(Mp, rows_per_warp)), kQuantThreads, 0, stream>>>(
-          x, M, Mp, ld_x, gamma, eps, global_sf, per_row ? row_gs : nullptr, per_row ? row_inv_gs : nullptr, row_rstd,
-          codes, sf);
-    };
-    switch (K / 512) {
-#define BSP_RMS_CASE(S_, R_, B_)                                                                        \
-  case S_:                                                                                             \
-    per_row ? launch(nvfp4_rmsnorm_quant_short_kernel<true, S_, R_, B_>, R_)                           \
-            : launch(nvfp4_rmsnorm_quant_short_kernel<false, S_, R_, B_>, R_);                         \
-    break;
-      BSP_RMS_CASE(3, BSP_RMSNORM_ROWS, BSP_RMSNORM_MIN_BLOCKS)
-      BSP_RMS_CASE(4, 1, 2)
-#undef BSP_RMS_CASE
-    }
-    return launch_status();
-  }
-  if (sf_mode == BSP_SF_PER_ROW) {
-    auto k = nvfp4_rmsnorm_quant_kernel<Sf128x4, true>;
-    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, row_gs,
-                                                               row_inv_gs, row_rstd, codes, sf);
+  if (norm == BSP_NORM_LAYER) {
+    auto k = norm_stats_kernel<true>;
+    k<<<grid_for_rows(dev, k, M), kQuantThreads, 0, stream>>>(x, M, K, ld_x, exact_only != 0, stat0, stat1, path);
   } else {
-    auto k = nvfp4_rmsnorm_quant_kernel<Sf128x4, false>;
-    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, eps, global_sf, nullptr,
-                                                               nullptr, row_rstd, codes, sf);
+    auto k = norm_stats_kernel<false>;
+    k<<<grid_for_rows(dev, k, M), kQuantThreads, 0, stream>>>(x, M, K, ld_x, exact_only != 0, stat0, nullptr, path);
   }
   return launch_status();
 }

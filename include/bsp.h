@@ -82,6 +82,12 @@ enum {
     BSP_SF_LAYOUT_8X4 = 1
 };
 
+/* Norms of the fused norm + quantize producers (bsp_debug_norm_stats). */
+enum {
+    BSP_NORM_RMS = 0,
+    BSP_NORM_LAYER = 1
+};
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *bsp_status_string(int status);
 
@@ -313,23 +319,51 @@ int nvfp4_quantize_ex(const uint16_t *x, int x_dtype, int64_t M, int64_t K, int6
  * fused norm+quant call.  The pages name the fused call but not its norm; this
  * is RMSNorm with a weight, whose normalised output is quantized as if it had
  * been written as bf16 and passed to nvfp4_quantize.  Per row m:
- *   ms   = mean_k x_k^2  (relative error <= 2^-24: pairs of exact squares
- *          added in fp32, pair sums in fp64 in any order, one rounding to fp32)
- *   rstd = fl32(1 / sqrt(fl32(ms + eps)))   (correctly rounded from that ms, so
- *          within 2 ulp of rstd from the exact mean)
+ *   ms   = mean_k x_k^2, the exact mean rounded once to fp32 (an fp64 sum with
+ *          a proven error bound decides it, or, where that bound does not
+ *          decide the rounding, exact integer sums)
+ *   rstd = fl32(1 / sqrt(fl32(ms + eps)))   (correctly rounded)
  *   y_k  = bf16(fl32(fl32(x_k * rstd) * gamma_k))
  *   then y is quantized as nvfp4_quantize does (per-tensor global_sf, or per
  *   row gs[m] from the row amax of y), without y being stored.
  *   x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf:
- *              as nvfp4_quantize (bf16 x)
+ *              as nvfp4_quantize (bf16 x); K <= 2^20
  *   gamma    : bf16 [K], 16-byte aligned
  *   eps      : host fp32, finite and >= 0
  *   row_rstd : fp32 [M] receives rstd of each row (may be NULL)
- * Errors as nvfp4_quantize; eps negative or not finite -> INVALID_ARG. */
+ * Errors as nvfp4_quantize; eps negative or not finite, K > 2^20 ->
+ * INVALID_ARG. */
 int nvfp4_rmsnorm_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
                            const uint16_t *gamma, float eps, const float *global_sf, int sf_mode,
                            float *row_gs, float *row_inv_gs, float *row_rstd, uint8_t *codes,
                            uint8_t *sf, bsp_stream_t stream);
+
+/* LayerNorm fused into the NVFP4 quantizer: the same producer as
+ * nvfp4_rmsnorm_quantize with the norm of the Wan-2.1 blocks whose attention
+ * and FFN projections the pages quantize (nvfp4_qat_config.py
+ * DEFAULT_FP4_LAYERS; nvfp4_config.py names the fused norm+quant call, not its
+ * norm).  Per row m:
+ *   mean = (1/K) sum_k x_k          the exact mean rounded once to fp32
+ *   var  = (1/K) sum_k (x_k - mu)^2 with mu the exact mean: the exact
+ *                                   population variance rounded once to fp32
+ *   rstd = fl32(1 / sqrt(fl32(var + eps)))   (correctly rounded)
+ *   y_k  = bf16(fl32(fl32(fl32(fl32(x_k - mean) * rstd) * gamma_k) + beta_k))
+ *          (gamma and beta optional: absent, their steps are left out)
+ *   then y is quantized as nvfp4_quantize does, without y being stored.
+ *   x, M, K, ld_x, global_sf, sf_mode, row_gs, row_inv_gs, codes, sf:
+ *              as nvfp4_quantize (bf16 x); K <= 32768
+ *   gamma    : bf16 [K], 16-byte aligned, or NULL (no scale)
+ *   beta     : bf16 [K], 16-byte aligned, or NULL (no shift)
+ *   eps      : host fp32, finite and >= 0
+ *   row_mean, row_rstd : fp32 [M] receive mean and rstd of each row (each
+ *              may be NULL)
+ * Errors as nvfp4_quantize; eps negative or not finite, K > 32768 ->
+ * INVALID_ARG. */
+int nvfp4_layernorm_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x,
+                             const uint16_t *gamma, const uint16_t *beta, float eps,
+                             const float *global_sf, int sf_mode, float *row_gs, float *row_inv_gs,
+                             float *row_mean, float *row_rstd, uint8_t *codes, uint8_t *sf,
+                             bsp_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * NVFP4 GEMM (nvfp4_qat_config.py, NVFP4QATQuantizeMethod.apply:
@@ -412,6 +446,16 @@ int bsp_debug_encode_e4m3(const float *v, int64_t n, uint8_t *bytes, bsp_stream_
  * with a limit of `limit_ns` nanoseconds (1e3 .. 1e10).  The wait runs out and
  * sets the error word, so bsp_device_status then returns BSP_ERR_TIMEOUT. */
 int bsp_debug_wait_timeout(int64_t limit_ns, bsp_stream_t stream);
+/* The row statistics of the fused norms alone, as those kernels decide them:
+ * per row r of bf16 x [M, K] (row stride ld_x), norm BSP_NORM_RMS writes
+ * stat0[r] = ms (the exact mean of squares rounded to fp32), BSP_NORM_LAYER
+ * writes stat0[r] = mean and stat1[r] = var (each exact, rounded to fp32).
+ * exact_only != 0 skips the fp64 decision and always takes the exact integer
+ * sums; path (int [M], or NULL) receives 0 where the fp64 decision settled the
+ * row and 1 where the exact sums did.  K % 16 == 0 and the K limits of the
+ * fused calls; errors as nvfp4_rmsnorm_quantize. */
+int bsp_debug_norm_stats(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int norm,
+                         int exact_only, float *stat0, float *stat1, int *path, bsp_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -382,7 +382,12 @@ def _rn_f32_ratio(p: int, q: int) -> np.float32:
 
 
 def _rsqrt_rn32(t: np.float32) -> np.float32:
-    """RN32(1/sqrt(t)) for a positive fp32 t, decided exactly."""
+    """RN32(1/sqrt(t)) for an fp32 t >= 0, decided exactly (IEEE: +0 for
+    t = +inf, +inf for t = 0)."""
+    if np.isinf(t):
+        return np.float32(0.0)
+    if t == 0:
+        return np.float32(np.inf)
     tf = Fraction(float(t))
     c = np.float32(1.0 / math.sqrt(float(t)))
     for _ in range(4):  # the fp64 estimate is within an fp32 ulp: at most one step either way
@@ -441,11 +446,10 @@ def rmsnorm_bf16(x: np.ndarray, gamma: np.ndarray, rstd: np.ndarray) -> np.ndarr
     return bf16_round(y.astype(np.float64))
 
 
-def rmsnorm_quantize(x: np.ndarray, gamma: np.ndarray, eps: float, gs=None, per_row: bool = False, rstd=None):
-    """RMSNorm to bf16, then NVFP4 quantization.  `rstd` may be given (e.g. the
-    values a kernel reports) to check everything downstream of the reduction.
+def rmsnorm_quantize(x: np.ndarray, gamma: np.ndarray, eps: float, gs=None, per_row: bool = False):
+    """RMSNorm to bf16, then NVFP4 quantization.
     Returns (codes, sf, rstd, row_gs or None, row_inv or None)."""
-    rstd = rmsnorm_rstd(x, eps) if rstd is None else np.asarray(rstd, np.float32)
+    rstd = rmsnorm_rstd(x, eps)
     y = rmsnorm_bf16(x, gamma, rstd)
     if per_row:
         g, inv = row_global_scales(y)
@@ -453,3 +457,81 @@ def rmsnorm_quantize(x: np.ndarray, gamma: np.ndarray, eps: float, gs=None, per_
         return codes, sf, rstd, g, inv
     codes, sf = nvfp4_quantize(y, gs)
     return codes, sf, rstd, None, None
+
+
+# --------------------------------------------------------------------------- LayerNorm before the quantizer
+# The same producer with the norm of the Wan-2.1 blocks whose projections the
+# pages quantize (hao-ai-lab-FastVideo nvfp4_qat_config.py, DEFAULT_FP4_LAYERS;
+# nvfp4_config.py names the fused norm+quant call, not its norm).  Reading:
+#   mean = (1/K) sum_k x_k                      (exact, then rounded once to fp32)
+#   var  = (1/K) sum_k (x_k - mean_exact)^2     (exact population variance, rounded once)
+#   rstd = RN32(1 / sqrt(RN32(var + eps)))
+#   y_k  = bf16(RN32(RN32(RN32(RN32(x_k - mean) * rstd) * gamma_k) + beta_k))
+# gamma and beta are optional; without them their steps are left out.
+def _rn_f32_signed_ratio(p: int, q: int) -> np.float32:
+    """The fp32 nearest to p/q for an integer p of either sign (q > 0), ties to
+    even; a negative ratio that rounds to zero gives -0."""
+    r = _rn_f32_ratio(abs(p), q)
+    return np.float32(-r) if p < 0 else r
+
+
+def layernorm_moments(x: np.ndarray):
+    """(mean, var) per row of bf16 bit patterns x [M, K], each the exact value
+    rounded once to fp32 (fp32 [M] each)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    mean = np.empty(M, np.float32)
+    var = np.empty(M, np.float32)
+    for r in range(M):
+        m, e = _bf16_exact_parts(x[r])
+        emin = int(e.min())
+        s1 = 0
+        s2 = 0
+        for mi, ei in zip(m.tolist(), e.tolist()):
+            s1 += mi << (ei - emin)
+            s2 += (mi * mi) << (2 * (ei - emin))
+        # sum x = s1 * 2^emin,  sum x^2 = s2 * 2^(2 emin)
+        # mean = s1 * 2^emin / K;  var = (K s2 - s1^2) * 2^(2 emin) / K^2
+        n = K * s2 - s1 * s1
+        if emin >= 0:
+            mean[r] = _rn_f32_signed_ratio(s1 << emin, K)
+            var[r] = _rn_f32_ratio(n << (2 * emin), K * K)
+        else:
+            mean[r] = _rn_f32_signed_ratio(s1, K << -emin)
+            var[r] = _rn_f32_ratio(n, (K * K) << (-2 * emin))
+    return mean, var
+
+
+def layernorm_stats(x: np.ndarray, eps: float):
+    """(mean, rstd) per row (fp32 [M] each): the exact-reading mean and
+    rstd = RN32(1/sqrt(RN32(var + eps)))."""
+    mean, var = layernorm_moments(x)
+    e32 = np.float32(eps)
+    rstd = np.array([_rsqrt_rn32(np.float32(v + e32)) for v in var], np.float32)
+    return mean, rstd
+
+
+def layernorm_bf16(x: np.ndarray, gamma, beta, mean: np.ndarray, rstd: np.ndarray) -> np.ndarray:
+    """y = bf16(RN32(RN32(RN32(RN32(x - mean) * rstd) * gamma) + beta)) as bf16
+    bit patterns [M, K]; gamma / beta None leave their steps out."""
+    xv = bf16_bits_to_f64(x).astype(np.float32)  # exact
+    d = xv - np.asarray(mean, np.float32)[:, None]  # fp32 subtraction, rounded
+    y = d * np.asarray(rstd, np.float32)[:, None]  # fp32 product, rounded
+    if gamma is not None:
+        y = y * bf16_bits_to_f64(gamma).astype(np.float32)[None, :]
+    if beta is not None:
+        y = y + bf16_bits_to_f64(beta).astype(np.float32)[None, :]
+    return bf16_round(y.astype(np.float64))
+
+
+def layernorm_quantize(x: np.ndarray, gamma, beta, eps: float, gs=None, per_row: bool = False):
+    """LayerNorm to bf16, then NVFP4 quantization.
+    Returns (codes, sf, mean, rstd, row_gs or None, row_inv or None)."""
+    mean, rstd = layernorm_stats(x, eps)
+    y = layernorm_bf16(x, gamma, beta, mean, rstd)
+    if per_row:
+        g, inv = row_global_scales(y)
+        codes, sf = nvfp4_quantize(y, g, per_row=True)
+        return codes, sf, mean, rstd, g, inv
+    codes, sf = nvfp4_quantize(y, gs)
+    return codes, sf, mean, rstd, None, None

@@ -82,6 +82,25 @@ def test_host_validation_rejects_bad_arguments():
             nat.BSP_ERR_INVALID_ARG
     assert L.nvfp4_rmsnorm_quantize(p, 4, 24, 24, p, 0.0, p, 0, None, None, None, p, p, None) == \
         nat.BSP_ERR_INVALID_ARG  # K % 16
+    assert L.nvfp4_rmsnorm_quantize(p, 4, 32, 32, None, 0.0, p, 0, None, None, None, p, p, None) == \
+        nat.BSP_ERR_INVALID_ARG  # no gamma
+    assert L.nvfp4_rmsnorm_quantize(p, 4, (1 << 20) + 16, (1 << 20) + 16, p, 0.0, p, 0, None, None, None, p, p,
+                                    None) == nat.BSP_ERR_INVALID_ARG  # K above the exact path's limit
+    ln = L.nvfp4_layernorm_quantize
+    for bad in (-1.0, float("inf"), float("nan")):  # eps
+        assert ln(p, 4, 32, 32, None, None, bad, p, 0, None, None, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert ln(p, 4, 24, 24, None, None, 0.0, p, 0, None, None, None, None, p, p, None) == nat.BSP_ERR_INVALID_ARG
+    assert ln(p, 4, 32784, 32784, None, None, 0.0, p, 0, None, None, None, None, p, p, None) == \
+        nat.BSP_ERR_INVALID_ARG  # K > 32768
+    assert ln(p, 4, 32, 32, None, None, 0.0, None, 0, None, None, None, None, p, p, None) == \
+        nat.BSP_ERR_INVALID_ARG  # per-tensor without a global scale
+    assert ln(p, 4, 32, 32, odd, None, 0.0, p, 0, None, None, None, None, p, p, None) == nat.BSP_ERR_ALIGNMENT
+    assert ln(p, 4, 32, 32, None, odd, 0.0, p, 0, None, None, None, None, p, p, None) == nat.BSP_ERR_ALIGNMENT
+    assert ln(p, 0, 32, 32, None, None, 0.0, p, 0, None, None, None, None, p, p, None) == nat.BSP_OK
+    ns = L.bsp_debug_norm_stats
+    assert ns(p, 4, 32, 32, 2, 0, p, p, None, None) == nat.BSP_ERR_INVALID_ARG  # norm
+    assert ns(p, 4, 32, 32, nat.BSP_NORM_LAYER, 0, p, None, None, None) == nat.BSP_ERR_INVALID_ARG  # no var out
+    assert ns(p, 4, 40, 40, nat.BSP_NORM_RMS, 0, p, None, None, None) == nat.BSP_ERR_INVALID_ARG  # K % 16
     for bad in (0.0, -2688.0, float("inf"), float("nan")):
         assert L.bsp_nvfp4_global_scale_max(p, bad, p, p, None) == nat.BSP_ERR_INVALID_ARG
     assert L.bsp_nvfp4_global_scale_max(p, 1536.0, None, None, None) == nat.BSP_ERR_INVALID_ARG

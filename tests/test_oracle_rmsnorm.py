@@ -82,3 +82,15 @@ def test_matches_torch_rms_norm_within_one_bf16_ulp():
     got = oracle.bf16_bits_to_f64(y)
     ulp = np.abs(oracle.bf16_bits_to_f64(oracle.bf16_round(ref) + 1) - oracle.bf16_bits_to_f64(oracle.bf16_round(ref)))
     assert (np.abs(got - ref) <= ulp).all()
+
+
+def test_rsqrt_at_zero_and_infinity_and_overflowing_mean():
+    assert oracle._rsqrt_rn32(np.float32(np.inf)) == 0.0
+    assert oracle._rsqrt_rn32(np.float32(0.0)) == np.float32(np.inf)
+    # squares of the largest bf16 overflow the fp32 mean: ms = inf, rstd = +0, y = 0
+    x = np.zeros((1, 32), np.uint16)
+    x[0, :4] = 0x7F7F
+    r = oracle.rmsnorm_rstd(x, 1e-6)
+    assert r[0] == 0.0 and not np.signbit(r[0])
+    y = oracle.rmsnorm_bf16(x, _bits(np.ones(32)), r)
+    assert (y & 0x7FFF == 0).all()
