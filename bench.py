@@ -14,7 +14,8 @@ second graph with events between the kernels).  `value` = sum of 2*M*N*K over
 the layers per step / step time (TFLOP/s), summed over ranks; L2 is flushed
 (256 MiB write) before every timed step, outside the timed events.
 
-Other --config values (wan13, wan14_in, wan14_out, mxfp8, skinny_m<M>, tiny)
+Other --config values (wan13, wan14_in, wan14_out, mxfp8, skinny_m<M>,
+skinny_out_m<M>, tiny)
 time the corresponding one-layer workload the same way; --config loadtime times
 the load-time conversion of the 240 weights of a 40-block DiT stack (GB/s).
 
@@ -232,6 +233,8 @@ def make_workloads(name: str):
         return [(wl.mxfp8(), "mxfp8")]
     if name.startswith("skinny_m"):
         return [(wl.skinny(int(name[len("skinny_m"):])), "nvfp4")]
+    if name.startswith("skinny_out_m"):
+        return [(wl.skinny_out(int(name[len("skinny_out_m"):])), "nvfp4")]
     raise SystemExit(f"unknown --config {name}")
 
 

@@ -52,11 +52,19 @@ def _stale(out: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+# Per-source flags.  The quantizers must round every fp32 product and sum on its
+# own (their results are compared bit for bit with an oracle that does), so no
+# multiply-add contraction there: explicit fma calls stay fused, nothing else is.
+SOURCE_FLAGS = {"quantize.cu": ["-fmad=false"]}
+
+
 def _compile(src: str, verbose: bool, extra: list[str]) -> str:
     obj = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
-    deps = [os.path.join(HERE, src)] + [os.path.join(HERE, h) for h in HEADERS] + [os.path.join(INCLUDE, "bsp.h")]
+    deps = [os.path.join(HERE, src)] + [os.path.join(HERE, h) for h in HEADERS] + [os.path.join(INCLUDE, "bsp.h"),
+                                                                                   os.path.abspath(__file__)]
     if _stale(obj, deps) or extra:
-        cmd = [nvcc(), *FLAGS, *extra, "-I", INCLUDE, "-I", HERE, "-c", os.path.join(HERE, src), "-o", obj]
+        cmd = [nvcc(), *FLAGS, *SOURCE_FLAGS.get(src, []), *extra, "-I", INCLUDE, "-I", HERE, "-c",
+               os.path.join(HERE, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)

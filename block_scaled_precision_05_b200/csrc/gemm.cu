@@ -140,6 +140,7 @@ struct Cfg {
 struct GemmParams {
   int M, N, K;
   int num_m, num_n, num_kb;
+  int split;    // CTAs of a cluster sharing one output tile's K range (skinny kernel)
   int group_m;  // m-blocks per rasterisation group
   const float* alpha;
   const float* row_scale;
@@ -544,7 +545,11 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
 // kSf8: the activation scales are in the 8x4 layout (32-byte tiles of 8 rows x
 // 4 K-groups, row-major); a stage's box is the BNA/8 row tiles x 4 K-group
 // tiles (fp4) of 32 bytes.
-template <int KIND, int BNA, bool kSf8 = false>
+// kSplit: the tile's K range is split over the CTAs of a thread-block cluster
+// (split-K); each keeps its fp32 partial in a shared-memory buffer of
+// 128 x (BNA + 4) floats (padded rows), and the cluster's rank 0 adds the
+// others' partials, in rank order, through distributed shared memory.
+template <int KIND, int BNA, bool kSf8 = false, bool kSplit = false>
 struct SkCfg {
   static constexpr int BM = 128;                         // weight rows per tile (MMA M)
   static constexpr int ROW_BYTES = 128;
@@ -564,31 +569,42 @@ struct SkCfg {
   static constexpr int TMEM_COLS = 512;
   static constexpr int SF_WARPS = 4, EPI_WARPS = 4;
   static constexpr int THREADS = 64 + (SF_WARPS + EPI_WARPS) * 32;
-  static constexpr int FIXED_BYTES = 1024 + 256;
+  static constexpr int RED_STRIDE = BNA + 4;  // floats per partial row (one row per output column n)
+  static constexpr int RED_BYTES = kSplit ? 128 * RED_STRIDE * 4 : 0;
+  static constexpr int FIXED_BYTES = 1024 + 256 + RED_BYTES;
   static constexpr int STAGES =
       cmin(cmin((232448 - FIXED_BYTES) / STAGE_BYTES, (TMEM_COLS - ACC_COLS) / SF_COLS), 8);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
   static_assert(STAGES >= 2 && ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "budget");
 };
 
-template <int KIND, int BNA, bool kSf8>
-__global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
+template <int KIND, int BNA, bool kSf8, bool kSplit>
+__global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8, kSplit>::THREADS, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmSFW, const __grid_constant__ CUtensorMap tmSFX,
                        const GemmParams p) {
-  using C = SkCfg<KIND, BNA, kSf8>;
+  using C = SkCfg<KIND, BNA, kSf8, kSplit>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  float* red = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);  // split-K partial (kSplit)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::RED_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* sf_ready = empty + C::STAGES;
   uint64_t* acc_full = sf_ready + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* part_ready = drain + 1;  // rank 0: the other ranks' partials of the tile are in their buffers
+  uint64_t* part_free = part_ready + 1;  // rank > 0: rank 0 has read this CTA's partial
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(part_free + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
+  // split-K: cluster rank r takes k-blocks [kb0, kb1) of every tile of its cluster
+  const int S = kSplit ? p.split : 1;
+  const uint32_t rank = kSplit ? cluster_ctarank() : 0u;
+  const int kb0 = static_cast<int>(static_cast<int64_t>(p.num_kb) * rank / S);
+  const int kb1 = static_cast<int>(static_cast<int64_t>(p.num_kb) * (rank + 1) / S);
+  const int first_tile = static_cast<int>(blockIdx.x) / S, tile_step = static_cast<int>(gridDim.x) / S;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -599,6 +615,10 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, C::EPI_WARPS);
     mbar_init(drain, 1);
+    if constexpr (kSplit) {
+      mbar_init(part_ready, static_cast<uint32_t>((S - 1) * C::EPI_WARPS * 32));
+      mbar_init(part_free, C::EPI_WARPS * 32);
+    }
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -614,6 +634,7 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
+  if constexpr (kSplit) cluster_sync();  // every CTA's barriers exist before another CTA arrives on them
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   grid_dependency_wait();  // as in the main kernel
@@ -626,9 +647,9 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
       uint32_t issued[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
         const int nb = t % p.num_n, mb = t / p.num_n;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -663,13 +684,13 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int it = 0;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+      for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
         if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -682,7 +703,7 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
           const uint64_t xdesc = desc_kmajor_sw128(sbase + C::W_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::MMAS; ++kk) {
-            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accumulate = (kb > kb0 || kk > 0) ? 1u : 0u;
             if constexpr (KIND == kNVF4)
               tc_mma_nvf4(tmem, wdesc + 2u * kk, xdesc + 2u * kk, idesc_nvf4(C::BM, BNA), sfw_t + 4u * kk,
                           sfx_t + 4u * kk, accumulate);
@@ -711,8 +732,8 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t stage = 0, phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+    for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag)) {
           ok = false;
           break;
@@ -772,11 +793,46 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
     // epilogue: lane = output column n, TMEM column c = activation row m
     const int q = warp & 3;
     const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+    const int nl = q * 32 + static_cast<int>(lane);  // output column within the panel
+    float* my_red = red + nl * C::RED_STRIDE;
     int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+    for (int t = first_tile; t < num_tiles; t += tile_step, ++it) {
       const int nb = t % p.num_n, mb = t / p.num_n;
-      const int n = nb * C::BM + q * 32 + static_cast<int>(lane);
+      const int n = nb * C::BM + nl;
       const bool n_ok = n < p.N;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      if (kSplit && rank != 0) {
+        // split-K partial of ranks > 0: into this CTA's buffer, once rank 0
+        // has read the previous tile's partial from it
+        if (it > 0 && !mbar_wait_cluster(part_free, static_cast<uint32_t>(it - 1) & 1u, abort_flag)) {
+          *abort_flag = 1u;
+          raise_error(p.err, kErrTimeout);
+          break;
+        }
+        if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
+          *abort_flag = 1u;
+          raise_error(p.err, kErrTimeout);
+          break;
+        }
+        tc_fence_after_sync();
+#pragma unroll
+        for (int c0 = 0; c0 < BNA; c0 += 16) {
+          if (mb * BNA + c0 >= p.M) break;  // warp-uniform
+          uint32_t r[16];
+          tmem_ld_16cols(taddr + static_cast<uint32_t>(c0), r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<float4*>(my_red + c0 + 4 * j) =
+                make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
+                            __uint_as_float(r[4 * j + 3]));
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        mbar_arrive_remote(mapa_shared(smem_u32(part_ready), 0u));  // every lane, after its own writes
+        continue;
+      }
       float b = 0.0f;
       if (p.bias != nullptr && n_ok) b = bf16_bits_to_f32(p.bias[n]);
       // alpha x row scale of this tile's activation rows, one row per lane,
@@ -792,20 +848,42 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
         raise_error(p.err, kErrTimeout);
         break;
       }
+      if (kSplit && !mbar_wait_cluster(part_ready, static_cast<uint32_t>(it) & 1u, abort_flag)) {
+        *abort_flag = 1u;
+        raise_error(p.err, kErrTimeout);
+        break;
+      }
       tc_fence_after_sync();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
       for (int c0 = 0; c0 < BNA; c0 += 16) {
         if (mb * BNA + c0 >= p.M) break;  // warp-uniform
         uint32_t r[16];
         tmem_ld_16cols(taddr + static_cast<uint32_t>(c0), r);
         tmem_ld_wait();
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(r[i]);
+        if constexpr (kSplit) {
+          // the other ranks' partials, added in rank order (the sum does not
+          // depend on which CTA finished first)
+          for (int s = 1; s < S; ++s) {
+            const uint32_t peer = mapa_shared(smem_u32(my_red + c0), static_cast<uint32_t>(s));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 v = ld_shared_cluster_f4(peer + 16u * j);
+              acc[4 * j] = __fadd_rn(acc[4 * j], v.x);
+              acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], v.y);
+              acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], v.z);
+              acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], v.w);
+            }
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int m = mb * BNA + c0 + i;
           if (m >= p.M) break;  // warp-uniform
           const float scale = __shfl_sync(0xFFFFFFFFu, rs[(c0 + i) >> 5], (c0 + i) & 31);
-          const float y = __fmaf_rn(__uint_as_float(r[i]), scale, b);
+          const float y = __fmaf_rn(acc[i], scale, b);
           if (n_ok) {
             if (p.out_f32)
               static_cast<float*>(p.D)[static_cast<int64_t>(m) * p.ld_d + n] = y;
@@ -817,11 +895,17 @@ __global__ void __launch_bounds__(SkCfg<KIND, BNA, kSf8>::THREADS, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
+      if constexpr (kSplit) {
+        // the partials are read: each rank may reuse its buffer
+        for (int s = 1; s < S; ++s) mbar_arrive_remote(mapa_shared(smem_u32(part_free), static_cast<uint32_t>(s)));
+      }
     }
   }
 
   tc_fence_before_sync();
   __syncthreads();
+  // no CTA leaves while another may still read its buffer or arrive on its barriers
+  if constexpr (kSplit) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
@@ -834,11 +918,11 @@ int encode_operand(CUtensorMap* m, const void* base, int64_t rows, int64_t row_b
 int encode_scales(CUtensorMap* m, const void* base, int64_t bands, int64_t tiles_per_band, int atoms, int box_bands);
 int encode_rows_plain(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows, int box_bytes);
 
-template <int KIND, int BNA, bool kSf8 = false>
+template <int KIND, int BNA, bool kSf8 = false, bool kSplit = false>
 int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                   int64_t row_bytes, int64_t tiles_per_band, GemmParams p, cudaStream_t stream) {
-  using C = SkCfg<KIND, BNA, kSf8>;
-  auto kernel = skinny_gemm_kernel<KIND, BNA, kSf8>;
+  using C = SkCfg<KIND, BNA, kSf8, kSplit>;
+  auto kernel = skinny_gemm_kernel<KIND, BNA, kSf8, kSplit>;
   static bool attr_set[64] = {};
   if (!attr_set[dev.id]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
@@ -860,11 +944,10 @@ int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, c
   }
   p.num_n = static_cast<int>(ceil_div(p.N, C::BM));
   p.num_m = static_cast<int>(ceil_div(p.M, BNA));
+  if (!kSplit) p.split = 1;
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
-  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -872,8 +955,46 @@ int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  int64_t clusters = tiles < dev.sm_count / p.split ? tiles : dev.sm_count / p.split;
+  if constexpr (kSplit) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(p.split);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    // no more clusters than are resident at once (a cluster's CTAs share one
+    // GPC): the grid is one wave of them, each looping over its tiles
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.split), 1, 1);
+    int resident = 0;
+    if (cudaOccupancyMaxActiveClusters(&resident, kernel, &cfg) != cudaSuccess) return launch_status();
+    if (resident < 1) return BSP_ERR_CUDA;  // a cluster of this size does not fit: nothing launched
+    if (clusters > resident) clusters = resident;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.split), 1, 1);
   if (cudaLaunchKernelEx(&cfg, kernel, tmW, tmX, tmSFW, tmSFX, p) != cudaSuccess) return launch_status();
   return launch_status();
+}
+
+// CTAs per tile of the skinny kernel: 1, or a split of K over a cluster of up
+// to 4 CTAs when the tiles alone would leave at least half of the SMs without
+// work (few weight panels: N <= ~9K), bounded by the tile's k-blocks.
+int skinny_split(const DeviceInfo& dev, int64_t tiles, int num_kb) {
+  if (tiles * 2 > dev.sm_count) return 1;
+  int64_t s = dev.sm_count / tiles;
+  s = s < 4 ? s : 4;
+  s = s < num_kb ? s : num_kb;
+  return s < 1 ? 1 : static_cast<int>(s);
+}
+
+template <int KIND, int BNA, bool kSf8 = false>
+int launch_skinny_any(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
+                      const uint8_t* sfB, int64_t row_bytes, int64_t tiles_per_band, GemmParams p,
+                      cudaStream_t stream) {
+  const int64_t tiles = ceil_div(p.N, 128) * ceil_div(p.M, BNA);
+  p.split = skinny_split(dev, tiles, p.num_kb);
+  if (p.split > 1)
+    return launch_skinny<KIND, BNA, kSf8, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+  return launch_skinny<KIND, BNA, kSf8, false>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
 }
 
 // Row-major uint8 matrix [rows, row_bytes], boxes of box_rows x box_bytes (128
@@ -1021,6 +1142,7 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.num_kb = static_cast<int>(ceil_div(row_bytes, 128));
+  p.split = 1;
   p.alpha = alpha;
   p.row_scale = row_scale;
   p.bias = bias;
@@ -1030,16 +1152,16 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   p.err = dev.err_word;
   if constexpr (KIND == kNVF4) {
     if (sf8) {  // 8x4 activation scales: M <= 64, the transposed kernel
-      if (M <= 16) return launch_skinny<KIND, 16, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
-      if (M <= 32) return launch_skinny<KIND, 32, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
-      return launch_skinny<KIND, 64, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+      if (M <= 16) return launch_skinny_any<KIND, 16, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+      if (M <= 32) return launch_skinny_any<KIND, 32, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+      return launch_skinny_any<KIND, 64, true>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
     }
   }
   if (skinny) {
-    if (M <= 16) return launch_skinny<KIND, 16>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
-    if (M <= 32) return launch_skinny<KIND, 32>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
-    if (M <= 64) return launch_skinny<KIND, 64>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
-    return launch_skinny<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    if (M <= 16) return launch_skinny_any<KIND, 16>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    if (M <= 32) return launch_skinny_any<KIND, 32>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    if (M <= 64) return launch_skinny_any<KIND, 64>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
+    return launch_skinny_any<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, p, stream);
   }
   // 128-column tiles when they still fit in one wave: twice the CTAs stream B
   // (for small M the weight stream, not the tensor pipe, sets the time)

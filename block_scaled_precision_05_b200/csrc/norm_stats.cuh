@@ -24,6 +24,10 @@
 //   - multiplying by RN64(1/K) adds two roundings (2u relative);
 //   - the LayerNorm variance is the fp64 mean of squares less the square of
 //     the fp64 mean, with the bound of ln_fast;
+//   - means of bf16 data often lie exactly halfway between two fp32 values
+//     (the exact mean has few bits); when the fp64 sum of the row is provably
+//     exact (ln_mean_exact) the mean is then decided exactly without the
+//     integer path;
 //   - every bound below carries a margin of several u (and the check itself is
 //     done in fp64 with a margin that covers its own roundings).
 #pragma once
@@ -73,27 +77,34 @@ __device__ __forceinline__ double sumsq8(const uint4& v, double acc) {
   return sumsq_word(v.w, acc);
 }
 
-// x * 2^-384 with its sign, built like mag_2m384 (zero and subnormal x: off
-// by at most 2^-510).
-__device__ __forceinline__ double x_2m384(uint32_t f) {
-  return hi_word_double((((f >> 3) & 0x0FFFE000u) | 0x20000000u) | (f & 0x80000000u));
-}
-
-// s1 + x0 + x1 (units 2^-384) and s2 + x0^2 + x1^2 (units 2^-768) for the two
-// elements of w, one rounding per addition.
-__device__ __forceinline__ void sums_word(uint32_t w, double& s1, double& s2) {
-  const double d0 = x_2m384(f32_lo(w)), d1 = x_2m384(f32_hi(w));
-  s1 += d0;
-  s2 = fma(d0, d0, s2);
-  s1 += d1;
-  s2 = fma(d1, d1, s2);
+// The LayerNorm sums in real units: |x| exactly (|x| * 2^-896 from the bit
+// pattern, zero and subnormals included, times 2^896) and +-1.0 carrying the
+// sign, so that s1 + x and s2 + x^2 each round once and a zero adds exactly 0.
+__device__ __forceinline__ void sums_elem(uint32_t f, double& s1, double& s2) {
+  const double a = mag_2m896(f) * 0x1p896;
+  const double sg = hi_word_double((f & 0x80000000u) | 0x3FF00000u);
+  s1 = fma(a, sg, s1);
+  s2 = fma(a, a, s2);
 }
 
 __device__ __forceinline__ void sums8(const uint4& v, double& s1, double& s2) {
-  sums_word(v.x, s1, s2);
-  sums_word(v.y, s1, s2);
-  sums_word(v.z, s1, s2);
-  sums_word(v.w, s1, s2);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sums_elem(f32_lo(w[i]), s1, s2);
+    sums_elem(f32_hi(w[i]), s1, s2);
+  }
+}
+
+// Running minimum, over 16-bit halves, of (|x| bits - 1) with a zero mapped
+// to 0xFFFF: |x| + 0x7FFF cannot carry out of a half (|x| <= 0x7FFF), and the
+// top bit of the sum is set exactly when |x| > 0, so flipping it gives
+// |x| - 1 for a nonzero x and 0xFFFF for a zero.
+__device__ __forceinline__ uint32_t min_nonzero_mag8(const uint4& v, uint32_t m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = __vminu2(m, ((w[i] & 0x7FFF7FFFu) + 0x7FFF7FFFu) ^ 0x80008000u);
+  return m;
 }
 
 // Sum over the warp; every lane ends with the same bits (each butterfly step
@@ -111,18 +122,20 @@ __host__ __device__ __forceinline__ int sum_depth(int64_t K) { return static_cas
 
 // RN32(v) for a real v >= 0 known as v_hat with |v_hat - v| <= err: true (and
 // the value in *out) when every real within err of v_hat rounds to the same
-// fp32.  The test keeps v a quarter of an fp32 ulp (at least 2^-151) from the
-// candidate c = RN32(v_hat) on both sides: then v lies strictly inside c's
-// rounding interval (half an ulp each side, a quarter below a power of two).
-// |v_hat - c| is exact (c is within a factor two of v_hat, or both are below
-// 2^-125 where the difference fits), and the final sum's rounding is covered
-// by the margins the callers put in err.
+// fp32.  c = RN32(v_hat) rounds every real strictly within half the spacing to
+// its neighbours; the test keeps [v_hat - err, v_hat + err] inside the smaller
+// of the two halves, h: half an ulp of c (2^(e-151) for biased exponent e >= 1),
+// a quarter at a power of two (the spacing below halves there), and 2^-150
+// among the subnormals and zero.  |v_hat - c| is exact (c is within a factor
+// two of v_hat, or both are below 2^-125 where the difference fits), and the
+// final sum's rounding is covered by the margins the callers put in err.
 __device__ __forceinline__ bool rn32_certain(double v_hat, double err, float* out) {
   if (!(v_hat >= 0.0) || !(err < 1e300)) return false;  // NaN / inf estimates: decided exactly
   const float c = __double2float_rn(v_hat);
-  const uint32_t e = __float_as_uint(c) >> 23;
+  const uint32_t cb = __float_as_uint(c), e = cb >> 23;
   if (e >= 254u) return false;  // at the top of the fp32 range: decided exactly
-  const double h = hi_word_double((max(e, 1u) + 871u) << 20);  // 2^(max(e,1) - 152)
+  const uint32_t he = (e >= 2u && (cb & 0x7FFFFFu) == 0u) ? e - 1u : max(e, 1u);
+  const double h = hi_word_double((he + 872u) << 20);  // 2^(he - 151)
   if (!(fabs(v_hat - static_cast<double>(c)) + err < h)) return false;
   *out = c;
   return true;
@@ -137,31 +150,76 @@ __device__ __forceinline__ bool ms_fast(double s_hat, int64_t K, double rK, floa
   return rn32_certain(v, err, ms);
 }
 
-// LayerNorm mean and variance from s1_hat (the fp64 sum of x, units 2^-384)
-// and s2_hat (the fp64 sum of x^2, units 2^-768), one pass over the row:
+// LayerNorm mean and variance from s1_hat = the fp64 sum of x and s2_hat =
+// the fp64 sum of x^2 (exact terms), one pass over the row:
 //   mean' = S1 / K,  ms' = S2 / K,  var' = ms' - mean'^2.
 // With A^2 = S2 / K = var + mean^2 (and |S1| <= K A):
-//   |mean' - mean| <= (D + 3) u A + 2^-127 (zero elements count 2^-127 each)
-//   |ms' - S2/K|   <= (D + 3) u A^2 + 2^-252
-//   |var' - var|   <= (3D + 12) u A^2 + 2^-126 A + 2^-251  (with the roundings
-//                     of mean'^2 and of the subtraction)
-// so the variance is decided by the fast path when var is not far below
-// mean^2 (a row whose mean is many standard deviations from 0 falls to the
-// exact path more often, not to a wrong result).
+//   |mean' - mean| <= (D + 3) u A
+//   |ms' - S2/K|   <= (D + 3) u A^2
+//   |var' - var|   <= (3D + 12) u A^2   (with the roundings of mean'^2 and of
+//                                        the subtraction)
+// A row whose mean is many standard deviations from 0 falls to the exact path
+// more often, never to a wrong result.
 __device__ __forceinline__ bool ln_fast(double s1_hat, double s2_hat, int64_t K, double rK, float* mean, float* var) {
   const double D = static_cast<double>(sum_depth(K));
-  const double mu = (s1_hat * 0x1p384) * rK;
-  const double a2 = (s2_hat * 0x1p768) * rK;
+  const double mu = s1_hat * rK;
+  const double a2 = s2_hat * rK;
   const double v = a2 - mu * mu;
   // sqrt(a2) bounded above with an fp32 square root widened by 1%
   const double a = 1.01 * static_cast<double>(sqrtf(static_cast<float>(a2)));
-  const double err_mu = (D + 8.0) * kU * a + 0x1p-125;
-  const double err_var = (3.0 * D + 24.0) * kU * a2 + 0x1p-124 * a + 0x1p-249;
+  const double err_mu = (D + 8.0) * kU * a;
+  const double err_var = (3.0 * D + 24.0) * kU * a2 + 0x1p-300;
   if (!(fabs(mu) > 2.0 * err_mu)) return false;  // the mean's sign is certain
   float m;
   if (!rn32_certain(fabs(mu), err_mu, &m)) return false;
   if (!rn32_certain(v, err_var, var)) return false;
   *mean = mu < 0.0 ? -m : m;
+  return true;
+}
+
+// The variance alone, as in ln_fast (for rows whose mean the fast bound left open).
+__device__ __forceinline__ bool ln_var_fast(double s1_hat, double s2_hat, int64_t K, double rK, float* var) {
+  const double D = static_cast<double>(sum_depth(K));
+  const double mu = s1_hat * rK;
+  const double a2 = s2_hat * rK;
+  return rn32_certain(a2 - mu * mu, (3.0 * D + 24.0) * kU * a2 + 0x1p-300, var);
+}
+
+// When the fp64 sum of a row is exact, the mean's rounding is decided exactly.
+// Every element is a multiple of 2^G, G = max(E, 1) - 134 for the exponent
+// field E of the smallest nonzero |x| (bf16: 7 fraction bits, subnormals on
+// the grid of E = 1), so every partial sum is; and every partial sum is at
+// most sum |x| <= sqrt(K S2) in magnitude.  If that is below 2^(G + 53), no
+// addition rounds and s1_hat = S1.  Then RN32(S1 / K) is settled by comparing
+// |S1| with K times the midpoints around the candidate, products that fp64
+// holds exactly (25-bit midpoints, K <= 2^15).
+__device__ __forceinline__ bool ln_mean_exact(double s1_hat, double s2_hat, int64_t K, double rK, uint32_t min_mag_m1,
+                                              float* mean) {
+  if (min_mag_m1 >= 0x7FFFu) {  // no nonzero element: S1 = 0
+    *mean = 0.0f;
+    return s1_hat == 0.0;
+  }
+  const int E = static_cast<int>((min_mag_m1 + 1u) >> 7);
+  const int G = (E > 1 ? E : 1) - 134;
+  const double lim = hi_word_double(static_cast<uint32_t>(2 * G + 106 + 1023) << 20);  // 2^(2G + 106)
+  if (!(static_cast<double>(K) * s2_hat * (1.0 + 0x1p-30) < lim)) return false;
+  const double a = fabs(s1_hat);
+  const float c = __double2float_rn(a * rK);
+  const float up = nextafterf(c, __int_as_float(0x7F800000)), dn = c > 0.0f ? nextafterf(c, 0.0f) : 0.0f;
+  const double kd = static_cast<double>(K);
+  const double k_hi = kd * (0.5 * (static_cast<double>(c) + static_cast<double>(up)));
+  const double k_lo = kd * (0.5 * (static_cast<double>(c) + static_cast<double>(dn)));
+  const bool c_even = (__float_as_uint(c) & 1u) == 0u;
+  float r = c;
+  if (a > k_hi)
+    r = up;
+  else if (a == k_hi)
+    r = c_even ? c : up;
+  else if (a < k_lo)
+    r = dn;
+  else if (a == k_lo)
+    r = c_even ? c : dn;
+  *mean = s1_hat < 0.0 ? -r : r;
   return true;
 }
 

@@ -178,8 +178,8 @@ __device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sf
 template <class In>
 __device__ __forceinline__ uint32_t nvfp4_codes8(const uint4& v, float inv) {
   const float2 i2 = make_float2(inv, inv);
-  const float2 p0 = __fmul2_rn(In::values2(v.x), i2), p1 = __fmul2_rn(In::values2(v.y), i2);
-  const float2 p2 = __fmul2_rn(In::values2(v.z), i2), p3 = __fmul2_rn(In::values2(v.w), i2);
+  const float2 p0 = mul2_rn(In::values2(v.x), i2), p1 = mul2_rn(In::values2(v.y), i2);
+  const float2 p2 = mul2_rn(In::values2(v.z), i2), p3 = mul2_rn(In::values2(v.w), i2);
   return cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y);
 }
 
@@ -497,7 +497,7 @@ __device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, floa
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     // two fp32 products per packed instruction, each rounded as a scalar one
-    const float2 y = __fmul2_rn(__fmul2_rn(InBf16::values2(xw[i]), r2), InBf16::values2(gw[i]));
+    const float2 y = mul2_rn(mul2_rn(InBf16::values2(xw[i]), r2), InBf16::values2(gw[i]));
     const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
     memcpy(&o[i], &h, 4);
   }
@@ -512,8 +512,8 @@ __device__ __forceinline__ uint4 layernorm8(const uint4& xv, const uint4& gv, co
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 d = __fadd2_rn(InBf16::values2(xw[i]), nm2);  // x - mean, rounded once
-    const float2 y = __fadd2_rn(__fmul2_rn(__fmul2_rn(d, r2), InBf16::values2(gw[i])), InBf16::values2(bw[i]));
+    const float2 d = add2_rn(InBf16::values2(xw[i]), nm2);  // x - mean, rounded once
+    const float2 y = add2_rn(mul2_rn(mul2_rn(d, r2), InBf16::values2(gw[i])), InBf16::values2(bw[i]));
     const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
     memcpy(&o[i], &h, 4);
   }
@@ -558,6 +558,21 @@ __device__ __noinline__ void norm_row_exact(const uint16_t* __restrict__ row, in
   __syncwarp();
 }
 
+// A LayerNorm row whose fast bounds left the statistics open: the mean
+// decided exactly from the fp64 sum when that sum is provably exact (the
+// row's smallest nonzero |x| is re-read), and the variance from its bound.
+__device__ __noinline__ bool ln_row_mean_exact(const uint16_t* __restrict__ row, int64_t K, double s1, double s2,
+                                               double rK, float* mean, float* var) {
+  uint32_t m = 0xFFFFFFFFu;
+  for (int64_t g = lane_id(); g < (K >> 4); g += 32) {
+    m = normstats::min_nonzero_mag8(ldg16(row + g * 16), m);
+    m = normstats::min_nonzero_mag8(ldg16(row + g * 16 + 8), m);
+  }
+  m = __reduce_min_sync(kFull, min(m & 0xFFFFu, m >> 16));
+  if (!normstats::ln_var_fast(s1, s2, K, rK, var)) return false;
+  return normstats::ln_mean_exact(s1, s2, K, rK, m, mean);
+}
+
 // Row statistics.  `each(f)` applies f to each of this lane's 16-byte chunks
 // of the row (any order; the chunks of the 32 lanes cover the row once);
 // `row` is the row in global memory, re-read by the exact path.
@@ -579,7 +594,9 @@ __device__ __forceinline__ NormRow norm_row_stats(Each each, const uint16_t* row
     s1 = normstats::warp_sum(s1);
     s2 = normstats::warp_sum(s2);
     float mean, var;
-    if (!normstats::ln_fast(s1, s2, K, rK, &mean, &var)) norm_row_exact<true>(row, K, xs, &mean, &var);  // warp-uniform
+    if (!normstats::ln_fast(s1, s2, K, rK, &mean, &var) &&  // warp-uniform
+        !ln_row_mean_exact(row, K, s1, s2, rK, &mean, &var))
+      norm_row_exact<true>(row, K, xs, &mean, &var);
     p.mean = mean;
     p.rstd = __frsqrt_rn(__fadd_rn(var, eps));
   }
@@ -757,6 +774,7 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_sh
         uint2 w;
         w.x = nvfp4_codes8<InBf16>(y0, inv);
         w.y = nvfp4_codes8<InBf16>(y1, inv);
+        if (!live) sfb = 0u;  // scale padding (LayerNorm's beta would make y nonzero there)
         const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
         const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
         const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
@@ -770,8 +788,9 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_sh
 
 // Row statistics alone (diagnostic entry bsp_debug_norm_stats): per row the
 // RMSNorm ms, or the LayerNorm mean and var, each as the fast decision with its
-// exact fallback (exact_only = false) or always from the exact sums; path[r]
-// = 1 where the exact sums were used.
+// exact fallbacks (exact_only = false) or always from the exact sums; path[r]
+// = 0 where the fp64 bounds decided, 2 where the LayerNorm mean came from a
+// provably exact fp64 sum, 1 where the exact integer sums were used.
 template <bool kLN>
 __global__ void __launch_bounds__(kQuantThreads) norm_stats_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                                     int64_t K, int64_t ld_x, bool exact_only,
@@ -793,7 +812,7 @@ __global__ void __launch_bounds__(kQuantThreads) norm_stats_kernel(const uint16_
       }
     };
     float a = 0.0f, b = 0.0f;
-    bool fast = false;
+    bool fast = false, certified = false;
     if (!exact_only) {
       if constexpr (kLN) {
         double s1 = 0.0, s2 = 0.0;
@@ -801,6 +820,7 @@ __global__ void __launch_bounds__(kQuantThreads) norm_stats_kernel(const uint16_
         s1 = normstats::warp_sum(s1);
         s2 = normstats::warp_sum(s2);
         fast = normstats::ln_fast(s1, s2, K, rK, &a, &b);
+        if (!fast && ln_row_mean_exact(row, K, s1, s2, rK, &a, &b)) certified = true;
       } else {
         double acc = 0.0;
         each([&](const uint4& v) { acc = normstats::sumsq8(v, acc); });
@@ -808,11 +828,11 @@ __global__ void __launch_bounds__(kQuantThreads) norm_stats_kernel(const uint16_
         fast = normstats::ms_fast(acc, K, rK, &a);
       }
     }
-    if (!fast) norm_row_exact<kLN>(row, K, xs, &a, &b);
+    if (!fast && !certified) norm_row_exact<kLN>(row, K, xs, &a, &b);
     if (lane == 0) {
       stat0[r] = a;
       if (stat1) stat1[r] = b;
-      if (path) path[r] = fast ? 0 : 1;
+      if (path) path[r] = fast ? 0 : (certified ? 2 : 1);
     }
   }
 }

@@ -22,6 +22,8 @@ hao-ai-lab-FastVideo nvfp4_qat_config.py, ``DEFAULT_FP4_LAYERS``):
             seed 3 (the GELU of an fc_in-like output, drawn independently)
   skinny    A [M, 5120] ~N(0,1), M in {1, 16, 128, 1024, 4096}; W [13824, 5120] ~N(0, 0.02);
             seed 4
+  skinny_out A [M, 13824] ~N(0,1); W [5120, 13824] ~N(0, 0.02) (the fc_out shape at
+            decode-sized M); seed 7
   mxfp8     A [32760, 5120] ~N(0,1) + outliers; W [5120, 5120] ~N(0, 1/sqrt(5120)); seed 5
   weights   the 240 weights of 40 DiT blocks (q, k, v, out 5120x5120; fc_in 13824x5120;
             fc_out 5120x13824) ~N(0, 0.02), drawn on the device by ``device_weight``
@@ -130,6 +132,15 @@ def skinny(M: int, seed: int = 4) -> Linear:
     W = normal_bf16(rng, (DIT_FFN, DIT_HIDDEN), 0.02)
     A = normal_bf16(np.random.default_rng([seed, M]), (M, DIT_HIDDEN))
     return Linear(f"skinny_m{M}", A, W, per_token=True)
+
+
+def skinny_out(M: int, seed: int = 7) -> Linear:
+    """Per-token-scaled activations against one fc_out-shaped weight [5120, 13824]
+    (few weight panels, long K)."""
+    rng = np.random.default_rng(seed)
+    W = normal_bf16(rng, (DIT_HIDDEN, DIT_FFN), 0.02)
+    A = normal_bf16(np.random.default_rng([seed, M]), (M, DIT_FFN))
+    return Linear(f"skinny_out_m{M}", A, W, per_token=True)
 
 
 def mxfp8(M: int = WAN_TOKENS, seed: int = 5) -> Linear:

@@ -451,9 +451,10 @@ int bsp_debug_wait_timeout(int64_t limit_ns, bsp_stream_t stream);
  * stat0[r] = ms (the exact mean of squares rounded to fp32), BSP_NORM_LAYER
  * writes stat0[r] = mean and stat1[r] = var (each exact, rounded to fp32).
  * exact_only != 0 skips the fp64 decision and always takes the exact integer
- * sums; path (int [M], or NULL) receives 0 where the fp64 decision settled the
- * row and 1 where the exact sums did.  K % 16 == 0 and the K limits of the
- * fused calls; errors as nvfp4_rmsnorm_quantize. */
+ * sums; path (int [M], or NULL) receives 0 where the fp64 error bounds settled
+ * the row, 2 where the LayerNorm mean was decided from a provably exact fp64
+ * sum, and 1 where the exact integer sums did.  K % 16 == 0 and the K limits
+ * of the fused calls; errors as nvfp4_rmsnorm_quantize. */
 int bsp_debug_norm_stats(const uint16_t *x, int64_t M, int64_t K, int64_t ld_x, int norm,
                          int exact_only, float *stat0, float *stat1, int *path, bsp_stream_t stream);
 

@@ -105,7 +105,7 @@ def test_rows_at_rounding_ties_take_the_exact_path(K, per_row):
     rand, g, b = _case(40, K, seed=K + 17)
     x = np.concatenate([_tie_rows(K, 24, seed=K), rand])
     _, path = api.norm_stats(up_bf16(x), "layer")
-    assert int(down(path)[:24].sum()) >= 8
+    assert int((down(path)[:24] != 0).sum()) >= 8  # the ties are not settled by the fp64 bounds
     q, mean, rstd = _run(x, g, b, 0.0, per_row)
     _check(q, mean, rstd, x, g, b, 0.0, per_row)
 
@@ -133,7 +133,7 @@ def test_norm_stats_exact_path_equals_fast_path():
     xt = up_bf16(xb)
     (m_fast, v_fast), _ = api.norm_stats(xt, "layer")
     (m_ex, v_ex), p_ex = api.norm_stats(xt, "layer", exact_only=True)
-    assert int(down(p_ex).min()) == 1
+    assert (down(p_ex) == 1).all()
     assert torch.equal(m_fast, m_ex) and torch.equal(v_fast, v_ex)
     m_ref, v_ref = oracle.layernorm_moments(xb)
     assert np.array_equal(down(m_ex).view(np.uint32), m_ref.view(np.uint32))
