@@ -218,19 +218,21 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- workloads
-def make_workloads(name: str):
-    """[(Linear, kind)] of the layers one step runs, in order."""
+def make_workloads(name: str, rows: int = 0):
+    """[(Linear, kind)] of the layers one step runs, in order (rows > 0: the
+    large-M workloads with that many activation rows, for profiler captures)."""
     from block_scaled_precision_05_b200 import workloads as wl
+    kw = {"M": rows} if rows > 0 else {}
     if name == "wan14":  # the FFN: fc_in then fc_out, each on its own resident input
-        return [(wl.wan14_in(), "nvfp4"), (wl.wan14_out(), "nvfp4")]
+        return [(wl.wan14_in(**kw), "nvfp4"), (wl.wan14_out(**kw), "nvfp4")]
     if name == "wan13":
-        return [(wl.wan13(), "nvfp4")]
+        return [(wl.wan13(**kw), "nvfp4")]
     if name == "tiny":
         return [(wl.tiny(), "nvfp4")]
     if name in ("wan14_in", "wan14_out"):
-        return [(getattr(wl, name)(), "nvfp4")]
+        return [(getattr(wl, name)(**kw), "nvfp4")]
     if name == "mxfp8":
-        return [(wl.mxfp8(), "mxfp8")]
+        return [(wl.mxfp8(**kw), "mxfp8")]
     if name.startswith("skinny_m"):
         return [(wl.skinny(int(name[len("skinny_m"):])), "nvfp4")]
     if name.startswith("skinny_out_m"):
@@ -482,7 +484,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    specs = [(apply_input_format(lin, kind, args.input), kind) for lin, kind in make_workloads(args.config)]
+    specs = [(apply_input_format(lin, kind, args.input), kind) for lin, kind in make_workloads(args.config, args.rows)]
     runs = [LayerRun(lin, kind, args, dev) for lin, kind in specs]
     flops = float(sum(r.lin.flops for r in runs))
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -1045,11 +1047,15 @@ def main():
                     help="rows of each layer's A per oracle step (reference arm and cpu_baseline; 0: up to 128)")
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="set up, run this many untimed eager steps and exit (for a profiler capture)")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="with --profile-launches: activation rows of the large-M workloads (0: the config's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--blocks", type=int, default=40, help="DiT blocks for --config loadtime")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.rows and not args.profile_launches:
+        ap.error("--rows applies to --profile-launches runs only")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

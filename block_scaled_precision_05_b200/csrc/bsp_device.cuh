@@ -103,6 +103,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute it with the same count): the launch gives every thread the same
+// budget; roles that need few registers hand theirs back so that others may
+// grow.  The counts of all warpgroups must add up to the launch's total.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Thread-block clusters: this CTA's rank, the address of a shared variable in
 // another CTA of the cluster, arrivals on and reads from that memory (the
 // distributed shared memory of the cluster), and the cluster-wide barrier.

@@ -18,21 +18,24 @@
 //               are ready, issues four block-scaled MMAs (K = 64 fp4 / 32 fp8
 //               each) accumulating fp32 in tensor memory, and releases the
 //               stage (tcgen05.commit).
-//   warps 10-13 scale-factor warps, one per 32-lane quarter of tensor memory:
+//   warps 4-7   scale-factor warps, one per 32-lane quarter of tensor memory:
 //               read the stage's 128x4 scale tiles from shared memory and write
 //               them into the stage's scale columns of tensor memory
 //               (tcgen05.st; each quarter holds the scales of all rows, which is
 //               the replicated layout the block-scaled MMA reads).  Keeping the
 //               scale traffic off the tensor pipe lets it overlap the MMAs of
 //               the previous stages.
-//   warps 2..9  epilogue, two warps per 32-lane quarter of tensor memory, each
-//               owning half of the tile's accumulator columns: read them into
-//               registers (tcgen05.ld), hand the accumulator back to the MMA
-//               warp at once, apply alpha, row scale and bias in fp32, round
-//               once, stage 32 rows x 32 bytes in swizzled shared memory and
-//               write them with TMA stores (full 32-byte sectors; rows/columns
-//               past M/N clipped).
-//   (roles by warp index: 0 producer, 1 MMA, 2-9 epilogue, 10-13 scales)
+//   warps 8-15  epilogue, two warps per 32-lane quarter of tensor memory, each
+//               owning half of the tile's accumulator columns: read all of them
+//               into registers (tcgen05.ld), hand the accumulator back to the
+//               MMA warp at once, then apply alpha, row scale and bias in fp32,
+//               round once, stage 32 rows x 32 bytes in swizzled shared memory
+//               and write them with TMA stores (full 32-byte sectors;
+//               rows/columns past M/N clipped).
+//   (roles by warp index: 0 producer, 1 MMA, 2-3 idle, 4-7 scales, 8-15
+//   epilogue: four warpgroups, so that setmaxnreg can move registers from the
+//   first two, which need few, to the epilogue's, which holds a 128 x 128
+//   half-accumulator per warpgroup)
 // Output tiles are 128 x 256 with one accumulator (256 tensor-memory
 // columns): two accumulators of 256 columns would leave no room for the stages'
 // scale factors, and 128-column tiles with two accumulators measured slower (an
@@ -123,8 +126,16 @@ struct Cfg {
   static constexpr int STAGING_BUFS = EPI_TMA ? BSP_GEMM_STAGING_BUFS : 0;
   static constexpr int STAGING_BYTES = 1024 * STAGING_BUFS;  // per epilogue warp: buffers of 32 rows x 32 bytes
   static constexpr int SF_WARPS = 4;
-  static constexpr int FIRST_SF_WARP = 2 + EPI_WARPS;
-  static constexpr int THREADS = 64 + (EPI_WARPS + SF_WARPS) * 32;
+  // Four warpgroups: 0 = producer, MMA issuer and two idle warps; 1 = the
+  // scale-factor warps; 2 and 3 = the epilogue.  Warpgroups 0 and 1 give up
+  // registers (WG0_REGS, SF_REGS) so that the epilogue (EPI_REGS) can read the
+  // whole accumulator into registers before handing it back to the MMA warp.
+  static constexpr int FIRST_SF_WARP = 4;
+  static constexpr int FIRST_EPI_WARP = 8;
+  static constexpr int THREADS = 16 * 32;
+  static constexpr int LAUNCH_REGS = 65536 / THREADS;  // 128
+  static constexpr int WG0_REGS = 40, SF_REGS = 88, EPI_REGS = 192;
+  static_assert(128 * (WG0_REGS + SF_REGS + 2 * EPI_REGS) == THREADS * LAUNCH_REGS, "register split");
   static constexpr int BAR_BYTES = 256;
   static constexpr int FIXED_BYTES = EPI_WARPS * STAGING_BYTES + 1024 + BAR_BYTES;
   static constexpr int ACC_COLS = BN;  // one fp32 accumulator
@@ -224,98 +235,103 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   const int first_tile = static_cast<int>(blockIdx.x);
   const int tile_step = static_cast<int>(gridDim.x);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      uint32_t issued[C::STAGES];
-      for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
-      bool ok = true;
-      for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
-        int mb, nb;
-        tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-          tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, mb * C::BM);
-          tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, nb * C::BN);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, mb);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, &full[stage], 0, kb * C::ATOMS,
-                      nb * C::B_BANDS);
-          ++issued[stage];
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+  if (warp < C::FIRST_SF_WARP) {
+    // warpgroup 0: producer, MMA issuer, two idle warps
+    regs_dec<C::WG0_REGS>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        uint32_t stage = 0, phase = 0;
+        uint32_t issued[C::STAGES];
+        for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
+        bool ok = true;
+        for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
+          int mb, nb;
+          tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
+          for (int kb = 0; kb < p.num_kb; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t* st = smem + stage * C::STAGE_BYTES;
+            mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+            tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, mb * C::BM);
+            tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, nb * C::BN);
+            tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, mb);
+            tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, &full[stage], 0, kb * C::ATOMS,
+                        nb * C::B_BANDS);
+            ++issued[stage];
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
-      }
-      if (!ok) {
-        *abort_flag = 1u;
-        raise_error(p.err, kErrTimeout);
-      }
-      // Every issued copy must have landed before the CTA may exit.
-      for (int s = 0; s < C::STAGES; ++s)
-        if (issued[s] && !mbar_wait(&full[s], (issued[s] - 1u) & 1u, nullptr)) raise_error(p.err, kErrTimeout);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      bool ok = true;
-      int it = 0;
-      for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
-        // the epilogue has read the previous tile's accumulator
-        if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
-          ok = false;
-          break;
+        if (!ok) {
+          *abort_flag = 1u;
+          raise_error(p.err, kErrTimeout);
         }
-        tc_fence_after_sync();
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          // the scale warps signal after the stage landed and its scales are in tensor memory
-          if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
+        // Every issued copy must have landed before the CTA may exit.
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued[s] && !mbar_wait(&full[s], (issued[s] - 1u) & 1u, nullptr)) raise_error(p.err, kErrTimeout);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        int it = 0;
+        for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
+          // the epilogue has read the previous tile's accumulator
+          if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sfa_t = tmem + C::ACC_COLS + stage * C::SF_COLS;
-          const uint32_t sfb_t = sfa_t + C::SFA_COLS;
-          const uint64_t adesc = desc_kmajor_swizzled(sbase, C::ROW_BYTES);
-          const uint64_t bdesc = desc_kmajor_swizzled(sbase + C::A_BYTES, C::ROW_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < C::MMAS; ++kk) {
-            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
-            // 32 bytes of K per MMA: advance the start address by 32 >> 4.
-            if constexpr (KIND == kNVF4)
-              tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_nvf4(C::BM, C::BN), sfa_t + 4u * kk,
-                          sfb_t + static_cast<uint32_t>(C::SFB_COLS_PER_MMA * kk), accumulate);
-            else
-              tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8(C::BM, C::BN, static_cast<uint32_t>(kk)),
-                          sfa_t, sfb_t, accumulate);
+          for (int kb = 0; kb < p.num_kb; ++kb) {
+            // the scale warps signal after the stage landed and its scales are in tensor memory
+            if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
+            const uint32_t sfa_t = tmem + C::ACC_COLS + stage * C::SF_COLS;
+            const uint32_t sfb_t = sfa_t + C::SFA_COLS;
+            const uint64_t adesc = desc_kmajor_swizzled(sbase, C::ROW_BYTES);
+            const uint64_t bdesc = desc_kmajor_swizzled(sbase + C::A_BYTES, C::ROW_BYTES);
+  #pragma unroll
+            for (int kk = 0; kk < C::MMAS; ++kk) {
+              const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+              // 32 bytes of K per MMA: advance the start address by 32 >> 4.
+              if constexpr (KIND == kNVF4)
+                tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_nvf4(C::BM, C::BN), sfa_t + 4u * kk,
+                            sfb_t + static_cast<uint32_t>(C::SFB_COLS_PER_MMA * kk), accumulate);
+              else
+                tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8(C::BM, C::BN, static_cast<uint32_t>(kk)),
+                            sfa_t, sfb_t, accumulate);
+            }
+            tc_commit(&empty[stage]);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          tc_commit(&empty[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          if (!ok) break;
+          tc_commit(acc_full);
         }
-        if (!ok) break;
-        tc_commit(acc_full);
+        if (!ok) {
+          *abort_flag = 1u;
+          raise_error(p.err, kErrTimeout);
+        }
+        // No MMA may still be running when tensor memory is freed.
+        tc_commit(drain);
+        if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
       }
-      if (!ok) {
-        *abort_flag = 1u;
-        raise_error(p.err, kErrTimeout);
-      }
-      // No MMA may still be running when tensor memory is freed.
-      tc_commit(drain);
-      if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
     }
-  } else if (warp >= C::FIRST_SF_WARP) {
-    // ------------------------------------------------------------ scale factors
+  } else if (warp < C::FIRST_EPI_WARP) {
+    // ------------------------------------------------------------ scale factors (warpgroup 1)
+    regs_dec<C::SF_REGS>();
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t stage = 0, phase = 0;
     bool ok = true;
@@ -384,8 +400,9 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       raise_error(p.err, kErrTimeout);
     }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;   // 0..7
+    // ------------------------------------------------------------ epilogue (warpgroups 2 and 3)
+    regs_inc<C::EPI_REGS>();
+    const int ew = warp - C::FIRST_EPI_WARP;  // 0..7
     const int q = warp & 3;    // tensor-memory lane quarter this warp may read
     const int half = ew >> 2;  // which half of the tile's columns
     uint8_t* stage_buf = staging + ew * C::STAGING_BYTES;
@@ -459,24 +476,28 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       tc_fence_after_sync();
 
       if (!p.out_f32) {
-        // bf16: read the columns 32 at a time, applying the epilogue and
-        // packing as they arrive, release tensor memory, then store from
-        // registers.
+        // bf16: read all of this warp's columns into registers and hand the
+        // accumulator back at once (the next tile's MMAs start while this
+        // one's epilogue arithmetic runs), then apply alpha, row scale and
+        // bias, pack, and store from registers.
+        uint32_t r[C::EPI_COLS];
+#pragma unroll
+        for (int c = 0; c < C::EPI_COLS / 32; ++c)
+          tmem_ld_32cols(taddr + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+        tmem_ld_wait();
+        release_accumulator();
         uint32_t packed[C::EPI_COLS / 2];
 #pragma unroll
         for (int c = 0; c < C::EPI_COLS / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32cols(taddr + 32u * c, r);
-          tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             // columns 32c + 2i, 2i + 1 are held by lane 8c + i/2
             const uint32_t bw = __shfl_sync(0xFFFFFFFFu, (i & 1) ? bias4.y : bias4.x, 8 * c + (i >> 1));
-            packed[16 * c + i] = pack_bf16x2(__fmaf_rn(__uint_as_float(r[2 * i]), scale, bf16_bits_to_f32(bw & 0xFFFFu)),
-                                             __fmaf_rn(__uint_as_float(r[2 * i + 1]), scale, bf16_bits_to_f32(bw >> 16)));
+            packed[16 * c + i] =
+                pack_bf16x2(__fmaf_rn(__uint_as_float(r[32 * c + 2 * i]), scale, bf16_bits_to_f32(bw & 0xFFFFu)),
+                            __fmaf_rn(__uint_as_float(r[32 * c + 2 * i + 1]), scale, bf16_bits_to_f32(bw >> 16)));
           }
         }
-        release_accumulator();
 #pragma unroll
         for (int j = 0; j < C::EPI_COLS / W_BF16; ++j) {
           const int n0 = col0 + j * W_BF16;
@@ -977,12 +998,15 @@ int launch_skinny(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, c
 
 // CTAs per tile of the skinny kernel: 1, or a split of K over a cluster of up
 // to 4 CTAs when the tiles alone would leave at least half of the SMs without
-// work (few weight panels: N <= ~9K), bounded by the tile's k-blocks.
+// work (few weight panels: N <= ~9K) and every rank keeps at least 16 k-blocks
+// (4096 fp4 elements of K): below that the cluster's start-up and reduction
+// cost more than the extra streams gain (measured: K = 13824 gains 1.5x at
+// S = 3, K = 5120 gains nothing, K = 1536 loses).
 int skinny_split(const DeviceInfo& dev, int64_t tiles, int num_kb) {
   if (tiles * 2 > dev.sm_count) return 1;
   int64_t s = dev.sm_count / tiles;
   s = s < 4 ? s : 4;
-  s = s < num_kb ? s : num_kb;
+  s = s < num_kb / 16 ? s : num_kb / 16;
   return s < 1 ? 1 : static_cast<int>(s);
 }
 

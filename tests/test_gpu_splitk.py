@@ -14,10 +14,11 @@ from tests.test_gpu_gemm import _mxfp8_case, _nvfp4_case, _rand
 
 pytestmark = pytest.mark.gpu
 
-# (M, N, K): few panels (N <= 9K) so that K is split over 2-4 CTAs; ragged N
-# and K, M across the three activation widths, K down to two k-blocks
-SPLIT_SHAPES = [(1, 5120, 13824), (16, 5120, 5120), (33, 1536, 1536), (48, 264, 4096), (5, 1024, 512),
-                (17, 136, 1056), (1, 128, 1024), (40, 2048, 768)]
+# (M, N, K): few panels (N <= 9K) and long K, so that K is split over 2-4
+# CTAs (at least 16 k-blocks of 256 elements per CTA); ragged N and K, M
+# across the three activation widths
+SPLIT_SHAPES = [(1, 5120, 13824), (16, 5120, 8192), (33, 1536, 12288), (48, 264, 16384), (5, 1024, 8192),
+                (17, 136, 12320), (1, 128, 16384), (40, 2048, 8192)]
 
 
 @pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
@@ -27,14 +28,14 @@ def test_split_k_matches_oracle(M, N, K, out_dtype):
     _nvfp4_case(A, W, bias=b, out_dtype=out_dtype)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 5120, 13824), (16, 1536, 1536), (45, 520, 2048)])
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 13824), (16, 1536, 12288), (45, 520, 8192)])
 def test_split_k_per_token(M, N, K):
     A, W, b = _rand(M, N, K, seed=M + N * 3 + K, bias=False)
     _nvfp4_case(A, W, per_token=True, out_dtype=torch.float32)
     _nvfp4_case(A, W, bias=b, per_token=True)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 5120, 5120), (24, 1024, 2048), (7, 264, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 13824), (24, 1024, 8192), (7, 264, 4096)])
 def test_split_k_mxfp8(M, N, K):
     A, W, b = _rand(M, N, K, seed=M + 2 * N + K)
     _mxfp8_case(A, W, bias=b)
@@ -42,7 +43,7 @@ def test_split_k_mxfp8(M, N, K):
 
 @pytest.mark.parametrize("M", [1, 9, 40, 64])
 def test_split_k_8x4_scales(M):
-    N, K = 2048, 5120
+    N, K = 2048, 8192
     A, W, _ = _rand(M, N, K, seed=M + 77, bias=False)
     w = up_bf16(W)
     gs_w, _ = api.nvfp4_global_scale(api.amax(w))
