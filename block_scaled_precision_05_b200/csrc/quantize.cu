@@ -22,6 +22,7 @@
 // scale bytes of a 128x4 tile row gathered by shuffles into one 4-byte store.
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "bsp_device.cuh"
@@ -171,6 +172,35 @@ __device__ __forceinline__ void nvfp4_scale(uint32_t mag, float gs, uint32_t& sf
   const float s = __fmul_rn(div6_rn(amax), gs);
   sfb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
   inv = inv_tab ? inv_tab[sfb] : ((sfb == 0u) ? 0.0f : __fdiv_rn(gs, e4m3_pos_to_f32(sfb)));
+}
+
+// Decode factor fl32(gs / e4m3(b)) without a division per group.  A positive
+// e4m3 value is an integer m in 1..15 times a power of two: m = 8 + f and
+// 2^(E-10) for a normal byte (E, f), m = f and 2^-9 (the scale of E = 1) for
+// a subnormal one.  Scaling by a power of two commutes with rounding while
+// the result stays normal, so fl32(gs / e4m3(b)) = fl32(gs / m) * 2^(10 -
+// max(E, 1)), with fl32(gs / m) taken from lane m of `quot` (quotient_lane).
+// Normal here: gs >= 2688 / max finite > 2^-117 and e4m3(b) <= 480 keep every
+// quotient and product at or above 2^-126; an overflow gives +inf in both
+// forms.  All 32 lanes must take part (a warp shuffle).
+__device__ __forceinline__ float quotient_lane(float gs) {
+  const uint32_t m = lane_id();
+  return (m == 0u || m > 15u) ? 0.0f : __fdiv_rn(gs, static_cast<float>(m));
+}
+
+__device__ __forceinline__ float inv_from_quotients(float quot, uint32_t sfb) {
+  const uint32_t e = (sfb >> 3) & 0xFu, f = sfb & 7u;
+  const float q = __shfl_sync(kFull, quot, e == 0u ? f : 8u + f);  // lane 0 holds 0: b = 0 gives 0
+  const uint32_t e1 = e == 0u ? 1u : e;
+  return __fmul_rn(q, __uint_as_float((137u - e1) << 23));
+}
+
+// NVFP4 scale byte and decode factor of one group from the row's quotients.
+template <class In>
+__device__ __forceinline__ void nvfp4_scale_q(uint32_t mag, float gs, float quot, uint32_t& sfb, float& inv) {
+  const float s = __fmul_rn(div6_rn(In::value(mag)), gs);
+  sfb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
+  inv = inv_from_quotients(quot, sfb);
 }
 
 // Eight elements (one 16-byte chunk) times inv -> eight e2m1 codes in one
@@ -386,6 +416,84 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowblock_kernel(
       }
     }
     __syncthreads();  // red / gs_sh are reused by the next row
+  }
+}
+
+// Per-row (per-token) scale, K = 512 * S * G (hidden sizes 1024, 1536, 2048,
+// 5120): each row by S warps whose threads hold it in registers (thread t of
+// the row's S * 32 owns groups t, t + 32 S, ... : 2G 16-byte loads, all
+// issued at once), the row amax by warp reductions and, for S > 1, a named
+// barrier over the row's warps, then the row quantized from the registers --
+// one DRAM round trip per row.  A block holds blockDim / (32 S) such row
+// teams.  S trades the serial work of one thread (G groups) against barrier
+// and reduction cost: few rows take large S, many rows S = 1.  Rows [M, Mp)
+// write their zero scale bytes only.
+constexpr int kRowTeamMax = 8;  // row teams per block at most
+
+template <class In, class L, int G, int S>
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_rowreg_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t ld_x, float* __restrict__ row_gs,
+    float* __restrict__ row_inv, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  allow_dependent_launch();  // the GEMM that consumes this output may set up meanwhile
+  constexpr int64_t K = 512 * S * G;
+  constexpr int kTeam = 32 * S;
+  __shared__ uint32_t red[2][kRowTeamMax][S];
+  const uint32_t lane = lane_id();
+  const int team = static_cast<int>(threadIdx.x) / kTeam;
+  const int t = static_cast<int>(threadIdx.x) % kTeam;
+  const int teams = static_cast<int>(blockDim.x) / kTeam;
+  const bool quad_lead = (lane & 3u) == 0u;
+  int parity = 0;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * teams + team; r < Mp;
+       r += static_cast<int64_t>(gridDim.x) * teams, parity ^= 1) {
+    const bool live = r < M;
+    const uint16_t* lp = x + r * ld_x + t * 16;
+    uint4 v[G][2];
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      v[i][0] = live ? ldg16(lp + i * 16 * kTeam) : make_uint4(0u, 0u, 0u, 0u);
+      v[i][1] = live ? ldg16(lp + i * 16 * kTeam + 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // group amaxes, kept for the scales; the row amax is their maximum with
+    // +-inf counted as the largest finite value (NaN-ignoring maxima compose)
+    uint32_t gm[G], mag = 0;
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      gm[i] = group_mag16<In>(v[i][0], v[i][1]);
+      mag = max(mag, gm[i]);
+    }
+    mag = min(warp_max(mag), In::kMaxFinite);
+    if constexpr (S > 1) {
+      // the team's warps meet at named barrier 1 + team; red alternates by
+      // row parity, so one barrier per row orders writes against old reads
+      if (lane == 0) red[parity][team][t >> 5] = mag;
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(kTeam) : "memory");
+#pragma unroll
+      for (int w = 0; w < S; ++w) mag = max(mag, red[parity][team][w]);
+    }
+    const float gs = global_scale_from_mag<In>(mag);
+    if (live && t == 0) {
+      if (row_gs) row_gs[r] = gs;
+      if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
+    }
+    const float quot = quotient_lane(gs);
+    uint8_t* cp = codes + r * (K >> 1) + t * 8;
+    uint8_t* sp = sf + L::row_base(r, K >> 6) + (t >> 2) * L::kTileBytes;
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      uint32_t sfb;
+      float inv;
+      nvfp4_scale_q<In>(gm[i], gs, quot, sfb, inv);
+      uint2 w;
+      w.x = nvfp4_codes8<In>(v[i][0], inv);
+      w.y = nvfp4_codes8<In>(v[i][1], inv);
+      const uint32_t s1 = __shfl_down_sync(kFull, sfb, 1);
+      const uint32_t s2 = __shfl_down_sync(kFull, sfb, 2);
+      const uint32_t s3 = __shfl_down_sync(kFull, sfb, 3);
+      if (live) *reinterpret_cast<uint2*>(cp + i * 8 * kTeam) = w;
+      if (quad_lead)
+        *reinterpret_cast<uint32_t*>(sp + i * (kTeam / 4) * L::kTileBytes) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    }
   }
 }
 
@@ -1235,6 +1343,49 @@ int amax_launch(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream, 
   return launch_status();
 }
 
+// Per-token quantize of a row that fits registers (K = 1024, 1536, 2048 or
+// 5120).  Warps per row S: enough that each SM gets about kRowWarpsPerSm of
+// them -- the fewest for many rows, up to one group a thread for a handful of
+// rows; teams per block fill 8 warps where rows allow.
+constexpr int kRowWarpsPerSm = 16;
+
+template <class In, class L>
+int launch_rowreg(const DeviceInfo& dev, const uint16_t* x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x,
+                  float* row_gs, float* row_inv, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
+  const int gk = static_cast<int>(K / 512);  // S * G
+  // warps per live row wanted (padding rows [M, Mp) load nothing); at most 5
+  // groups a thread (K = 5120 on one warp holds 120 registers a thread, and its
+  // low occupancy measured slower than two warps a row at every row count)
+  const int64_t want = ceil_div(static_cast<int64_t>(dev.sm_count) * kRowWarpsPerSm, M);
+  int S = 0;
+  for (int s = 1; s <= gk && s <= 8; ++s)
+    if (gk % s == 0 && gk / s <= 5 && (S == 0 || s <= want)) S = s;
+  auto go = [&](auto k, int s) -> int {
+    const int64_t teams_wanted = ceil_div(Mp, static_cast<int64_t>(dev.sm_count));
+    const int teams = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(teams_wanted, std::min(8 / s, kRowTeamMax))));
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 32 * s * teams, 0) != cudaSuccess || per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+    const int64_t blocks = std::min<int64_t>(ceil_div(Mp, teams), static_cast<int64_t>(dev.sm_count) * per_sm);
+    k<<<static_cast<int>(blocks), 32 * s * teams, 0, stream>>>(x, M, Mp, ld_x, row_gs, row_inv, codes, sf);
+    return BSP_OK;
+  };
+  switch (gk * 16 + S) {
+    case 2 * 16 + 1: return go(nvfp4_quant_rowreg_kernel<In, L, 2, 1>, 1);
+    case 2 * 16 + 2: return go(nvfp4_quant_rowreg_kernel<In, L, 1, 2>, 2);
+    case 3 * 16 + 1: return go(nvfp4_quant_rowreg_kernel<In, L, 3, 1>, 1);
+    case 3 * 16 + 3: return go(nvfp4_quant_rowreg_kernel<In, L, 1, 3>, 3);
+    case 4 * 16 + 1: return go(nvfp4_quant_rowreg_kernel<In, L, 4, 1>, 1);
+    case 4 * 16 + 2: return go(nvfp4_quant_rowreg_kernel<In, L, 2, 2>, 2);
+    case 4 * 16 + 4: return go(nvfp4_quant_rowreg_kernel<In, L, 1, 4>, 4);
+    case 10 * 16 + 2: return go(nvfp4_quant_rowreg_kernel<In, L, 5, 2>, 2);
+    case 10 * 16 + 5: return go(nvfp4_quant_rowreg_kernel<In, L, 2, 5>, 5);
+    default: return BSP_ERR_INVALID_ARG;
+  }
+}
+
 template <class In, class L>
 int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* global_sf, int sf_mode,
                        float* row_gs, float* row_inv_gs, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
@@ -1260,7 +1411,10 @@ int run_nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, co
       }
       rowblock_cap = dev.sm_count * per_sm;
     }
-    if (per_row && Mp <= rowblock_cap) {
+    if (per_row && (K == 1024 || K == 1536 || K == 2048 || K == 5120)) {
+      st = launch_rowreg<In, L>(dev, x, M, Mp, K, ld_x, row_gs, row_inv_gs, codes, sf, stream);
+      if (st != BSP_OK) return st;
+    } else if (per_row && Mp <= rowblock_cap) {
       // few rows: one block per row, all rows in one wave, one memory round trip
       nvfp4_quant_rowblock_kernel<In, L><<<static_cast<int>(Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, row_gs,
                                                                                       row_inv_gs, codes, sf);

@@ -326,7 +326,10 @@ void bspo_nvfp4_quantize_group(const float *x, float gs, uint8_t *sfb_out, uint8
     float inv = (sf == 0.0f) ? 0.0f : gs / sf;
     for (int i = 0; i < 16; ++i) {
         float v = x[i] * inv;
-        codes[i] = (uint8_t)bspo_e2m1_encode((double)v);
+        /* A NaN product (a NaN element, or 0 * inf once the encode scale has
+         * overflowed to +inf) has no e2m1 value; the saturating conversion
+         * the quantizers use gives it the largest positive magnitude, code 7. */
+        codes[i] = isnan(v) ? 7 : (uint8_t)bspo_e2m1_encode((double)v);
     }
     *sfb_out = (uint8_t)sfb;
 }

@@ -35,11 +35,14 @@ SHAPES = [(1, 16), (1, 64), (7, 48), (128, 256), (129, 64), (130, 80), (300, 153
 # reach each of them:
 #
 # nvfp4_quantize / _f16 / _ex (run_nvfp4_quantize):
-#   K % 64 == 0, per-row, round_up(M) <= resident blocks (at most 148 x 8)
-#       nvfp4_quant_rowblock_kernel     test_nvfp4_quantize_per_row_bit_exact (M <= 300),
+#   per-row, K == 1024 / 1536 / 2048 / 5120 (any M)
+#       nvfp4_quant_rowreg_kernel<G>    test_nvfp4_quantize_per_row_bit_exact (1536, 5120),
+#                                       test_dispatch_branch_bit_exact[rowreg-*] (M 1 to 4100)
+#   other K % 64 == 0, per-row, round_up(M) <= resident blocks (at most 148 x 8)
+#       nvfp4_quant_rowblock_kernel     test_nvfp4_quantize_per_row_bit_exact (K 64, 256, 13824),
 #                                       test_dispatch_branch_bit_exact[rowblock-*]
-#   K % 64 == 0, per-row, more rows
-#       nvfp4_quant_k64_kernel<true>    test_dispatch_branch_bit_exact[k64-per-row-*] (M = 4100)
+#   other K % 64 == 0, per-row, more rows
+#       nvfp4_quant_k64_kernel<true>    test_dispatch_branch_bit_exact[k64-per-row-*] (M 2000, 4100)
 #   per-tensor, K == 1024
 #       nvfp4_quant_short_kernel<S=2>   test_dispatch_branch_bit_exact[short-1024-*]
 #   per-tensor, K == 1536
@@ -59,8 +62,13 @@ BRANCH_CASES = [
     # (name, M, K, per_row)
     ("short-1024", 1, 1024, False), ("short-1024", 129, 1024, False), ("short-1024", 300, 1024, False),
     ("short-1024", 4100, 1024, False), ("short-1536", 4100, 1536, False),
-    ("rowblock", 129, 1024, True), ("rowblock", 300, 5120, True),
-    ("k64-per-row", 4100, 1024, True), ("k64-per-row", 4100, 5120, True),
+    # rowreg: every (groups a thread G, warps a row S) the launcher picks
+    ("rowreg", 1, 1024, True), ("rowreg", 4100, 1024, True),          # G1 S2, G2 S1
+    ("rowreg", 1030, 1536, True), ("rowreg", 2000, 1536, True),       # G1 S3, G3 S1
+    ("rowreg", 129, 2048, True), ("rowreg", 1000, 2048, True), ("rowreg", 4100, 2048, True),  # S4, S2, S1
+    ("rowreg", 129, 5120, True), ("rowreg", 4100, 5120, True),        # G2 S5, G5 S2
+    ("rowblock", 129, 3072, True), ("rowblock", 300, 13824, True),
+    ("k64-per-row", 4100, 3072, True), ("k64-per-row", 2000, 4096, True),
 ]
 
 
@@ -116,6 +124,40 @@ def test_nvfp4_quantize_per_row_bit_exact(M, K):
     x = _data(M, K, seed=M + K * 3, kind="special")
     q = api.nvfp4_quantize(up_bf16(x), per_row=True)
     gs, inv = oracle.row_global_scales(x)
+    codes, sf = oracle.nvfp4_quantize(x, gs, per_row=True)
+    assert np.array_equal(down(q.row_gs).view(np.uint32), gs.view(np.uint32))
+    assert np.array_equal(down(q.row_inv_gs).view(np.uint32), inv.view(np.uint32))
+    assert np.array_equal(down(q.codes), codes)
+    assert np.array_equal(down(q.sf), sf)
+
+
+def _wide_range_rows(M, K, seed):
+    """Rows scaled by powers of two across the whole bf16 range, so the
+    per-row scale 2688 / amax runs from ~1e-35 to +inf (a row of the
+    smallest subnormal), plus all-zero, all -0, +-inf and NaN rows."""
+    rng = np.random.default_rng(seed)
+    e = rng.integers(-150, 125, size=(M, 1)).astype(np.float64)
+    x = (rng.standard_normal((M, K)) * np.exp2(e)).astype(np.float32)
+    bits = wl.f32_to_bf16_bits(x)
+    bits[0] = 0
+    bits[1 % M] = 0
+    bits[1 % M, 7] = 0x0001                      # amax 2^-133: gs overflows to +inf
+    bits[2 % M] = 0x8000
+    bits[3 % M, 5] = 0x7F80                      # +inf counts as the largest finite
+    bits[4 % M, 16:32] = 0x7FC1                  # a NaN group
+    bits[4 % M, 40:44] = 0xFFC3                  # negative NaNs among finite values
+    bits[5 % M, :] = wl.f32_to_bf16_bits(np.full(K, 2.0 ** -126, np.float32))
+    return bits
+
+
+@pytest.mark.parametrize("K", [1024, 1536, 2048, 5120])
+@pytest.mark.parametrize("M", [40, 3000])
+def test_per_row_scales_across_the_range(M, K):
+    """The per-token decode factors fl32(gs / e4m3) at the extremes of gs."""
+    x = _wide_range_rows(M, K, seed=M + K)
+    q = api.nvfp4_quantize(up_bf16(x), per_row=True)
+    gs, inv = oracle.row_global_scales(x)
+    assert np.isinf(gs[1 % M]) and gs.min() < 1e-30
     codes, sf = oracle.nvfp4_quantize(x, gs, per_row=True)
     assert np.array_equal(down(q.row_gs).view(np.uint32), gs.view(np.uint32))
     assert np.array_equal(down(q.row_inv_gs).view(np.uint32), inv.view(np.uint32))

@@ -123,6 +123,30 @@ def test_nvfp4_rejects_k_not_multiple_of_16():
         oracle.nvfp4_quantize(np.zeros((2, 24), np.uint16), 1.0)
 
 
+def _nibbles(codes):
+    c = np.asarray(codes, np.uint8)
+    return np.stack([c & 0xF, c >> 4], axis=-1).reshape(c.shape[0], -1)
+
+
+def test_nvfp4_nan_products_encode_as_code_7():
+    # NaN elements are left out of the group amax (6 here: scale byte 1.0,
+    # decode factor 1) and written as code 7; the finite ones are unaffected
+    x = _bf16([[3.0, -6.0, 0.5, 1.0] + [0.0] * 12])
+    x[0, 2], x[0, 3] = 0x7FC1, 0xFFC3
+    codes, sf = oracle.nvfp4_quantize(x, np.float32(1.0))
+    assert sf[0] == 0x38
+    assert list(_nibbles(codes)[0, :4]) == [5, 0xF, 7, 7]
+    # a row whose amax (2^-133) is below 2688 / FLT_MAX: its scale is +inf,
+    # the nonzero elements saturate to +-6 and the zeros (0 * inf) are code 7
+    x = np.zeros((1, 16), np.uint16)
+    x[0, 0], x[0, 1] = 0x0001, 0x8001
+    gs, _ = oracle.row_global_scales(x)
+    assert np.isinf(gs[0])
+    codes, sf = oracle.nvfp4_quantize(x, gs, per_row=True)
+    assert sf[0] == 0x7E  # fl32(2^-133 / 6) * inf = inf saturates to 448
+    assert list(_nibbles(codes)[0]) == [7, 0xF] + [7] * 14
+
+
 # ----------------------------------------------------------------------------- global scales
 def test_weight_amax_ignores_nan_and_caps_inf():
     x = _bf16([1.0, -3.5, 2.0])
