@@ -762,30 +762,47 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
       return norm8<kLN>(ldg16(row + c), ldg16_or(gamma ? gamma + c : nullptr, kBf16OnePair),
                         ldg16_or(bt ? bt + c : nullptr, kBf16NegZeroPair), p);
     };
-    float gs = gs_tensor;
+    float gs = gs_tensor, quot = 0.0f;
     if (kPerRow) {
       uint32_t mag = 0;
       for (int64_t g = lane; g < groups; g += 32)
         mag = max(mag, max(max_sane_mag8<InBf16>(y8(g * 16)), max_sane_mag8<InBf16>(y8(g * 16 + 8))));
       mag = warp_max(mag);
       gs = global_scale_from_mag<InBf16>(mag);
+      quot = quotient_lane(gs);
       if (lane == 0) {
         if (row_gs) row_gs[r] = gs;
         if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
       }
     }
-    for (int64_t c = lane; c < cols4; c += 32) {
+    // warp-uniform trip count: the per-token decode factor takes a shuffle
+    for (int64_t c0 = 0; c0 < cols4; c0 += 32) {
+      const int64_t c = c0 + lane;
       uint32_t sfb = 0;
-      if (c < groups) {
+      if constexpr (kPerRow) {
+        const bool in = c < groups;
+        const uint4 y0 = in ? y8(c * 16) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 y1 = in ? y8(c * 16 + 8) : make_uint4(0u, 0u, 0u, 0u);
+        float inv;
+        nvfp4_scale_q<InBf16>(group_mag16<InBf16>(y0, y1), gs, quot, sfb, inv);  // all lanes
+        if (in) {
+          uint2 w;
+          w.x = nvfp4_codes8<InBf16>(y0, inv);
+          w.y = nvfp4_codes8<InBf16>(y1, inv);
+          *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
+        } else {
+          sfb = 0;  // scale padding columns
+        }
+      } else if (c < groups) {
         const uint4 y0 = y8(c * 16), y1 = y8(c * 16 + 8);
         float inv;
-        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, kPerRow ? nullptr : inv_tab);
+        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, inv_tab);
         uint2 w;
         w.x = nvfp4_codes8<InBf16>(y0, inv);
         w.y = nvfp4_codes8<InBf16>(y1, inv);
         *reinterpret_cast<uint2*>(codes + r * (K >> 1) + c * 8) = w;
       }
-      sf[sfb_row + (c >> 2) * L::kTileBytes + (c & 3)] = static_cast<uint8_t>(sfb);
+      if (c < cols4) sf[sfb_row + (c >> 2) * L::kTileBytes + (c & 3)] = static_cast<uint8_t>(sfb);
     }
   }
 }
@@ -862,14 +879,18 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_sh
         return norm8<kLN>(v[h][s][half], ldg16_or(gp ? gp + s * 512 + half * 8 : nullptr, kBf16OnePair),
                           ldg16_or(bp ? bp + s * 512 + half * 8 : nullptr, kBf16NegZeroPair), p);
       };
-      float gs = gs_tensor;
+      float gs = gs_tensor, quot = 0.0f;
+      uint32_t gm[S];  // per-token: the group amaxes of y, kept for the scales
       if (kPerRow) {
         uint32_t mag = 0;
 #pragma unroll
-        for (int s = 0; s < S; ++s)
-          mag = max(mag, max(max_sane_mag8<InBf16>(y8(s, 0)), max_sane_mag8<InBf16>(y8(s, 1))));
-        mag = warp_max(mag);
+        for (int s = 0; s < S; ++s) {
+          gm[s] = group_mag16<InBf16>(y8(s, 0), y8(s, 1));
+          mag = max(mag, gm[s]);
+        }
+        mag = min(warp_max(mag), InBf16::kMaxFinite);
         gs = global_scale_from_mag<InBf16>(mag);
+        quot = quotient_lane(gs);
         if (live && lane == 0) {
           if (row_gs) row_gs[r] = gs;
           if (row_inv) row_inv[r] = __fdiv_rn(1.0f, gs);
@@ -882,7 +903,10 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_sh
         const uint4 y0 = y8(s, 0), y1 = y8(s, 1);
         uint32_t sfb;
         float inv;
-        nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, kPerRow ? nullptr : inv_tab);
+        if constexpr (kPerRow)
+          nvfp4_scale_q<InBf16>(gm[s], gs, quot, sfb, inv);
+        else
+          nvfp4_scale<InBf16>(group_mag16<InBf16>(y0, y1), gs, sfb, inv, inv_tab);
         uint2 w;
         w.x = nvfp4_codes8<InBf16>(y0, inv);
         w.y = nvfp4_codes8<InBf16>(y1, inv);
