@@ -69,6 +69,10 @@
 #endif
 // Rasterisation: m-blocks per tile group; 0 chooses by operand size (see
 // launch_gemm).
+// Smallest M for which the main kernel runs as CTA pairs (cta_group::2).
+#ifndef BSP_GEMM_PAIR_MIN_M
+#define BSP_GEMM_PAIR_MIN_M 512
+#endif
 #ifndef BSP_GEMM_GROUP_M
 #define BSP_GEMM_GROUP_M 0
 #endif
@@ -99,20 +103,24 @@ constexpr int64_t kSf8MaxM = 64;  // rows of an activation whose scales may be i
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
-template <int KIND, int BN_ = 256>
+template <int KIND, int BN_ = 256, int CG_ = 1>
 struct Cfg {
-  static constexpr int BM = 128;                        // accumulator rows (tensor-memory lanes)
+  static constexpr int BM = 128;                        // accumulator rows (tensor-memory lanes) per CTA
   static constexpr int BN = BN_;                        // output tile columns (256, or 128 for few tiles)
+  static constexpr int CG = CG_;                        // CTAs sharing one MMA (2: a CTA pair)
   static_assert(BN == 256 || BN == 128, "tile width");
+  static_assert(CG == 1 || (CG == 2 && BN == 256), "CTA pairs take 256 x 256 tiles");
+  static constexpr int TILE_M = BM * CG;                // output tile rows
+  static constexpr int B_ROWS = BN / CG;                // rows of B each CTA loads
   static constexpr int ROW_BYTES = KIND == kNVF4 ? BSP_GEMM_NVF4_ROW_BYTES : 128;  // K bytes per row per stage
   static constexpr int MMAS = ROW_BYTES / 32;                                    // per stage, 32 bytes of K each
   static constexpr int ATOMS = KIND == kNVF4 ? ROW_BYTES / 32 : 1;  // 128x4 scale tiles per 128 rows per stage
   static_assert(ROW_BYTES == 128 || ROW_BYTES == 64, "stage row width");
   static constexpr int B_BANDS = BN / 128;              // 128-row bands of B per tile
   static constexpr int A_BYTES = BM * ROW_BYTES;
-  static constexpr int B_BYTES = BN * ROW_BYTES;
+  static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
   static constexpr int SFA_BYTES = ATOMS * 512;
-  static constexpr int SFB_BYTES = B_BANDS * ATOMS * 512;
+  static constexpr int SFB_BYTES = B_BANDS * ATOMS * 512;  // the scales of all BN rows of B, in each CTA
   static constexpr int TX_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // per stage
   static constexpr int STAGE_BYTES = (TX_BYTES + 1023) / 1024 * 1024;
   static constexpr int SFA_COLS = ATOMS * 4;            // per stage, replicated layout
@@ -145,7 +153,7 @@ struct Cfg {
   static_assert(STAGES >= 2, "pipeline depth");
   static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(3 * STAGES + 3 <= BAR_BYTES / 8 - 1, "barrier space");
+  static_assert(4 * STAGES + 4 <= BAR_BYTES / 8 - 1, "barrier space");
 };
 
 struct GemmParams {
@@ -180,12 +188,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int KIND, int BN>
-__global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
+template <int KIND, int BN, int CG>
+__global__ void __launch_bounds__(Cfg<KIND, BN, CG>::THREADS, 1)
     blockscaled_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                             const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-  using C = Cfg<KIND, BN>;
+  using C = Cfg<KIND, BN, CG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
@@ -195,20 +203,33 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   uint64_t* acc_full = sf_ready + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_local = drain + 1;              // pair follower: its scale warps, per stage
+  uint64_t* acc_local = sf_local + C::STAGES;  // pair follower: its epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_local + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
+  // CTA pair: rank 0 (the leader) issues the MMAs for both, and its commits
+  // arrive on the barriers of both CTAs.  The follower's scale and epilogue
+  // warps arrive on barriers of their own CTA; one of its idle warps forwards
+  // each completed phase to the leader with a single cluster-scope arrival (a
+  // cluster-scope release straight from the warps that wrote tensor memory
+  // measured about 1 us per arrival).
+  const uint32_t rank = C::CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0u;
+  constexpr uint32_t kPeerArrivals = C::CG == 2 ? 1u : 0u;  // the follower's forwarded arrival
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_ready[s], C::SF_WARPS);
+      mbar_init(&sf_ready[s], C::SF_WARPS + kPeerArrivals);
+      mbar_init(&sf_local[s], C::SF_WARPS);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, C::EPI_WARPS);
+    mbar_init(acc_empty, C::EPI_WARPS + kPeerArrivals);
+    mbar_init(acc_local, C::EPI_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -221,19 +242,28 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     prefetch_tensormap(&tmD);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (C::CG == 2) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (C::CG == 2)
+    cluster_sync();  // the peer's barriers are initialised before anything arrives on them
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   // Set-up above overlaps the previous kernel under programmatic launch; every
   // global access below comes after its completion.
   grid_dependency_wait();
   const int num_tiles = p.num_m * p.num_n;
-  const int first_tile = static_cast<int>(blockIdx.x);
-  const int tile_step = static_cast<int>(gridDim.x);
+  const int first_tile = static_cast<int>(blockIdx.x) / C::CG;
+  const int tile_step = static_cast<int>(gridDim.x) / C::CG;
 
   if (warp < C::FIRST_SF_WARP) {
     // warpgroup 0: producer, MMA issuer, two idle warps
@@ -248,6 +278,10 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
         for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
           int mb, nb;
           tile_coords(t, p.num_m, p.num_n, p.group_m, mb, nb);
+          // this CTA's 128 rows of A and its share of B's rows (all of them,
+          // or its half in a pair); the scales of all BN rows of B
+          const int a_band = mb * C::CG + static_cast<int>(rank);
+          const int b_row = nb * C::BN + static_cast<int>(rank) * C::B_ROWS;
           for (int kb = 0; kb < p.num_kb; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
               ok = false;
@@ -255,9 +289,9 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             }
             uint8_t* st = smem + stage * C::STAGE_BYTES;
             mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-            tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, mb * C::BM);
-            tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, nb * C::BN);
-            tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, mb);
+            tma_load_2d(st, &tmA, &full[stage], kb * C::ROW_BYTES, a_band * C::BM);
+            tma_load_2d(st + C::A_BYTES, &tmB, &full[stage], kb * C::ROW_BYTES, b_row);
+            tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, &full[stage], 0, kb * C::ATOMS, a_band);
             tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, &full[stage], 0, kb * C::ATOMS,
                         nb * C::B_BANDS);
             ++issued[stage];
@@ -277,20 +311,35 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
+      if (lane == 0 && leader) {
         uint32_t stage = 0, phase = 0;
         bool ok = true;
         int it = 0;
+        constexpr uint16_t kPair = 0x3;  // commits arrive on the barriers of both CTAs of a pair
+        auto commit = [&](uint64_t* bar) {
+          if constexpr (C::CG == 2)
+            tc_commit_pair(bar, kPair);
+          else
+            tc_commit(bar);
+        };
+        // barriers that the peer CTA arrives on are read with cluster-scope acquire
+        auto wait_shared = [&](uint64_t* bar, uint32_t par) {
+          if constexpr (C::CG == 2)
+            return mbar_wait_cluster(bar, par, abort_flag);
+          else
+            return mbar_wait(bar, par, abort_flag);
+        };
         for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
-          // the epilogue has read the previous tile's accumulator
-          if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag)) {
+          // the epilogue (of both CTAs) has read the previous tile's accumulator
+          if (!wait_shared(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
           for (int kb = 0; kb < p.num_kb; ++kb) {
-            // the scale warps signal after the stage landed and its scales are in tensor memory
-            if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
+            // the scale warps (of both CTAs) signal after their stage landed and
+            // its scales are in tensor memory
+            if (!wait_shared(&sf_ready[stage], phase)) {
               ok = false;
               break;
             }
@@ -300,33 +349,81 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             const uint32_t sfb_t = sfa_t + C::SFA_COLS;
             const uint64_t adesc = desc_kmajor_swizzled(sbase, C::ROW_BYTES);
             const uint64_t bdesc = desc_kmajor_swizzled(sbase + C::A_BYTES, C::ROW_BYTES);
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < C::MMAS; ++kk) {
               const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
               // 32 bytes of K per MMA: advance the start address by 32 >> 4.
-              if constexpr (KIND == kNVF4)
-                tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_nvf4(C::BM, C::BN), sfa_t + 4u * kk,
-                            sfb_t + static_cast<uint32_t>(C::SFB_COLS_PER_MMA * kk), accumulate);
-              else
-                tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8(C::BM, C::BN, static_cast<uint32_t>(kk)),
-                            sfa_t, sfb_t, accumulate);
+              if constexpr (KIND == kNVF4) {
+                const uint32_t idesc = idesc_nvf4(C::TILE_M, C::BN);
+                const uint32_t sfb_k = sfb_t + static_cast<uint32_t>(C::SFB_COLS_PER_MMA * kk);
+                if constexpr (C::CG == 2)
+                  tc_mma_nvf4_pair(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t + 4u * kk, sfb_k, accumulate);
+                else
+                  tc_mma_nvf4(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t + 4u * kk, sfb_k, accumulate);
+              } else {
+                const uint32_t idesc = idesc_mxf8(C::TILE_M, C::BN, static_cast<uint32_t>(kk));
+                if constexpr (C::CG == 2)
+                  tc_mma_mxf8_pair(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t, sfb_t, accumulate);
+                else
+                  tc_mma_mxf8(tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, sfa_t, sfb_t, accumulate);
+              }
             }
-            tc_commit(&empty[stage]);
+            commit(&empty[stage]);
             if (++stage == C::STAGES) {
               stage = 0;
               phase ^= 1u;
             }
           }
           if (!ok) break;
-          tc_commit(acc_full);
+          commit(acc_full);
         }
         if (!ok) {
           *abort_flag = 1u;
           raise_error(p.err, kErrTimeout);
         }
         // No MMA may still be running when tensor memory is freed.
-        tc_commit(drain);
+        commit(drain);
         if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
+      } else if (lane == 0) {
+        // pair follower: its MMAs are issued by the leader, whose last commit
+        // arrives here too
+        if (!mbar_wait(drain, 0u, nullptr)) raise_error(p.err, kErrTimeout);
+      }
+    } else if (C::CG == 2 && !leader && lane == 0) {
+      // pair follower, warp 2: each stage its scale warps complete, one
+      // arrival on the leader's sf_ready; warp 3: each accumulator its
+      // epilogue releases, one arrival on the leader's acc_empty
+      bool ok = true;
+      if (warp == 2) {
+        const uint32_t peer = mapa_shared(smem_u32(sf_ready), 0u);
+        uint32_t stage = 0, phase = 0;
+        for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
+          for (int kb = 0; kb < p.num_kb; ++kb) {
+            if (!mbar_wait(&sf_local[stage], phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_remote_relaxed(peer + 8u * stage);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      } else if (warp == 3) {
+        const uint32_t peer = mapa_shared(smem_u32(acc_empty), 0u);
+        int it = 0;
+        for (int t = first_tile; t < num_tiles && ok; t += tile_step, ++it) {
+          if (!mbar_wait(acc_local, static_cast<uint32_t>(it) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_remote_relaxed(peer);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1u;
+        raise_error(p.err, kErrTimeout);
       }
     }
   } else if (warp < C::FIRST_EPI_WARP) {
@@ -335,6 +432,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t stage = 0, phase = 0;
     bool ok = true;
+    uint64_t* sf_mine = leader ? sf_ready : sf_local;  // the follower's phases are forwarded
     for (int t = first_tile; t < num_tiles && ok; t += tile_step) {
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag)) {
@@ -388,7 +486,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_ready[stage]);
+        if (lane == 0) mbar_arrive(&sf_mine[stage]);
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -445,10 +543,11 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       }
     };
 
+    uint64_t* acc_mine = leader ? acc_empty : acc_local;  // the follower's releases are forwarded
     auto release_accumulator = [&]() {
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) mbar_arrive(acc_mine);
     };
 
     int it = 0;
@@ -460,7 +559,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       // (lane j: columns col0 + 4j .. 4j + 3), and handed to every lane by
       // shuffles while the accumulator is read.
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * C::EPI_COLS);
-      const int row0 = mb * C::BM + q * 32;
+      const int row0 = mb * C::TILE_M + static_cast<int>(rank) * C::BM + q * 32;
       const int row = row0 + static_cast<int>(lane);
       float scale = alpha;
       if (p.row_scale != nullptr && row < p.M) scale = __fmul_rn(alpha, __ldg(p.row_scale + row));
@@ -468,7 +567,9 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       uint2 bias4 = make_uint2(0u, 0u);
       if (p.bias != nullptr && col0 + 4 * static_cast<int>(lane) < p.N)
         bias4 = __ldg(reinterpret_cast<const uint2*>(p.bias + col0 + 4 * static_cast<int>(lane)));
-      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)) {
+      const bool got = C::CG == 2 ? mbar_wait_cluster(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag)
+                                  : mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag);
+      if (!got) {
         *abort_flag = 1u;
         raise_error(p.err, kErrTimeout);
         break;
@@ -544,11 +645,18 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (C::CG == 2)
+    cluster_sync();  // no CTA of the pair leaves while the other may still signal it
+  else
+    __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (C::CG == 2)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -1074,33 +1182,34 @@ int encode_output(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
   return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_INVALID_ARG;
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, int CG = 1>
 int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                 int64_t row_bytes, int64_t tiles_per_band, const CUtensorMap& tmD, GemmParams p,
                 cudaStream_t stream) {
-  using C = Cfg<KIND, BN>;
+  using C = Cfg<KIND, BN, CG>;
   CUtensorMap tmA, tmB, tmSFA, tmSFB;
   int st;
   if ((st = encode_operand(&tmA, A, p.M, row_bytes, C::BM, C::ROW_BYTES)) != BSP_OK) return st;
-  if ((st = encode_operand(&tmB, B, p.N, row_bytes, C::BN, C::ROW_BYTES)) != BSP_OK) return st;
+  if ((st = encode_operand(&tmB, B, p.N, row_bytes, C::B_ROWS, C::ROW_BYTES)) != BSP_OK) return st;
   if ((st = encode_scales(&tmSFA, sfA, ceil_div(p.M, 128), tiles_per_band, C::ATOMS, 1)) != BSP_OK) return st;
   if ((st = encode_scales(&tmSFB, sfB, ceil_div(p.N, 128), tiles_per_band, C::ATOMS, C::B_BANDS)) != BSP_OK)
     return st;
   p.num_kb = static_cast<int>(ceil_div(row_bytes, C::ROW_BYTES));
-  auto kernel = blockscaled_gemm_kernel<KIND, BN>;
+  auto kernel = blockscaled_gemm_kernel<KIND, BN, CG>;
   static bool attr_set[64] = {};
   if (!attr_set[dev.id]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return launch_status();
     attr_set[dev.id] = true;
   }
-  p.num_m = static_cast<int>(ceil_div(p.M, C::BM));
+  p.num_m = static_cast<int>(ceil_div(p.M, C::TILE_M));
   p.num_n = static_cast<int>(ceil_div(p.N, C::BN));
   const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
-  const int ctas = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  // one CTA (or CTA pair) per SM (pair of SMs), each looping over its tiles
+  int64_t groups = dev.sm_count / CG;
+  if (tiles < groups) groups = tiles;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -1109,6 +1218,20 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if constexpr (CG == 2) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    cfg.gridDim = dim3(static_cast<unsigned>(groups * 2), 1, 1);
+    int resident = 0;  // no more pairs than are resident at once
+    if (cudaOccupancyMaxActiveClusters(&resident, kernel, &cfg) != cudaSuccess) return launch_status();
+    if (resident < 1) return BSP_ERR_CUDA;  // a pair does not fit: nothing launched
+    if (groups > resident) groups = resident;
+  }
+  const int ctas = static_cast<int>(groups * CG);
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
   if (BSP_GEMM_GROUP_M > 0) {
     p.group_m = BSP_GEMM_GROUP_M < p.num_m ? BSP_GEMM_GROUP_M : p.num_m;
   } else {
@@ -1119,9 +1242,9 @@ int launch_gemm(const DeviceInfo& dev, const uint8_t* A, const uint8_t* sfA, con
     const int64_t b_bytes = static_cast<int64_t>(p.N) * row_bytes * 17 / 16;
     int64_t g;
     if (b_bytes < (32ll << 20)) {
-      g = ceil_div(2ll * ctas, p.num_n);
+      g = ceil_div(2ll * groups, p.num_n);
     } else {
-      const int64_t a_panel = static_cast<int64_t>(C::BM) * row_bytes * 17 / 16;
+      const int64_t a_panel = static_cast<int64_t>(C::TILE_M) * row_bytes * 17 / 16;
       g = (24ll << 20) / (a_panel > 0 ? a_panel : 1);
     }
     g = g < 8 ? 8 : g;
@@ -1191,6 +1314,9 @@ int run_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
   // (for small M the weight stream, not the tensor pipe, sets the time)
   if (ceil_div(M, 128) * ceil_div(N, 128) <= dev.sm_count)
     return launch_gemm<KIND, 128>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
+  // many tiles: CTA pairs with 256 x 256 tiles, half of B per SM
+  if (M >= BSP_GEMM_PAIR_MIN_M)
+    return launch_gemm<KIND, 256, 2>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
   return launch_gemm<KIND, 256>(dev, A, sfA, B, sfB, row_bytes, tiles_per_band, tmD, p, stream);
 }
 

@@ -120,6 +120,36 @@ def test_mxfp8_gemm_shapes(M, N, K, out_dtype):
     _mxfp8_case(A, W, bias=b, out_dtype=out_dtype)
 
 
+# Shapes that take the CTA-pair form of the main kernel (M >= 512 and more
+# 128 x 128 tiles than SMs): 256 x 256 tiles over two CTAs, each loading its
+# 128 rows of A and half of B.  Ragged M where the second CTA's rows are all
+# past M (600, 1000), N whose last tile leaves the second CTA's half of B past
+# N (2568), a K tail shorter than a stage (352), several tiles per pair with
+# more K stages than the ring (4096 x 4096 x 2048).
+PAIR_SHAPES = [(600, 4096, 256), (1000, 2568, 352), (4096, 4096, 2048), (2100, 1536, 1536)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_nvfp4_gemm_cta_pairs(M, N, K, out_dtype):
+    A, W, b = _rand(M, N, K, seed=M + 3 * N + K)
+    rows = None if M * N <= 4096 * 4096 else band_rows(M, sample_bands(M, 4, seed=1))
+    _nvfp4_case(A, W, b, rows=rows, out_dtype=out_dtype)
+
+
+@pytest.mark.parametrize("M,N,K", [(1100, 2304, 1024), (640, 4104, 512)])
+def test_nvfp4_gemm_cta_pairs_per_token(M, N, K):
+    A, W, b = _rand(M, N, K, seed=M + N)
+    _nvfp4_case(A, W, b, per_token=True)
+
+
+@pytest.mark.parametrize("M,N,K", [(700, 4096, 256), (1030, 2568, 384)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_mxfp8_gemm_cta_pairs(M, N, K, out_dtype):
+    A, W, b = _rand(M, N, K, seed=M + 7 * N + K)
+    _mxfp8_case(A, W, b, out_dtype=out_dtype)
+
+
 def test_one_hot_scale_through_the_tensor_core():
     """All codes 1.0 and all scales 1.0, except one scale byte of A set to 2.0:
     exactly the 16 products of that (row, group) double, so only that output row
