@@ -10,7 +10,7 @@
 //   vllm-omni mxfp8_config.py, NPUMxfp8LinearMethod._quant_matmul.
 //
 // Design (persistent, one CTA per SM, warp-specialised):
-//   warp 0      TMA producer: per stage, the tile's 128 rows of A and BN rows
+//   warp 0      TMA producer: per stage, the CTA's 128 rows of A and its rows
 //               of B (128 bytes of K each, 128-byte swizzle) plus the matching
 //               128x4 scale tiles, into shared memory; completion is counted on
 //               the stage's mbarrier.
@@ -32,10 +32,24 @@
 //               round once, stage 32 rows x 32 bytes in swizzled shared memory
 //               and write them with TMA stores (full 32-byte sectors;
 //               rows/columns past M/N clipped).
-//   (roles by warp index: 0 producer, 1 MMA, 2-3 idle, 4-7 scales, 8-15
-//   epilogue: four warpgroups, so that setmaxnreg can move registers from the
-//   first two, which need few, to the epilogue's, which holds a 128 x 128
-//   half-accumulator per warpgroup)
+//   (roles by warp index: 0 producer, 1 MMA, 2-3 idle (relays in a pair
+//   follower), 4-7 scales, 8-15 epilogue: four warpgroups, so that setmaxnreg
+//   can move registers from the first two, which need few, to the epilogue's,
+//   which holds a 128 x 128 half-accumulator per warpgroup)
+// CTA pairs (CG = 2, large M): a cluster of two CTAs computes a 256 x 256
+// tile with tcgen05.mma.cta_group::2.  Each CTA loads its 128 rows of A and
+// 128 of the tile's 256 rows of B (the MMA reads both CTAs' shared memory and
+// writes each CTA's 128 accumulator rows into its own tensor memory), and the
+// scale tiles of all 256 rows of B, which each CTA's scale warps write into
+// its own tensor memory.  Per SM that is 38 KB of operands per stage instead
+// of 54 KB for the same MMA work, which is what sets the stage rate: the SMs
+// take in operands from L2 more slowly than the tensor pipe consumes them.
+// The leader (rank 0) issues the MMAs and multicasts its commits to both
+// CTAs' barriers; the follower's scale and epilogue warps arrive on barriers
+// of their own CTA, and its idle warps 2 and 3 relay each completed phase to
+// the leader with one relaxed cluster-scope arrival (an arrival with
+// cluster-scope release from the warps that had just written tensor memory
+// took about 1 us under load).
 // Output tiles are 128 x 256 with one accumulator (256 tensor-memory
 // columns): two accumulators of 256 columns would leave no room for the stages'
 // scale factors, and 128-column tiles with two accumulators measured slower (an
