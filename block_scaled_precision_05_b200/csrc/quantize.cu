@@ -623,7 +623,8 @@ __device__ __forceinline__ uint4 layernorm8(const uint4& xv, const uint4& gv, co
     const float2 d = add2_rn(InBf16::values2(xw[i]), nm2);  // x - mean, rounded once
     const float2 t = mul2_rn(mul2_rn(d, r2), InBf16::values2(gw[i]));
     // the shift as scalar adds: a packed add right after a packed multiply has
-    // been seen fused into one multiply-add (one rounding instead of two)
+    // been seen fused into one multiply-add (one rounding instead of two), even
+    // with contraction switched off for this file
     const float2 b2 = InBf16::values2(bw[i]);
     const float2 y = make_float2(__fadd_rn(t.x, b2.x), __fadd_rn(t.y, b2.y));
     const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
