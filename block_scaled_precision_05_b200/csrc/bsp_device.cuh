@@ -187,7 +187,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 
 // ----------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), loads into this CTA's shared memory, completion
-// counted in bytes on an mbarrier.  No multicast anywhere in this library.
+// counted in bytes on an mbarrier.  No TMA or bulk load in this library uses
+// multicast (the only multicast is tcgen05.commit's arrival on the barriers
+// of a CTA pair).
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
