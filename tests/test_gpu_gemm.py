@@ -150,6 +150,43 @@ def test_mxfp8_gemm_cta_pairs(M, N, K, out_dtype):
     _mxfp8_case(A, W, b, out_dtype=out_dtype)
 
 
+@pytest.mark.parametrize("M,N,K,kind", [(32760, 1536, 1536, "nvfp4"), (600, 4096, 256, "nvfp4"),
+                                         (1100, 2304, 1024, "per_token"), (2100, 4096, 1024, "mxfp8")])
+def test_cta_pair_gemm_relaunches_are_bit_identical(M, N, K, kind):
+    """The pair form hands stage and accumulator phases from one CTA to the
+    other; relaunched on the same inputs (back to back, no synchronisation in
+    between) it must give the same bits every time."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + N + K)
+    A = torch.randn((M, K), generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g, device=DEV) / K ** 0.5).to(torch.bfloat16)
+    b = (torch.randn((N,), generator=g, device=DEV) * 0.01).to(torch.bfloat16)
+    if kind == "mxfp8":
+        layer = api.MXFP8Linear(W, b)
+        aq = api.mxfp8_quantize(A)
+
+        def run(out):
+            return api.mxfp8_gemm(aq, layer.weight, None, layer.bias, out=out)
+    else:
+        layer = api.NVFP4Linear(W, b, per_token=kind == "per_token")
+        aq = layer.quantize_input(A)
+        rs = aq.row_inv_gs if kind == "per_token" else None
+
+        def run(out):
+            return api.nvfp4_gemm(aq, layer.weight, layer.alpha, rs, layer.bias, out=out)
+    ref = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    run(ref)
+    outs = [torch.full_like(ref, float("nan")) for _ in range(4)]
+    for _ in range(8):
+        for o in outs:
+            run(o)
+        torch.cuda.synchronize()
+        assert all(torch.equal(o, ref) for o in outs)
+        for o in outs:
+            o.fill_(float("nan"))
+    assert api.device_status() == 0
+
+
 def test_one_hot_scale_through_the_tensor_core():
     """All codes 1.0 and all scales 1.0, except one scale byte of A set to 2.0:
     exactly the 16 products of that (row, group) double, so only that output row
