@@ -187,6 +187,28 @@ def test_cta_pair_gemm_relaunches_are_bit_identical(M, N, K, kind):
     assert api.device_status() == 0
 
 
+@pytest.mark.parametrize("M,N,K", [(600, 4096, 256), (300, 520, 1024)])  # CTA pairs; one CTA per tile
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_strided_output_without_alpha_or_bias(M, N, K, out_dtype):
+    """D written into a column slice of a wider buffer (row stride N + 24):
+    the columns past N keep their contents; alpha and bias absent (alpha 1)."""
+    A, W, _ = _rand(M, N, K, seed=M * 3 + N, bias=False)
+    w = up_bf16(W)
+    gs_w, _ = api.nvfp4_global_scale(api.amax(w))
+    wq = api.nvfp4_quantize(w, gs_w)
+    aq = api.nvfp4_quantize(up_bf16(A), torch.ones(1, device=DEV))
+    wide = torch.full((M, N + 24), float("nan"), dtype=out_dtype, device=DEV)
+    D = api.nvfp4_gemm(aq, wq, None, None, None, out_dtype=out_dtype, out=wide[:, :N])
+    assert api.device_status() == 0
+    assert D.stride(0) == N + 24
+    assert torch.isnan(wide[:, N:]).all()
+    gso = oracle.nvfp4_global_scale(oracle.amax_bf16(W))
+    cb, sb = oracle.nvfp4_quantize(W, gso)
+    ca, sa = oracle.nvfp4_quantize(A, 1.0)
+    ref, bound = oracle.linear_reference(oracle.nvfp4_dequantize(ca, sa, K), oracle.nvfp4_dequantize(cb, sb, K))
+    assert_gemm_close(D, ref, bound, f"strided D, no alpha / bias, M={M}")
+
+
 def test_one_hot_scale_through_the_tensor_core():
     """All codes 1.0 and all scales 1.0, except one scale byte of A set to 2.0:
     exactly the 16 products of that (row, group) double, so only that output row
