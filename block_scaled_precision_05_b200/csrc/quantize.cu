@@ -597,41 +597,49 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quant_generic_kernel(
 constexpr int kNormWarps = kQuantThreads / 32;
 constexpr uint32_t kBf16OnePair = 0x3F803F80u, kBf16NegZeroPair = 0x80008000u;
 
-// Eight normalised outputs as bf16 pairs (RMSNorm).
-__device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const uint4& gv, float rstd) {
-  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+// Eight normalised outputs as bf16 pairs (RMSNorm), gamma as fp32 pairs.
+__device__ __forceinline__ uint4 rmsnorm8(const uint4& xv, const float2 (&g)[4], float rstd) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
   const float2 r2 = make_float2(rstd, rstd);
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     // two fp32 products per packed instruction, each rounded as a scalar one
-    const float2 y = mul2_rn(mul2_rn(InBf16::values2(xw[i]), r2), InBf16::values2(gw[i]));
+    const float2 y = mul2_rn(mul2_rn(InBf16::values2(xw[i]), r2), g[i]);
     const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
     memcpy(&o[i], &h, 4);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Eight normalised outputs as bf16 pairs (LayerNorm).
-__device__ __forceinline__ uint4 layernorm8(const uint4& xv, const uint4& gv, const uint4& bv, float mean,
+// Eight normalised outputs as bf16 pairs (LayerNorm), gamma and beta as fp32 pairs.
+__device__ __forceinline__ uint4 layernorm8(const uint4& xv, const float2 (&g)[4], const float2 (&b)[4], float mean,
                                             float rstd) {
-  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
   const float2 nm2 = make_float2(-mean, -mean), r2 = make_float2(rstd, rstd);
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 d = add2_rn(InBf16::values2(xw[i]), nm2);  // x - mean, rounded once
-    const float2 t = mul2_rn(mul2_rn(d, r2), InBf16::values2(gw[i]));
+    const float2 t = mul2_rn(mul2_rn(d, r2), g[i]);
     // the shift as scalar adds: a packed add right after a packed multiply has
     // been seen fused into one multiply-add (one rounding instead of two), even
     // with contraction switched off for this file
-    const float2 b2 = InBf16::values2(bw[i]);
-    const float2 y = make_float2(__fadd_rn(t.x, b2.x), __fadd_rn(t.y, b2.y));
+    const float2 y = make_float2(__fadd_rn(t.x, b[i].x), __fadd_rn(t.y, b[i].y));
     const __nv_bfloat162 h = __floats2bfloat162_rn(y.x, y.y);
     memcpy(&o[i], &h, 4);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
+
+// Eight bf16 values as fp32 pairs (exact).
+struct Pairs8 {
+  float2 v[4];
+  __device__ __forceinline__ explicit Pairs8(const uint4& w)
+      : v{InBf16::values2(w.x), InBf16::values2(w.y), InBf16::values2(w.z), InBf16::values2(w.w)} {}
+  __device__ __forceinline__ Pairs8(const float4& a, const float4& b)
+      : v{make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)} {}
+};
 
 // The per-row parameters of either norm and its elementwise map.
 struct NormRow {
@@ -640,11 +648,11 @@ struct NormRow {
 };
 
 template <bool kLN>
-__device__ __forceinline__ uint4 norm8(const uint4& xv, const uint4& gv, const uint4& bv, const NormRow& p) {
+__device__ __forceinline__ uint4 norm8(const uint4& xv, const Pairs8& g, const Pairs8& b, const NormRow& p) {
   if constexpr (kLN)
-    return layernorm8(xv, gv, bv, p.mean, p.rstd);
+    return layernorm8(xv, g.v, b.v, p.mean, p.rstd);
   else
-    return rmsnorm8(xv, gv, p.rstd);
+    return rmsnorm8(xv, g.v, p.rstd);
 }
 
 // Exact row statistics from the row in global memory (the rare path; the row
@@ -760,8 +768,8 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
       if (kLN && row_mean) row_mean[r] = p.mean;
     }
     auto y8 = [&](int64_t c) {  // normalised elements [c, c + 8) as bf16 pairs
-      return norm8<kLN>(ldg16(row + c), ldg16_or(gamma ? gamma + c : nullptr, kBf16OnePair),
-                        ldg16_or(bt ? bt + c : nullptr, kBf16NegZeroPair), p);
+      return norm8<kLN>(ldg16(row + c), Pairs8(ldg16_or(gamma ? gamma + c : nullptr, kBf16OnePair)),
+                        Pairs8(ldg16_or(bt ? bt + c : nullptr, kBf16NegZeroPair)), p);
     };
     float gs = gs_tensor, quot = 0.0f;
     if (kPerRow) {
@@ -811,8 +819,9 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
 // K = 512 * S (S = 3, 4: the Wan-1.3B hidden size 1536 among them): the same
 // arithmetic with every row read from DRAM once and kept in registers.  Lane
 // l holds elements [512 s + 16 l, 512 s + 16 l + 16) of the row for s < S (one
-// group of 16 per slab); gamma (and beta) are re-read per row (they stay in
-// L1).  A warp loads R rows before working on the first, like
+// group of 16 per slab); gamma (and beta) are converted to fp32 once per block
+// into shared memory, in the order the lanes read them.  A warp loads R rows
+// before working on the first, like
 // nvfp4_quant_short_kernel.  Rows [M, Mp) are scale padding: y = 0, so their
 // scale bytes are 0.
 #ifndef BSP_RMSNORM_ROWS
@@ -840,8 +849,24 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_sh
   if constexpr (!kPerRow) build_inv_table(inv_tab, gs_tensor);
   normstats::ExactSums* xs = &xsum[threadIdx.x >> 5];
   const bool quad_lead = (lane & 3u) == 0u;
-  const uint16_t* gp = gamma ? gamma + lane * 16 : nullptr;  // re-read per row from L1
-  const uint16_t* bp = (kLN && beta) ? beta + lane * 16 : nullptr;
+  // float4 [((s * 2 + half) * 2 + j) * 32 + l] holds elements [512 s + 16 l +
+  // 8 half + 4 j, +4) of gamma (beta): for fixed (s, half, j) the 32 lanes read
+  // one contiguous 512-byte line.  Absent: gamma 1, beta -0 (exact identities).
+  constexpr int kQuads = S * 128;
+  __shared__ float4 g_s[kQuads];
+  __shared__ float4 b_s[kLN ? kQuads : 1];
+  for (int i = threadIdx.x; i < kQuads; i += blockDim.x) {
+    const int c = (i >> 7) * 512 + (i & 31) * 16 + ((i >> 6) & 1) * 8 + ((i >> 5) & 1) * 4;
+    auto quad = [&](const uint16_t* t, float fill) {
+      if (!t) return make_float4(fill, fill, fill, fill);
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(t + c));
+      const float2 a = InBf16::values2(w.x), b = InBf16::values2(w.y);
+      return make_float4(a.x, a.y, b.x, b.y);
+    };
+    g_s[i] = quad(gamma, 1.0f);
+    if constexpr (kLN) b_s[i] = quad(beta, -0.0f);
+  }
+  __syncthreads();
   for (int64_t r0 = R * warp; r0 < Mp; r0 += R * nwarps) {
     uint4 v[R][S][2];
 #pragma unroll
@@ -877,8 +902,11 @@ __global__ void __launch_bounds__(kQuantThreads, kMinBlocks) nvfp4_norm_quant_sh
       }
       // y is recomputed where it is needed rather than held (register pressure)
       auto y8 = [&](int s, int half) {
-        return norm8<kLN>(v[h][s][half], ldg16_or(gp ? gp + s * 512 + half * 8 : nullptr, kBf16OnePair),
-                          ldg16_or(bp ? bp + s * 512 + half * 8 : nullptr, kBf16NegZeroPair), p);
+        const int q = (s * 2 + half) * 64 + static_cast<int>(lane);
+        if constexpr (kLN)
+          return norm8<kLN>(v[h][s][half], Pairs8(g_s[q], g_s[q + 32]), Pairs8(b_s[q], b_s[q + 32]), p);
+        else
+          return norm8<kLN>(v[h][s][half], Pairs8(g_s[q], g_s[q + 32]), Pairs8(g_s[q], g_s[q + 32]), p);
       };
       float gs = gs_tensor, quot = 0.0f;
       uint32_t gm[S];  // per-token: the group amaxes of y, kept for the scales
