@@ -728,9 +728,26 @@ __device__ __forceinline__ uint4 ldg16_or(const uint16_t* p, uint32_t fill) {
   return p ? ldg16(p) : make_uint4(fill, fill, fill, fill);
 }
 
+// gamma (and beta) as fp32 in the dynamic shared memory of a block of the
+// general norm kernel: float4 [((g >> 5) * 4 + 2 half + j) * 32 + (g & 31)]
+// holds elements [16 g + 8 half + 4 j, +4), so that the 32 lanes of a warp
+// (groups g = lane + 32 i) read one contiguous 512-byte line per 16-byte load;
+// beta follows gamma.  Used while both fit in kNormStageMaxBytes: on a
+// 32760 x 5120 activation (the Wan-14B hidden size) staging took RMSNorm from 113 to 110 us and LayerNorm
+// from 177 to 170 us (20 and 40 KB a block), but 54 KB at K = 13824 (RMSNorm)
+// made it 17% slower, the shared memory taking L1 from the row re-reads.
+constexpr size_t kNormStageMaxBytes = 40 * 1024;
+static_assert(kNormStageMaxBytes + 4096 <= 48 * 1024, "staged bytes + static shared memory within the default limit");
+__host__ __device__ constexpr int64_t norm_stage_quads(int64_t K) { return ((K >> 4) + 31) / 32 * 128; }
+inline size_t norm_stage_bytes(int64_t K, bool ln) {
+  return static_cast<size_t>(norm_stage_quads(K)) * sizeof(float4) * (ln ? 2 : 1);
+}
+
 // Any K % 16 == 0: the statistics pass(es), then (per-token scales) the row
 // amax of y, then the groups; the later passes re-read the row from cache.
-template <class L, bool kPerRow, bool kLN>
+// kStaged: gamma and beta from shared memory as fp32 (converted once per
+// block), else re-read as bf16 for every row.
+template <class L, bool kPerRow, bool kLN, bool kStaged>
 __global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t Mp, int64_t K, int64_t ld_x, const uint16_t* __restrict__ gamma,
     const uint16_t* __restrict__ beta, float eps, const float* __restrict__ gs_ptr, float* __restrict__ row_gs,
@@ -748,6 +765,23 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
   if constexpr (!kPerRow) build_inv_table(inv_tab, gs_tensor);
   normstats::ExactSums* xs = &xsum[threadIdx.x >> 5];
   const uint16_t* bt = kLN ? beta : nullptr;
+  extern __shared__ float4 aff[];  // kStaged: gamma, then beta
+  const int64_t nq = norm_stage_quads(K);
+  if constexpr (kStaged) {
+    for (int64_t i = threadIdx.x; i < nq; i += blockDim.x) {
+      const int64_t g = (i >> 7) * 32 + (i & 31);
+      const int64_t c = g * 16 + ((i >> 6) & 1) * 8 + ((i >> 5) & 1) * 4;
+      auto quad = [&](const uint16_t* t, float fill) {
+        if (!t || g >= groups) return make_float4(fill, fill, fill, fill);
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(t + c));
+        const float2 a = InBf16::values2(w.x), b = InBf16::values2(w.y);
+        return make_float4(a.x, a.y, b.x, b.y);
+      };
+      aff[i] = quad(gamma, 1.0f);
+      if constexpr (kLN) aff[nq + i] = quad(bt, -0.0f);
+    }
+    __syncthreads();
+  }
 
   for (int64_t r = warp; r < Mp; r += nwarps) {
     const int64_t sfb_row = L::row_base(r, cols4 >> 2);
@@ -768,8 +802,15 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_norm_quant_kernel(
       if (kLN && row_mean) row_mean[r] = p.mean;
     }
     auto y8 = [&](int64_t c) {  // normalised elements [c, c + 8) as bf16 pairs
-      return norm8<kLN>(ldg16(row + c), Pairs8(ldg16_or(gamma ? gamma + c : nullptr, kBf16OnePair)),
-                        Pairs8(ldg16_or(bt ? bt + c : nullptr, kBf16NegZeroPair)), p);
+      if constexpr (kStaged) {
+        const int64_t g = c >> 4;
+        const int64_t q = ((g >> 5) * 4 + ((c >> 3) & 1) * 2) * 32 + (g & 31);
+        const Pairs8 gp(aff[q], aff[q + 32]);
+        return norm8<kLN>(ldg16(row + c), gp, kLN ? Pairs8(aff[nq + q], aff[nq + q + 32]) : gp, p);
+      } else {
+        return norm8<kLN>(ldg16(row + c), Pairs8(ldg16_or(gamma ? gamma + c : nullptr, kBf16OnePair)),
+                          Pairs8(ldg16_or(bt ? bt + c : nullptr, kBf16NegZeroPair)), p);
+      }
     };
     float gs = gs_tensor, quot = 0.0f;
     if (kPerRow) {
@@ -1367,9 +1408,10 @@ __global__ void debug_wait_kernel(uint64_t limit_ns, uint32_t* err) {
 // spread over warps by a grid-stride loop), so no block starts in a second,
 // partial wave.
 template <typename Kernel>
-int grid_for_rows(const DeviceInfo& dev, Kernel kernel, int64_t rows) {
+int grid_for_rows(const DeviceInfo& dev, Kernel kernel, int64_t rows, size_t dynamic_smem = 0) {
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, 0) != cudaSuccess || per_sm < 1) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, dynamic_smem) != cudaSuccess ||
+      per_sm < 1) {
     cudaGetLastError();
     per_sm = 1;
   }
@@ -1665,16 +1707,17 @@ int run_norm_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, con
     }
     return launch_status();
   }
-  if (per_row) {
-    auto k = nvfp4_norm_quant_kernel<Sf128x4, true, kLN>;
-    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, beta, eps, global_sf, rg, ri,
-                                                               row_mean, row_rstd, codes, sf);
-  } else {
-    auto k = nvfp4_norm_quant_kernel<Sf128x4, false, kLN>;
-    k<<<grid_for_rows(dev, k, Mp), kQuantThreads, 0, stream>>>(x, M, Mp, K, ld_x, gamma, beta, eps, global_sf, rg, ri,
-                                                               row_mean, row_rstd, codes, sf);
-  }
-  return launch_status();
+  const size_t stage = norm_stage_bytes(K, kLN);
+  auto launch = [&](auto k, size_t smem) -> int {
+    k<<<grid_for_rows(dev, k, Mp, smem), kQuantThreads, smem, stream>>>(x, M, Mp, K, ld_x, gamma, beta, eps, global_sf,
+                                                                      rg, ri, row_mean, row_rstd, codes, sf);
+    return launch_status();
+  };
+  if (stage <= kNormStageMaxBytes)
+    return per_row ? launch(nvfp4_norm_quant_kernel<Sf128x4, true, kLN, true>, stage)
+                   : launch(nvfp4_norm_quant_kernel<Sf128x4, false, kLN, true>, stage);
+  return per_row ? launch(nvfp4_norm_quant_kernel<Sf128x4, true, kLN, false>, 0)
+                 : launch(nvfp4_norm_quant_kernel<Sf128x4, false, kLN, false>, 0);
 }
 
 }  // namespace
