@@ -142,3 +142,20 @@ def test_matches_torch_layer_norm_within_one_bf16_ulp():
     m_o, v_o = oracle.layernorm_moments(x)
     assert np.all(np.abs(m_o - m64.numpy()) <= np.spacing(np.abs(m_o)))
     assert np.all(np.abs(v_o - v64.numpy()) <= np.spacing(np.abs(v_o)))
+
+
+def test_variance_beyond_fp32_rounds_to_inf_and_rstd_to_zero():
+    # +-2^64 alternating: mean 0, var = 2^128 exactly, above the largest finite
+    # fp32 and past the midpoint to it, so RN32 gives +inf; then rstd =
+    # RN32(1/sqrt(inf)) = 0 and y = ((x - 0) * 0) * 1 + beta = beta
+    x = _bits(np.array([[2.0 ** 64, -(2.0 ** 64)] * 16]))
+    mean, var = oracle.layernorm_moments(x)
+    assert mean[0] == 0.0 and np.isposinf(var[0])
+    m, rstd = oracle.layernorm_stats(x, 1e-6)
+    assert rstd[0] == 0.0
+    beta = _bits(np.linspace(-1, 1, 32))
+    assert (oracle.layernorm_bf16(x, None, beta, m, rstd) == beta).all()
+    # +-255 * 2^56: var = 65025 * 2^112 = 16646400 * 2^104, exact in fp32 (below 2^24 * 2^104)
+    x = _bits(np.array([[255 * 2.0 ** 56, -255 * 2.0 ** 56] * 16]))
+    mean, var = oracle.layernorm_moments(x)
+    assert mean[0] == 0.0 and var[0] == np.float32(16646400 * 2.0 ** 104)
