@@ -67,3 +67,12 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert r0.returncode == 0
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # the contract's keys, and the reference arm's own figures in cpu_baseline and e2e
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["higher_is_better"] is True
+    assert line["config"]["workload"] and line["value"] > 0
+    cb, e2e = line["cpu_baseline"], line["e2e"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"] and e2e["d2h_bytes_per_step"] == 0
